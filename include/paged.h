@@ -1,0 +1,239 @@
+/*
+ * paged.h — C ABI of libpaged: paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * Sources this interface follows (web pages, cited by title and section):
+ *   [P1] "vLLM框架中的KV cache优化与PagedAttention机制详解" (trdm.cn)
+ *   [P2] "vLLM推理引擎架构：PagedAttention机制与高吞吐推理" (maplevalley.com.cn)
+ *   [P3] "Paged KVCache：大模型推理显存管理优化方案" (intelliparadigm.com)
+ *   [P4] "大模型推理KV Cache内存管理与PagedAttention分页显存实战" (yunthe.com)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Device pointers are plain CUDA device addresses owned by the caller; the
+ *    library never allocates, frees or retains device memory. Host pointers are
+ *    read (or written) only during the call.
+ *  - Every device call is asynchronous on `stream` and performs no device
+ *    synchronisation. Argument errors are detected on the host before any
+ *    launch; the call then returns a non-zero status, launches nothing and
+ *    records a message readable with pa_last_error() (thread-local).
+ *  - Launch failures return PA_ERR_CUDA with the CUDA error string.
+ *  - Every device pointer must be 16-byte aligned; rows of head_dim elements
+ *    must be a multiple of 16 bytes (always true for the supported head_dim).
+ *  - Integer tables (block tables, context lengths, slot mappings) are int32.
+ *    All element offsets are formed in 64 bits, so caches larger than 2^31
+ *    elements are fine.
+ *  - Caches are laid out [num_blocks, block_size, num_kv_heads, head_dim]
+ *    ([P2] §2.2 "Block管理器实现"; the per-head dimension is num_kv_heads,
+ *    which equals num_heads for multi-head attention).
+ */
+#ifndef LIBPAGED_PAGED_H
+#define LIBPAGED_PAGED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same ABI as cudaStream_t; NULL is the legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, inconsistent shape */
+  PA_ERR_UNSUPPORTED = 2, /* valid but not implemented: head_dim, block_size, group size, dtype pair */
+  PA_ERR_OOM = 3,         /* host allocator: not enough free blocks (nothing was allocated) */
+  PA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed; see pa_last_error() */
+  PA_ERR_BAD_TABLE = 5    /* a block-table entry, slot or context length is out of range */
+} pa_status;
+
+typedef enum {
+  PA_F16 = 0,      /* IEEE binary16 */
+  PA_BF16 = 1,     /* bfloat16 */
+  PA_FP8_E4M3 = 2  /* OCP FP8 E4M3 (bias 7, max finite 448, no infinities) */
+} pa_dtype;
+
+/* Thread-local description of the last failing call on this thread ("" if none). */
+const char* pa_last_error(void);
+
+/* ------------------------------------------------------------------------- */
+/* reshape_and_cache: scatter one step's new K/V into the paged cache.        */
+/* ------------------------------------------------------------------------- */
+/*
+ * For every token n in [0, num_tokens) with slot = slot_mapping[n] >= 0:
+ *     blk = slot / block_size, off = slot % block_size
+ *     key_cache  [blk][off][h][:] = enc(key  [n][h][:], k_scale[h])
+ *     value_cache[blk][off][h][:] = enc(value[n][h][:], v_scale[h])     for all h
+ * Tokens with a negative slot are skipped (padding). The slot is the physical
+ * address of a token: physical block * block_size + offset inside the block,
+ * the address translation of [P3] §2.3 "地址转换流程" with the page size
+ * counted in tokens ([P4] "Block大小为16"), as in [P1] §5.1.
+ *
+ * key, value      device, [num_tokens, num_kv_heads, head_dim] of kv_dtype (F16 or BF16).
+ * key_cache,      device, [num_blocks, block_size, num_kv_heads, head_dim] of cache_dtype.
+ *   value_cache
+ * slot_mapping    device int32 [num_tokens]; slots must be unique (caller's duty) and
+ *                 < num_blocks * block_size.
+ * cache_dtype     == kv_dtype: the bytes are copied unchanged.
+ *                 == PA_FP8_E4M3: enc(x, s) = e4m3_rne_satfinite((float)x / s), one IEEE
+ *                 fp32 division and one rounding (FP8 KV storage, [P4] "FP8 KV Cache量化").
+ * k_scale,        device fp32 [num_kv_heads] (FP8 cache only; NULL otherwise).
+ *   v_scale
+ * Errors: PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED on the host before launch. A slot
+ * outside the pool is not written (the kernel checks every slot).
+ * head_dim in {64, 128}; block_size in {16, 32}.
+ */
+pa_status pa_reshape_and_cache(const void* key, const void* value,
+                               void* key_cache, void* value_cache,
+                               const int32_t* slot_mapping, int32_t num_tokens,
+                               int32_t num_kv_heads, int32_t head_dim,
+                               int32_t block_size, int64_t num_blocks,
+                               pa_dtype kv_dtype, pa_dtype cache_dtype,
+                               const float* k_scale, const float* v_scale,
+                               pa_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* decode: one query token per sequence against its paged context.            */
+/* ------------------------------------------------------------------------- */
+/*
+ * The kernel of [P2] §2.3 "PagedAttention Kernel": for each sequence s and query
+ * head h, with kvh = h / (num_heads / num_kv_heads) (contiguous query groups) and
+ * n = context_lens[s]:
+ *     K_s[t] = key_cache  [block_tables[s][t / block_size]][t % block_size][kvh][:]
+ *     V_s[t] = value_cache[block_tables[s][t / block_size]][t % block_size][kvh][:]
+ *     out[s][h][:] = sum_t softmax_t(scale * query[s][h]·K_s[t]) * V_s[t],  t < n
+ * i.e. the logical->physical block translation of [P1] §5.1 followed by
+ * attention accumulated across blocks. n == 0 gives an all-zero output row.
+ * For an FP8 cache the stored codes are dequantised as code * k_scale[kvh]
+ * (keys) and code * v_scale[kvh] (values).
+ *
+ * out             device [num_seqs, num_heads, head_dim] of q_dtype (written).
+ * query           device [num_seqs, num_heads, head_dim] of q_dtype (F16 or BF16).
+ * key_cache,      device [num_blocks, block_size, num_kv_heads, head_dim] of cache_dtype
+ *   value_cache   (cache_dtype == q_dtype, or PA_FP8_E4M3).
+ * block_tables    device int32 [num_seqs, max_blocks_per_seq]; entries past
+ *                 ceil(n / block_size) are never read (any value, e.g. -1).
+ * context_lens    device int32 [num_seqs].
+ * max_context_len host int, >= every context_lens[s]; sizes the launch.
+ * scale           softmax scale (e.g. 1/sqrt(head_dim)).
+ * k_scale,        device fp32 [num_kv_heads] for an FP8 cache, else NULL.
+ *   v_scale
+ * partition_tokens 0 = choose automatically; otherwise the context is cut into
+ *                 partitions of this many tokens (a multiple of block_size) that
+ *                 are processed independently and combined by a second kernel.
+ *                 A value >= max_context_len forces the single-pass path.
+ * workspace       device scratch of at least pa_decode_workspace_size(...) bytes,
+ *                 caller-owned, 256-byte aligned. Its first 256 bytes hold an error
+ *                 word (see pa_decode_check); the rest holds per-partition partial
+ *                 results. Two calls in flight at once must not share it.
+ * Supported: head_dim in {64, 128}; block_size in {16, 32};
+ *            num_heads / num_kv_heads in {1, 2, 4, 8}.
+ * Run-time table errors (an entry outside [0, num_blocks), a context length above
+ * max_context_len or above max_blocks_per_seq * block_size) never cause an
+ * out-of-range access: the offending block reads as zeros, the context is
+ * clipped, and the error word is set for pa_decode_check to report.
+ */
+pa_status pa_decode(void* out, const void* query,
+                    const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t max_context_len,
+                    int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                    float scale, pa_dtype q_dtype, pa_dtype cache_dtype,
+                    const float* k_scale, const float* v_scale,
+                    int32_t partition_tokens,
+                    void* workspace, size_t workspace_bytes,
+                    pa_stream_t stream);
+
+/*
+ * Bytes of workspace pa_decode needs for these sizes on the current device
+ * (the automatic partition choice depends on the device's SM count).
+ * Returns 0 for invalid sizes.
+ */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t block_size,
+                                int32_t max_context_len, int32_t partition_tokens);
+
+/*
+ * The partition length (tokens) pa_decode will use for these sizes on the
+ * current device; a result >= max_context_len means the single-pass path.
+ */
+int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                   int32_t head_dim, int32_t block_size,
+                                   int32_t max_context_len, int32_t partition_tokens);
+
+/*
+ * Synchronises `stream`, reads and clears the error word of `workspace`.
+ * Returns PA_OK, or PA_ERR_BAD_TABLE if a previous pa_decode on this workspace
+ * met an out-of-range table entry or context length, or PA_ERR_CUDA.
+ */
+pa_status pa_decode_check(void* workspace, pa_stream_t stream);
+
+/*
+ * Zero the error word of a fresh workspace (asynchronous on `stream`).
+ * pa_decode never needs the rest of the workspace cleared.
+ */
+pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Host block allocator (no device memory; produces integer tables only).      */
+/* ------------------------------------------------------------------------- */
+/*
+ * The free list of [P2] §2.2 "Block管理器实现": allocate(n) takes the first n
+ * free ids or fails with PA_ERR_OOM leaving the list untouched; free appends
+ * released ids to the back. Blocks shared by several sequences (shared
+ * prompt prefix) carry a reference count ([P4] "通过引用计数管理生命周期"):
+ * share() adds a reference, free() drops one, and a block returns to the
+ * free list when its count reaches zero.
+ */
+typedef struct pa_alloc pa_alloc;
+
+/* initial_free_order: NULL for 0..num_blocks-1, else a permutation of it (e.g. a
+ * seeded shuffle) that becomes the initial free list, front first. */
+pa_status pa_alloc_create(int64_t num_blocks, const int32_t* initial_free_order, pa_alloc** out);
+void pa_alloc_destroy(pa_alloc* a);
+/* All-or-nothing: on PA_ERR_OOM nothing changes. n == 0 is a no-op. */
+pa_status pa_alloc_allocate(pa_alloc* a, int32_t n, int32_t* ids_out);
+/* refcount++ of an allocated block; PA_ERR_INVALID_ARG if the block is free. */
+pa_status pa_alloc_share(pa_alloc* a, int32_t id);
+/* refcount-- of each id, in order; all ids are validated first (an id that is
+ * free or listed more often than its refcount gives PA_ERR_INVALID_ARG and
+ * changes nothing). */
+pa_status pa_alloc_free(pa_alloc* a, const int32_t* ids, int32_t n);
+int64_t pa_alloc_num_free(const pa_alloc* a);
+int64_t pa_alloc_num_blocks(const pa_alloc* a);
+/* Reference count of a block (0 = free), -1 for an id out of range. */
+int32_t pa_alloc_refcount(const pa_alloc* a, int32_t id);
+/* Copy the free list, front first, into ids_out (capacity cap); returns the
+ * number of free blocks. */
+int64_t pa_alloc_free_list(const pa_alloc* a, int32_t* ids_out, int64_t cap);
+
+/*
+ * Row-major block table [num_seqs, max_blocks_per_seq] from per-sequence id
+ * lists; unused entries are set to -1. PA_ERR_INVALID_ARG if a list is longer
+ * than max_blocks_per_seq.
+ */
+pa_status pa_build_block_table(const int32_t* const* seq_block_ids,
+                               const int32_t* num_blocks_per_seq, int32_t num_seqs,
+                               int32_t max_blocks_per_seq, int32_t* table_out);
+
+/*
+ * slots_out[i] = block_tables[seq][pos / block_size] * block_size + pos % block_size
+ * with seq = seq_ids ? seq_ids[i] : i and pos = positions[i] ([P3] §2.3 address
+ * translation, page size in tokens). pos < 0 gives slot -1 (padding token).
+ * PA_ERR_BAD_TABLE if pos / block_size >= max_blocks_per_seq, the table entry is
+ * negative, or the slot does not fit in int32; slots_out is then unspecified.
+ * All arrays are host memory.
+ */
+pa_status pa_build_slot_mapping(const int32_t* block_tables, int32_t num_seqs,
+                                int32_t max_blocks_per_seq, const int32_t* seq_ids,
+                                const int32_t* positions, int32_t num_tokens,
+                                int32_t block_size, int32_t* slots_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBPAGED_PAGED_H */
