@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode step of a LLaMA-7B-shaped layer (32 sequences x 2048
+context tokens, 32 heads, head_dim 128, block_size 16, fp16 K/V, pool of
+32*128+256 shuffled blocks): reshape_and_cache of the step's 32 new tokens
+into their slots, then paged decode attention over the whole context.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...     (one process per GPU)
+
+Multi-GPU: every rank runs its own batch on its own GPU (sequences are
+independent; no collective on the data path): weak scaling, value = bytes of
+all ranks / max-over-ranks device time.
+
+Rank 0 prints one JSON line. `value` is KV-read GB/s: the decode's
+algorithmic bytes (K/V rows read once per kv-head + query + output + block
+table entries + context lengths) per step over the device time of the step.
+`--impl reference` times the CPU oracle (plain fp64 C) on the host cores
+instead, on a sample of the same workload sized so the run ends in minutes.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_448_b200 import workloads as wl  # noqa: E402
+
+METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode tokens/s per layer"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2, help="workload 1..5 (2 = headline)")
+    ap.add_argument("--partition", type=int, default=-1,
+                    help="decode partition tokens (-1: the workload's setting, 0: automatic)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU time budget of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def sources_digest() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_448_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel sources and this workload; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f).get("decode", {})
+    if j.get("sources_sha256") != sources_digest() or j.get("workload") != workload:
+        return None
+    return j.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception as e:  # no nvidia-smi: clocks unknown
+            log("clock sampler unavailable:", e)
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def workload_name(sp: wl.Spec, st: wl.Structure) -> str:
+    ctx = sp.context_lens
+    ctxs = f"ctx {int(ctx[0])}" if ctx.min() == ctx.max() else f"ctx {int(ctx.min())}-{int(ctx.max())}"
+    return (f"{sp.name}: {sp.num_seqs} seqs, {ctxs}, {sp.num_heads} q / {sp.num_kv_heads} kv heads, "
+            f"head_dim {sp.head_dim}, block_size {sp.block_size}, q {sp.q_dtype}, "
+            f"KV {sp.cache_dtype}, pool {st.num_blocks} shuffled blocks")
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(sp: wl.Spec, seqs: int, heads: int):
+    """A sub-workload of the same shape (first `seqs` sequences, `heads` kv-heads
+    and their query groups) with its host inputs, for timing the oracle."""
+    g = sp.num_heads // sp.num_kv_heads
+    sub = dataclasses.replace(sp, num_seqs=seqs, context_lens=sp.context_lens[:seqs].copy(),
+                              num_kv_heads=heads, num_heads=heads * g, spare_blocks=0)
+    st = wl.structure(sub)
+    return sub, st, wl.host_data(sub, st)
+
+
+def time_oracle(sub, st, hd) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.decode(hd.query, hd.key_cache, hd.value_cache, st.block_tables, sub.context_lens,
+                  scale=np.float32(sub.scale), q_dtype=sub.q_dtype, cache_dtype=sub.cache_dtype,
+                  k_scale=hd.k_scale, v_scale=hd.v_scale)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(sp: wl.Spec, budget_s: float) -> dict:
+    """The oracle as it stands (single-threaded C, fp64) on a bounded sample."""
+    import oracle
+    oracle.build()
+    one = oracle_sample(sp, 1, sp.num_kv_heads)
+    t1 = time_oracle(*one)
+    seqs = int(max(1, min(sp.num_seqs, budget_s // max(t1, 1e-3))))
+    sub = oracle_sample(sp, seqs, sp.num_kv_heads)
+    t = time_oracle(*sub)
+    gb = wl.decode_bytes(sub[0], sub[1]) / 1e9
+    return {"value": round(gb / t, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {seqs} of {sp.num_seqs} sequences of the same workload "
+                      f"(all {sp.num_heads} heads, full contexts); {t:.1f} s single-threaded fp64 C",
+            "tokens_per_s_per_layer": round(seqs / t, 3)}
+
+
+def run_reference(args, sp, st):
+    """--impl reference: the oracle on the host cores, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    budget = 150.0
+    per_step = budget / max(1, args.steps + args.warmup)
+    one_head = oracle_sample(sp, 1, 1)
+    t_pair = time_oracle(*one_head)
+    pairs_total = sp.num_seqs * sp.num_kv_heads
+    pairs = int(max(1, min(pairs_total, per_step // max(t_pair, 1e-4))))
+    if pairs >= sp.num_kv_heads:
+        seqs, heads = max(1, pairs // sp.num_kv_heads), sp.num_kv_heads
+    else:
+        seqs, heads = 1, pairs
+    sub = oracle_sample(sp, seqs, heads)
+    for _ in range(args.warmup):
+        time_oracle(*sub)
+    t = sum(time_oracle(*sub) for _ in range(args.steps))
+    gb = wl.decode_bytes(sub[0], sub[1]) / 1e9 * args.steps
+    value = gb / t
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_name(sp, st), "global_batch": sp.num_seqs,
+                       "seq_len": int(sp.context_lens.max()), "parallelism": "none (host CPU)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"each step: {seqs} sequence(s) x {heads} kv-head(s) of "
+                                       f"the workload, full context, single-threaded fp64 C"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def main():
+    args = parse()
+    sp = wl.spec(args.config)
+    st = wl.structure(sp)
+    if args.impl == "reference":
+        run_reference(args, sp, st)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import paged_kv_cache_448_b200 as pk
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    part = sp.partition_tokens if args.partition < 0 else args.partition
+    sp_r = dataclasses.replace(sp, seed=sp.seed + 97 * rank)
+    d = wl.device_data(sp_r, st, device=dev)
+    slots = pk.build_slot_mapping(st.block_tables, st.positions, sp.block_size)
+    bt = torch.from_numpy(st.block_tables).to(dev)
+    cl = torch.from_numpy(sp.context_lens).to(dev)
+    sl = torch.from_numpy(slots).to(dev)
+    out = torch.empty_like(d["query"])
+    max_ctx = int(sp.context_lens.max())
+    ws = pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                             sp.block_size, max_ctx, part, device=dev)
+    eff_part = pk.decode_partition_tokens(sp.num_seqs, sp.num_heads, sp.num_kv_heads,
+                                          sp.head_dim, sp.block_size, max_ctx, part)
+    split = eff_part < max_ctx
+    launches_per_step = 2 + (1 if split else 0)
+
+    def step(q, nk, nv, btab, ctx, slot, o, ev=None):
+        pk.reshape_and_cache(nk, nv, d["key_cache"], d["value_cache"], slot,
+                             k_scale=d["k_scale"], v_scale=d["v_scale"])
+        if ev is not None:
+            ev[0].record()
+        pk.decode(o, q, d["key_cache"], d["value_cache"], btab, ctx, max_ctx, sp.scale,
+                  k_scale=d["k_scale"], v_scale=d["v_scale"], partition_tokens=part,
+                  workspace=ws)
+        if ev is not None:
+            ev[1].record()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(d["query"], d["new_key"], d["new_value"], bt, cl, sl, out)
+    torch.cuda.synchronize()
+    pk.decode_check(ws)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0.record()
+    for k in range(args.steps):
+        step(d["query"], d["new_key"], d["new_value"], bt, cl, sl, out, evs[k])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    pk.decode_check(ws)
+
+    # e2e: the same step through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = {k: d[k].cpu().pin_memory() for k in ("query", "new_key", "new_value")}
+        pin["bt"] = torch.from_numpy(st.block_tables).pin_memory()
+        pin["cl"] = torch.from_numpy(sp.context_lens).pin_memory()
+        pin["sl"] = torch.from_numpy(slots).pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dq, dnk, dnv = (torch.empty_like(d[k]) for k in ("query", "new_key", "new_value"))
+        dbt, dcl, dsl = torch.empty_like(bt), torch.empty_like(cl), torch.empty_like(sl)
+        h2d = sum(t.numel() * t.element_size() for t in pin.values())
+        d2h = out_h.numel() * out_h.element_size()
+        e2e_steps = max(1, min(args.steps, 2000))
+
+        def e2e_step():
+            dq.copy_(pin["query"], non_blocking=True)
+            dnk.copy_(pin["new_key"], non_blocking=True)
+            dnv.copy_(pin["new_value"], non_blocking=True)
+            dbt.copy_(pin["bt"], non_blocking=True)
+            dcl.copy_(pin["cl"], non_blocking=True)
+            dsl.copy_(pin["sl"], non_blocking=True)
+            step(dq, dnk, dnv, dbt, dcl, dsl, out)
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = a.elapsed_time(b) / e2e_steps
+        e2e = {"ms_per_step": e2e_ms, "h2d": h2d, "d2h": d2h}
+
+    # max over ranks
+    step_ms = elapsed_ms / args.steps
+    vals = torch.tensor([step_ms, dec_ms, e2e["ms_per_step"] if e2e else 0.0],
+                        dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    step_ms, dec_ms, e2e_ms = vals.tolist()
+
+    if rank == 0:
+        dbytes = wl.decode_bytes(sp, st)
+        peak, peak_kind = measured_peaks()
+        value = world * dbytes / (step_ms * 1e-3) / 1e9
+        achieved = dbytes / (dec_ms * 1e-3) / 1e9
+        traffic = recorded_traffic(sp.name)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": sp.cache_dtype, "data": "synthetic",
+            "config": {"workload": workload_name(sp, st), "global_batch": sp.num_seqs * world,
+                       "seq_len": max_ctx, "parallelism": f"dp{world}",
+                       "partition_tokens": eff_part if split else None,
+                       "l2": f"inputs larger than L2: {wl.kv_bytes(sp) / 1e9:.2f} GB of K/V "
+                             "per step vs 126 MB L2; no flush"},
+            "pct_of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+            "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+            "tokens_per_s_per_layer": round(world * sp.num_seqs / (step_ms * 1e-3), 1),
+            "roofline": {"bound": "hbm", "kernel": "pa_decode (decode" +
+                         (" + partition combine)" if split else ")"),
+                         "achieved": round(achieved, 2), "peak": peak,
+                         "peak_kind": f"{peak_kind} HBM copy GB/s", "unit": "GB/s",
+                         "frac": round(achieved / peak, 4),
+                         "traffic": traffic,
+                         "algorithmic_bytes_per_launch": dbytes,
+                         "launch_ms": round(dec_ms, 5)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if e2e:
+            line["e2e"] = {"value": round(world * dbytes / (e2e_ms * 1e-3) / 1e9, 2),
+                           "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
+                           "d2h_bytes_per_step": e2e["d2h"],
+                           "ms_per_step": round(e2e_ms, 5)}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(sp, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -32,6 +32,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -56,7 +62,7 @@ typedef enum {
 } pa_dtype;
 
 /* Thread-local description of the last failing call on this thread ("" if none). */
-const char* pa_last_error(void);
+PA_API const char* pa_last_error(void);
 
 /* ------------------------------------------------------------------------- */
 /* reshape_and_cache: scatter one step's new K/V into the paged cache.        */
@@ -85,7 +91,7 @@ const char* pa_last_error(void);
  * outside the pool is not written (the kernel checks every slot).
  * head_dim in {64, 128}; block_size in {16, 32}.
  */
-pa_status pa_reshape_and_cache(const void* key, const void* value,
+PA_API pa_status pa_reshape_and_cache(const void* key, const void* value,
                                void* key_cache, void* value_cache,
                                const int32_t* slot_mapping, int32_t num_tokens,
                                int32_t num_kv_heads, int32_t head_dim,
@@ -135,7 +141,7 @@ pa_status pa_reshape_and_cache(const void* key, const void* value,
  * out-of-range access: the offending block reads as zeros, the context is
  * clipped, and the error word is set for pa_decode_check to report.
  */
-pa_status pa_decode(void* out, const void* query,
+PA_API pa_status pa_decode(void* out, const void* query,
                     const void* key_cache, const void* value_cache,
                     const int32_t* block_tables, int32_t max_blocks_per_seq,
                     const int32_t* context_lens, int32_t max_context_len,
@@ -152,7 +158,7 @@ pa_status pa_decode(void* out, const void* query,
  * (the automatic partition choice depends on the device's SM count).
  * Returns 0 for invalid sizes.
  */
-size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                 int32_t head_dim, int32_t block_size,
                                 int32_t max_context_len, int32_t partition_tokens);
 
@@ -160,7 +166,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
  * The partition length (tokens) pa_decode will use for these sizes on the
  * current device; a result >= max_context_len means the single-pass path.
  */
-int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+PA_API int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                    int32_t head_dim, int32_t block_size,
                                    int32_t max_context_len, int32_t partition_tokens);
 
@@ -169,13 +175,13 @@ int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads, int32_t 
  * Returns PA_OK, or PA_ERR_BAD_TABLE if a previous pa_decode on this workspace
  * met an out-of-range table entry or context length, or PA_ERR_CUDA.
  */
-pa_status pa_decode_check(void* workspace, pa_stream_t stream);
+PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream);
 
 /*
  * Zero the error word of a fresh workspace (asynchronous on `stream`).
  * pa_decode never needs the rest of the workspace cleared.
  */
-pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_stream_t stream);
+PA_API pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_stream_t stream);
 
 /* ------------------------------------------------------------------------- */
 /* Host block allocator (no device memory; produces integer tables only).      */
@@ -192,30 +198,30 @@ typedef struct pa_alloc pa_alloc;
 
 /* initial_free_order: NULL for 0..num_blocks-1, else a permutation of it (e.g. a
  * seeded shuffle) that becomes the initial free list, front first. */
-pa_status pa_alloc_create(int64_t num_blocks, const int32_t* initial_free_order, pa_alloc** out);
-void pa_alloc_destroy(pa_alloc* a);
+PA_API pa_status pa_alloc_create(int64_t num_blocks, const int32_t* initial_free_order, pa_alloc** out);
+PA_API void pa_alloc_destroy(pa_alloc* a);
 /* All-or-nothing: on PA_ERR_OOM nothing changes. n == 0 is a no-op. */
-pa_status pa_alloc_allocate(pa_alloc* a, int32_t n, int32_t* ids_out);
+PA_API pa_status pa_alloc_allocate(pa_alloc* a, int32_t n, int32_t* ids_out);
 /* refcount++ of an allocated block; PA_ERR_INVALID_ARG if the block is free. */
-pa_status pa_alloc_share(pa_alloc* a, int32_t id);
+PA_API pa_status pa_alloc_share(pa_alloc* a, int32_t id);
 /* refcount-- of each id, in order; all ids are validated first (an id that is
  * free or listed more often than its refcount gives PA_ERR_INVALID_ARG and
  * changes nothing). */
-pa_status pa_alloc_free(pa_alloc* a, const int32_t* ids, int32_t n);
-int64_t pa_alloc_num_free(const pa_alloc* a);
-int64_t pa_alloc_num_blocks(const pa_alloc* a);
+PA_API pa_status pa_alloc_free(pa_alloc* a, const int32_t* ids, int32_t n);
+PA_API int64_t pa_alloc_num_free(const pa_alloc* a);
+PA_API int64_t pa_alloc_num_blocks(const pa_alloc* a);
 /* Reference count of a block (0 = free), -1 for an id out of range. */
-int32_t pa_alloc_refcount(const pa_alloc* a, int32_t id);
+PA_API int32_t pa_alloc_refcount(const pa_alloc* a, int32_t id);
 /* Copy the free list, front first, into ids_out (capacity cap); returns the
  * number of free blocks. */
-int64_t pa_alloc_free_list(const pa_alloc* a, int32_t* ids_out, int64_t cap);
+PA_API int64_t pa_alloc_free_list(const pa_alloc* a, int32_t* ids_out, int64_t cap);
 
 /*
  * Row-major block table [num_seqs, max_blocks_per_seq] from per-sequence id
  * lists; unused entries are set to -1. PA_ERR_INVALID_ARG if a list is longer
  * than max_blocks_per_seq.
  */
-pa_status pa_build_block_table(const int32_t* const* seq_block_ids,
+PA_API pa_status pa_build_block_table(const int32_t* const* seq_block_ids,
                                const int32_t* num_blocks_per_seq, int32_t num_seqs,
                                int32_t max_blocks_per_seq, int32_t* table_out);
 
@@ -227,7 +233,7 @@ pa_status pa_build_block_table(const int32_t* const* seq_block_ids,
  * negative, or the slot does not fit in int32; slots_out is then unspecified.
  * All arrays are host memory.
  */
-pa_status pa_build_slot_mapping(const int32_t* block_tables, int32_t num_seqs,
+PA_API pa_status pa_build_slot_mapping(const int32_t* block_tables, int32_t num_seqs,
                                 int32_t max_blocks_per_seq, const int32_t* seq_ids,
                                 const int32_t* positions, int32_t num_tokens,
                                 int32_t block_size, int32_t* slots_out);

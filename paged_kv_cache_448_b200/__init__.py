@@ -1,4 +1,189 @@
-"""libpaged: paged KV-cache decode attention for B200 (sm_100a), Python binding.
+"""libpaged: paged KV-cache decode attention for B200 (sm_100a) — Python binding.
 
-Placeholder until the binding lands.
+Every op here marshals arguments into one call of the C ABI in
+``include/paged.h`` (``libpaged.so``, built in-tree); all compute runs in the
+library's CUDA kernels. PyTorch supplies device memory and the current stream
+only. If the library is missing the first op raises ``ImportError``.
+
+Ops:
+  * ``reshape_and_cache`` — scatter a step's new K/V rows into cache slots.
+  * ``decode`` — paged attention of one query token per sequence.
+  * ``BlockAllocator``, ``build_block_table``, ``build_slot_mapping`` — host
+    allocator and integer-table builders (no GPU).
 """
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import _native
+from ._native import PagedError, check
+
+__all__ = ["reshape_and_cache", "decode", "decode_workspace", "decode_workspace_size",
+           "decode_partition_tokens", "decode_check", "BlockAllocator", "build_block_table",
+           "build_slot_mapping", "PagedError", "dtype_code"]
+
+
+def dtype_code(t) -> int:
+    """pa_dtype of a torch tensor (uint8 / float8_e4m3fn storage is E4M3)."""
+    import torch
+    if t.dtype == torch.float16:
+        return _native.PA_F16
+    if t.dtype == torch.bfloat16:
+        return _native.PA_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return _native.PA_FP8_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_handle(stream) -> int | None:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, *, k_scale=None,
+                      v_scale=None, stream=None) -> None:
+    """key/value [T, Hkv, D] f16|bf16; caches [NB, BS, Hkv, D] (same dtype, or uint8 E4M3
+    with fp32 k_scale/v_scale [Hkv]); slot_mapping int32 [T] (negative = skip)."""
+    T, Hkv, D = key.shape
+    NB, BS = key_cache.shape[:2]
+    check(_native.lib().pa_reshape_and_cache(
+        _ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(slot_mapping), T, Hkv,
+        D, BS, NB, dtype_code(key), dtype_code(key_cache), _ptr(k_scale), _ptr(v_scale),
+        _stream_handle(stream)))
+
+
+def decode_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_context_len, partition_tokens=0) -> int:
+    return int(_native.lib().pa_decode_partition_tokens(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+        partition_tokens))
+
+
+def decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                          max_context_len, partition_tokens=0) -> int:
+    return int(_native.lib().pa_decode_workspace_size(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+        partition_tokens))
+
+
+def decode_workspace(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                     partition_tokens=0, device="cuda", stream=None):
+    """A device workspace (torch uint8) of the size pa_decode needs, error word zeroed."""
+    import torch
+    n = decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                              max_context_len, partition_tokens)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    check(_native.lib().pa_workspace_init(_ptr(ws), ws.numel(), _stream_handle(stream)))
+    return ws
+
+
+def decode(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
+           scale: float, *, k_scale=None, v_scale=None, partition_tokens: int = 0,
+           workspace=None, stream=None):
+    """out/query [S, H, D] f16|bf16; caches [NB, BS, Hkv, D]; block_tables int32
+    [S, max_blocks]; context_lens int32 [S]; max_context_len >= every context length.
+    Returns ``out``."""
+    S, H, D = query.shape
+    NB, BS, Hkv = key_cache.shape[:3]
+    if workspace is None:
+        workspace = decode_workspace(S, H, Hkv, D, BS, max_context_len, partition_tokens,
+                                     device=query.device, stream=stream)
+    check(_native.lib().pa_decode(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, H, Hkv, D, BS, NB,
+        float(scale), dtype_code(query), dtype_code(key_cache), _ptr(k_scale), _ptr(v_scale),
+        int(partition_tokens), _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+    return out
+
+
+def decode_check(workspace, stream=None) -> None:
+    """Synchronise and raise PagedError if a decode on `workspace` met a bad table entry."""
+    check(_native.lib().pa_decode_check(_ptr(workspace), _stream_handle(stream)))
+
+
+# ---------------------------------------------------------------- host side
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+class BlockAllocator:
+    """Host free list with refcounts (pa_alloc_*)."""
+
+    def __init__(self, num_blocks: int, initial_free_order=None):
+        self._lib = _native.lib()
+        order = None if initial_free_order is None else _i32(initial_free_order)
+        h = ctypes.c_void_p()
+        check(self._lib.pa_alloc_create(num_blocks, None if order is None else order.ctypes.data,
+                                        ctypes.byref(h)))
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.pa_alloc_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def allocate(self, n: int) -> list:
+        ids = np.empty(max(n, 1), np.int32)
+        check(self._lib.pa_alloc_allocate(self._h, n, ids.ctypes.data))
+        return [int(i) for i in ids[:n]]
+
+    def share(self, block_id: int) -> None:
+        check(self._lib.pa_alloc_share(self._h, int(block_id)))
+
+    def free(self, ids) -> None:
+        a = _i32(ids)
+        check(self._lib.pa_alloc_free(self._h, a.ctypes.data if a.size else None, a.size))
+
+    @property
+    def num_free(self) -> int:
+        return int(self._lib.pa_alloc_num_free(self._h))
+
+    @property
+    def num_blocks(self) -> int:
+        return int(self._lib.pa_alloc_num_blocks(self._h))
+
+    def refcount(self, block_id: int) -> int:
+        return int(self._lib.pa_alloc_refcount(self._h, int(block_id)))
+
+    def free_list(self) -> list:
+        n = self.num_free
+        out = np.empty(max(n, 1), np.int32)
+        self._lib.pa_alloc_free_list(self._h, out.ctypes.data, n)
+        return [int(i) for i in out[:n]]
+
+
+def build_block_table(seq_block_ids, max_blocks_per_seq: int) -> np.ndarray:
+    """int32 [S, max_blocks_per_seq] from per-sequence id lists; unused = -1."""
+    rows = [_i32(ids) for ids in seq_block_ids]
+    S = len(rows)
+    ptrs = (ctypes.c_void_p * max(S, 1))(*[r.ctypes.data if r.size else None for r in rows])
+    counts = _i32([r.size for r in rows]) if S else np.zeros(1, np.int32)
+    out = np.empty((max(S, 1), max_blocks_per_seq), np.int32)
+    check(_native.lib().pa_build_block_table(ctypes.cast(ptrs, ctypes.c_void_p),
+                                             counts.ctypes.data, S, max_blocks_per_seq,
+                                             out.ctypes.data))
+    return out[:S]
+
+
+def build_slot_mapping(block_tables, positions, block_size: int, seq_ids=None) -> np.ndarray:
+    """int32 slots for (sequence, position) pairs; position < 0 gives -1."""
+    bt = _i32(block_tables)
+    pos = _i32(positions)
+    sid = None if seq_ids is None else _i32(seq_ids)
+    out = np.empty(max(pos.size, 1), np.int32)
+    check(_native.lib().pa_build_slot_mapping(bt.ctypes.data, bt.shape[0], bt.shape[1],
+                                              None if sid is None else sid.ctypes.data,
+                                              pos.ctypes.data, pos.size, block_size,
+                                              out.ctypes.data))
+    return out[:pos.size]

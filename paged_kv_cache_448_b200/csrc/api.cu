@@ -1,0 +1,319 @@
+// api.cu — the C ABI of libpaged's device calls: argument validation on the
+// host, the launch plan (single pass or context partitions + combine), TMA
+// descriptors for the cache, and the kernel launches. No device memory is
+// allocated here; the caller owns every buffer.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "decode_args.h"
+#include "paged.h"
+#include "status.h"
+
+namespace paged {
+namespace {
+
+constexpr size_t kHeaderBytes = 256;          // error word + padding
+constexpr int32_t kMaxPartitionBlocks = 1024; // block ids staged in shared memory per CTA
+constexpr int32_t kMinAutoPartition = 256;    // tokens
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) dev = 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a cache viewed as [num_blocks*block_size rows][num_kv_heads][head_dim]
+// with a box of one kv-head's block_size rows and <=128 bytes of each row.
+pa_status encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks,
+                           int32_t block_size, int32_t hkv, int32_t head_dim, int elem) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int row_bytes = head_dim * elem;
+  const int bb = box_bytes(row_bytes);
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(hkv),
+                        static_cast<cuuint64_t>(num_blocks) * block_size};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes),
+                           static_cast<cuuint64_t>(row_bytes) * hkv};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(bb / elem), 1u,
+                       static_cast<cuuint32_t>(block_size)};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapSwizzle swz = bb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                               : bb == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                                           : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = enc(map, elem == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                   3, const_cast<void*>(cache), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return PA_OK;
+}
+
+pa_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return PA_OK;
+  if (e == cudaErrorNotSupported)
+    return fail(PA_ERR_UNSUPPORTED, "%s: no kernel for this shape", what);
+  return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int elem_bytes(pa_dtype t) { return t == PA_FP8_E4M3 ? 1 : 2; }
+
+// Launch plan shared by pa_decode and the sizing queries.
+struct Plan {
+  int32_t partition_tokens;  // tokens per partition
+  int32_t partition_blocks;
+  int32_t max_parts;         // 1 = single pass
+};
+
+Plan make_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
+               int32_t max_context_len, int32_t requested) {
+  const int32_t blocks_max = std::max<int32_t>(1, (max_context_len + block_size - 1) / block_size);
+  Plan p{};
+  int32_t pb;
+  if (requested > 0) {
+    pb = (requested + block_size - 1) / block_size;
+  } else {
+    // Enough independent work units to fill every SM several times over;
+    // otherwise cut the context into partitions (>= 256 tokens each).
+    const int64_t pairs = static_cast<int64_t>(num_seqs) * num_kv_heads;
+    const int64_t want = 4LL * sm_count() * 3;
+    pb = blocks_max;
+    if (pairs < want && static_cast<int64_t>(blocks_max) * block_size > kMinAutoPartition) {
+      const int32_t min_pb = std::max(1, kMinAutoPartition / block_size);
+      pb = min_pb;
+      // largest power-of-two multiple of the minimum that still gives `want` units
+      for (int32_t cand = min_pb; cand < blocks_max; cand *= 2) {
+        const int64_t units = pairs * ((blocks_max + cand - 1) / cand);
+        if (units >= want) pb = cand;
+      }
+    }
+  }
+  pb = std::min(std::max(pb, 1), std::min(blocks_max, kMaxPartitionBlocks));
+  p.partition_blocks = pb;
+  p.partition_tokens = pb * block_size;
+  p.max_parts = (blocks_max + pb - 1) / pb;
+  return p;
+}
+
+size_t workspace_bytes_for(const Plan& p, int32_t num_seqs, int32_t num_heads, int32_t head_dim) {
+  if (p.max_parts <= 1) return kHeaderBytes;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_heads * p.max_parts;
+  const size_t ml = (rows * sizeof(float2) + 255) & ~size_t(255);
+  return kHeaderBytes + ml + rows * head_dim * sizeof(float);
+}
+
+bool shape_supported(int32_t head_dim, int32_t block_size) {
+  return (head_dim == 64 || head_dim == 128) && (block_size == 16 || block_size == 32);
+}
+
+}  // namespace
+}  // namespace paged
+
+using namespace paged;
+
+extern "C" {
+
+PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
+                                      void* value_cache, const int32_t* slot_mapping,
+                                      int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t block_size, int64_t num_blocks, pa_dtype kv_dtype,
+                                      pa_dtype cache_dtype, const float* k_scale,
+                                      const float* v_scale, pa_stream_t stream) {
+  clear_error();
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: negative or zero size");
+  if (!shape_supported(head_dim, block_size))
+    return fail(PA_ERR_UNSUPPORTED, "reshape_and_cache: head_dim %d / block_size %d unsupported",
+                head_dim, block_size);
+  if (kv_dtype != PA_F16 && kv_dtype != PA_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "reshape_and_cache: new K/V must be f16 or bf16");
+  if (cache_dtype != kv_dtype && cache_dtype != PA_FP8_E4M3)
+    return fail(PA_ERR_UNSUPPORTED, "reshape_and_cache: cache dtype must equal kv dtype or be e4m3");
+  const bool fp8 = cache_dtype == PA_FP8_E4M3;
+  if (fp8 != (k_scale != nullptr) || fp8 != (v_scale != nullptr))
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: k_scale/v_scale required exactly for e4m3");
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping)
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: null pointer");
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(key_cache, 16) ||
+      !aligned(value_cache, 16) || !aligned(slot_mapping, 4) || (k_scale && !aligned(k_scale, 4)) ||
+      (v_scale && !aligned(v_scale, 4)))
+    return fail(PA_ERR_INVALID_ARG, "reshape_and_cache: misaligned pointer");
+  cudaError_t e = launch_reshape_and_cache(
+      key, value, key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
+      block_size, num_blocks, kv_dtype, cache_dtype, k_scale, v_scale, nullptr,
+      reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e, "reshape_and_cache");
+}
+
+PA_API int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads,
+                                          int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t block_size, int32_t max_context_len,
+                                          int32_t partition_tokens) {
+  (void)num_heads;
+  (void)head_dim;
+  if (num_seqs < 0 || num_kv_heads <= 0 || block_size <= 0 || max_context_len < 0) return 0;
+  Plan p = make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
+  return p.max_parts <= 1 ? std::max(p.partition_tokens, max_context_len) : p.partition_tokens;
+}
+
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t block_size,
+                                       int32_t max_context_len, int32_t partition_tokens) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_context_len < 0)
+    return 0;
+  Plan p = make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
+  return workspace_bytes_for(p, num_seqs, num_heads, head_dim);
+}
+
+PA_API pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+  clear_error();
+  if (!workspace || workspace_bytes < kHeaderBytes || !aligned(workspace, 256))
+    return fail(PA_ERR_INVALID_ARG, "workspace_init: need >= 256 bytes, 256-byte aligned");
+  return cuda_status(
+      cudaMemsetAsync(workspace, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)),
+      "workspace_init");
+}
+
+PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream) {
+  clear_error();
+  if (!workspace) return fail(PA_ERR_INVALID_ARG, "decode_check: null workspace");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && word != 0) e = cudaMemset(workspace, 0, sizeof(word));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode_check: %s", cudaGetErrorString(e));
+  if (word & kErrWaitTimeout) return fail(PA_ERR_CUDA, "decode: a pipeline wait timed out");
+  if (word & (kErrBadBlockId | kErrContextClipped))
+    return fail(PA_ERR_BAD_TABLE, "decode: %s%s",
+                (word & kErrBadBlockId) ? "block-table entry outside the pool; " : "",
+                (word & kErrContextClipped) ? "context length beyond the launch; clipped" : "");
+  return PA_OK;
+}
+
+PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
+                           const void* value_cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* context_lens,
+                           int32_t max_context_len, int32_t num_seqs, int32_t num_heads,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                           int64_t num_blocks, float scale, pa_dtype q_dtype,
+                           pa_dtype cache_dtype, const float* k_scale, const float* v_scale,
+                           int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                           pa_stream_t stream) {
+  clear_error();
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
+      max_context_len < 0 || num_blocks <= 0 || partition_tokens < 0)
+    return fail(PA_ERR_INVALID_ARG, "decode: negative or zero size");
+  if (num_heads % num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "decode: num_heads %% num_kv_heads != 0");
+  const int32_t group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return fail(PA_ERR_UNSUPPORTED, "decode: query group %d not in {1,2,4,8}", group);
+  if (!shape_supported(head_dim, block_size))
+    return fail(PA_ERR_UNSUPPORTED, "decode: head_dim %d / block_size %d unsupported", head_dim,
+                block_size);
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "decode: query must be f16 or bf16");
+  if (cache_dtype != q_dtype && cache_dtype != PA_FP8_E4M3)
+    return fail(PA_ERR_UNSUPPORTED, "decode: cache dtype must equal query dtype or be e4m3");
+  const bool fp8 = cache_dtype == PA_FP8_E4M3;
+  if (fp8 != (k_scale != nullptr) || fp8 != (v_scale != nullptr))
+    return fail(PA_ERR_INVALID_ARG, "decode: k_scale/v_scale required exactly for e4m3");
+  if (num_blocks * block_size > INT32_MAX)
+    return fail(PA_ERR_UNSUPPORTED, "decode: pool rows exceed 2^31");
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "decode: scale is not finite");
+  if (!workspace || !aligned(workspace, 256))
+    return fail(PA_ERR_INVALID_ARG, "decode: workspace missing or not 256-byte aligned");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens)
+    return fail(PA_ERR_INVALID_ARG, "decode: null pointer");
+  if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) ||
+      !aligned(value_cache, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4) ||
+      (k_scale && !aligned(k_scale, 4)) || (v_scale && !aligned(v_scale, 4)))
+    return fail(PA_ERR_INVALID_ARG, "decode: misaligned pointer");
+
+  const Plan plan =
+      make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
+  if (num_seqs > 65535 || plan.max_parts > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "decode: %d sequences x %d partitions exceed the grid",
+                num_seqs, plan.max_parts);
+  const size_t need = workspace_bytes_for(plan, num_seqs, num_heads, head_dim);
+  if (workspace_bytes < need)
+    return fail(PA_ERR_INVALID_ARG, "decode: workspace %zu bytes < %zu needed", workspace_bytes,
+                need);
+
+  const int elem = elem_bytes(cache_dtype);
+  CUtensorMap kmap, vmap;
+  pa_status st =
+      encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads, head_dim, elem);
+  if (st == PA_OK)
+    st = encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim,
+                          elem);
+  if (st != PA_OK) return st;
+
+  DecodeArgs a{};
+  a.out = out;
+  a.query = query;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.err = reinterpret_cast<int32_t*>(ws);
+  if (plan.max_parts > 1) {
+    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * plan.max_parts;
+    a.ws_ml = reinterpret_cast<float2*>(ws + kHeaderBytes);
+    a.ws_o = reinterpret_cast<float*>(ws + kHeaderBytes +
+                                      ((rows * sizeof(float2) + 255) & ~size_t(255)));
+  }
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.ctx_limit = std::min<int64_t>(max_context_len,
+                                  static_cast<int64_t>(max_blocks_per_seq) * block_size);
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.partition_blocks = plan.partition_blocks;
+  a.max_parts = plan.max_parts;
+  a.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  DecodeFn fn = nullptr;
+  if (q_dtype == PA_F16) fn = fp8 ? decode_f16_e4m3 : decode_f16_f16;
+  else fn = fp8 ? decode_bf16_e4m3 : decode_bf16_bf16;
+  st = cuda_status(fn(a, kmap, vmap, head_dim, block_size, group, cs), "decode");
+  if (st != PA_OK || plan.max_parts <= 1) return st;
+  return cuda_status(launch_reduce(a, q_dtype, head_dim, block_size, cs), "decode reduce");
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// decode_args.h — host/device argument block of the decode kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace paged {
+
+enum DType : int { kF16 = 0, kBF16 = 1, kE4M3 = 2 };
+
+// Bits of the workspace error word.
+enum : int32_t {
+  kErrBadBlockId = 1,      // a block-table entry outside [0, num_blocks)
+  kErrContextClipped = 2,  // a context length above what the launch covers
+  kErrWaitTimeout = 4,     // a pipeline wait gave up (never expected)
+  kErrBadSlot = 8,         // reshape_and_cache: a slot outside the pool
+};
+
+
+struct DecodeArgs {
+  void* out;                    // [S, H, D] q dtype
+  const void* query;            // [S, H, D] q dtype
+  const int32_t* block_tables;  // [S, max_blocks_per_seq]
+  const int32_t* context_lens;  // [S]
+  const float* k_scale;         // [Hkv] (FP8 cache) or null
+  const float* v_scale;
+  float* ws_o;                  // [S, H, max_parts, D] partial outputs (split mode)
+  float2* ws_ml;                // [S, H, max_parts] (running max, sum) in log2 units
+  int32_t* err;                 // error word (bits of the kErr* enum)
+  int64_t num_blocks;
+  int32_t max_blocks_per_seq;
+  int32_t ctx_limit;            // min(max_context_len, max_blocks_per_seq * block_size)
+  int32_t num_seqs;
+  int32_t num_heads;
+  int32_t num_kv_heads;
+  int32_t partition_blocks;     // blocks per partition (single pass: covers max context)
+  int32_t max_parts;            // partitions per sequence in the launch (1 = single pass)
+  float scale_log2;             // softmax scale * log2(e)
+};
+
+// Launch configuration chosen on the host.
+struct DecodeLaunch {
+  dim3 grid;
+  int32_t threads;
+  size_t smem_bytes;
+};
+
+// Per (q dtype, cache dtype) dispatchers, defined in decode_<q>_<c>.cu.
+// Return cudaErrorNotSupported for a (head_dim, block_size, group) they lack.
+using DecodeFn = cudaError_t (*)(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&,
+                                 int head_dim, int block_size, int group, cudaStream_t);
+
+cudaError_t decode_f16_f16(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int, int,
+                           int, cudaStream_t);
+cudaError_t decode_bf16_bf16(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int,
+                             int, int, cudaStream_t);
+cudaError_t decode_f16_e4m3(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int, int,
+                            int, cudaStream_t);
+cudaError_t decode_bf16_e4m3(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int,
+                             int, int, cudaStream_t);
+
+cudaError_t launch_reduce(const DecodeArgs& a, int q_dtype, int head_dim, int block_size,
+                          cudaStream_t stream);
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
+                                     void* value_cache, const int32_t* slot_mapping,
+                                     int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int64_t num_blocks, int kv_dtype,
+                                     int cache_dtype, const float* k_scale, const float* v_scale,
+                                     int32_t* err, cudaStream_t stream);
+
+// Box geometry shared by the host tensor-map encoder and the kernels: a row
+// of head_dim elements is cut into boxes of at most 128 bytes, each loaded
+// with the matching shared-memory swizzle.
+__host__ __device__ constexpr int box_bytes(int row_bytes) { return row_bytes < 128 ? row_bytes : 128; }
+
+}  // namespace paged

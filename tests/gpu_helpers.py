@@ -1,0 +1,105 @@
+"""Helpers shared by the GPU tests: moving raw host codes to torch device
+tensors, running one decode step (reshape_and_cache of the new token, then
+decode) through the library, and the oracle's side of the same step."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import paged_kv_cache_448_b200 as pk
+from paged_kv_cache_448_b200 import workloads as wl
+
+# Element-wise acceptance: |gpu - ref| <= ATOL + RTOL * |ref|.
+TOL = {"f16": (2e-3, 1e-2), "bf16": (2e-3, 1e-2), "e4m3": (3e-2, 3e-2)}
+
+_TORCH = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def dev(codes: np.ndarray, dt: str, device="cuda") -> torch.Tensor:
+    """Raw host codes -> device tensor of the storage dtype (E4M3 as uint8)."""
+    a = np.ascontiguousarray(codes)
+    if dt == "e4m3":
+        return torch.from_numpy(a.view(np.uint8)).to(device)
+    return torch.from_numpy(a.view(np.int16)).view(_TORCH[dt]).to(device)
+
+
+def host_codes(t: torch.Tensor) -> np.ndarray:
+    """Device tensor -> raw host codes (uint16 for 16-bit types, uint8 for E4M3)."""
+    t = t.detach().contiguous().cpu()
+    if t.dtype in (torch.float16, torch.bfloat16):
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.view(torch.uint8).numpy()
+
+
+def i32(a, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+
+def f32(a, device="cuda"):
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+
+
+def within_tol(gpu: np.ndarray, ref: np.ndarray, cache_dtype: str):
+    atol, rtol = TOL[cache_dtype]
+    err = np.abs(gpu - ref)
+    ok = err <= atol + rtol * np.abs(ref)
+    return bool(ok.all()), float(err.max(initial=0.0))
+
+
+def assert_close(gpu: np.ndarray, ref: np.ndarray, cache_dtype: str, what=""):
+    ok, worst = within_tol(gpu, ref, cache_dtype)
+    assert np.isfinite(gpu).all(), f"{what}: non-finite output"
+    if not ok:
+        atol, rtol = TOL[cache_dtype]
+        bad = np.argwhere(np.abs(gpu - ref) > atol + rtol * np.abs(ref))
+        i = tuple(bad[0])
+        raise AssertionError(f"{what}: {len(bad)} elements out of tolerance; first {i}: "
+                             f"gpu={gpu[i]!r} ref={ref[i]!r} (max abs err {worst:.3g})")
+
+
+class GpuStep:
+    """Device copies of a workload and the library calls of one decode step."""
+
+    def __init__(self, sp: wl.Spec, st: wl.Structure, hd: wl.HostData, device="cuda"):
+        self.sp, self.st, self.hd = sp, st, hd
+        self.q = dev(hd.query, sp.q_dtype, device)
+        self.kc = dev(hd.key_cache, sp.cache_dtype, device)
+        self.vc = dev(hd.value_cache, sp.cache_dtype, device)
+        self.nk = dev(hd.new_key, sp.q_dtype, device)
+        self.nv = dev(hd.new_value, sp.q_dtype, device)
+        self.ks, self.vs = f32(hd.k_scale, device), f32(hd.v_scale, device)
+        self.bt = i32(st.block_tables, device)
+        self.cl = i32(sp.context_lens, device)
+        slots = pk.build_slot_mapping(st.block_tables, st.positions, sp.block_size)
+        self.slots = i32(slots, device)
+        self.out = torch.empty_like(self.q)
+        self.max_ctx = int(sp.context_lens.max())
+
+    def reshape(self):
+        pk.reshape_and_cache(self.nk, self.nv, self.kc, self.vc, self.slots, k_scale=self.ks,
+                             v_scale=self.vs)
+
+    def decode(self, partition_tokens=None, workspace=None):
+        p = self.sp.partition_tokens if partition_tokens is None else partition_tokens
+        return pk.decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, self.max_ctx,
+                         self.sp.scale, k_scale=self.ks, v_scale=self.vs, partition_tokens=p,
+                         workspace=workspace)
+
+    def out_f64(self) -> np.ndarray:
+        return self.out.double().cpu().numpy()
+
+
+def oracle_step(sp: wl.Spec, st: wl.Structure, hd: wl.HostData, seqs=None):
+    """The oracle's reshape_and_cache of the new tokens followed by decode.
+    Returns (key_cache, value_cache, out[S, H, D] fp64) on the host."""
+    kc, vc = hd.key_cache.copy(), hd.value_cache.copy()
+    slots = oracle.slot_mapping(st.block_tables, st.positions, sp.block_size)
+    oracle.reshape_and_cache(hd.new_key, hd.new_value, kc, vc, slots, block_size=sp.block_size,
+                             kv_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype,
+                             k_scale=hd.k_scale, v_scale=hd.v_scale)
+    sel = slice(None) if seqs is None else np.asarray(seqs)
+    out = oracle.decode(hd.query[sel], kc, vc, st.block_tables[sel], sp.context_lens[sel],
+                        scale=np.float32(sp.scale), q_dtype=sp.q_dtype,
+                        cache_dtype=sp.cache_dtype, k_scale=hd.k_scale, v_scale=hd.v_scale)
+    return kc, vc, out

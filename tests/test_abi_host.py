@@ -1,0 +1,195 @@
+"""CPU tests of libpaged.so: it loads, exports every call include/paged.h
+declares, the host allocator and table builders agree with the oracle model
+bit for bit, and argument errors are rejected on the host before any launch."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.block_manager import BlockManager, OutOfBlocks
+import paged_kv_cache_448_b200 as pk
+from paged_kv_cache_448_b200 import _native
+from paged_kv_cache_448_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "paged.h")).read()
+    return sorted(set(re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_call():
+    lib = _native.lib()
+    declared = header_functions()
+    assert len(declared) >= 18
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(n for n, _, _ in _native.SIGNATURES) == declared
+
+
+def test_library_is_the_in_tree_build():
+    assert os.path.dirname(_native.LIB_PATH) == os.path.join(ROOT, "paged_kv_cache_448_b200")
+
+
+# ------------------------------------------------------------- allocator
+
+def test_allocator_matches_oracle_model_on_random_ops():
+    rng = np.random.default_rng(21)
+    for trial in range(20):
+        nb = int(rng.integers(1, 200))
+        order = rng.permutation(nb).astype(np.int32)
+        ours = pk.BlockAllocator(nb, order)
+        ref = BlockManager(nb, order)
+        live = []                      # references held (block ids, with repeats)
+        for _ in range(300):
+            op = rng.integers(0, 4)
+            if op == 0:
+                n = int(rng.integers(0, 12))
+                try:
+                    expect = ref.allocate(n)
+                except OutOfBlocks:
+                    with pytest.raises(pk.PagedError) as ei:
+                        ours.allocate(n)
+                    assert ei.value.status == _native.PA_ERR_OOM
+                    continue
+                assert ours.allocate(n) == expect
+                live.extend(expect)
+            elif op == 1 and live:
+                b = int(rng.choice(live))
+                ref.share(b); ours.share(b)
+                live.append(b)
+            elif op == 2 and live:
+                k = int(rng.integers(1, min(6, len(live)) + 1))
+                idx = rng.choice(len(live), size=k, replace=False)
+                ids = [live[i] for i in idx]
+                ref.free(ids); ours.free(ids)
+                for i in sorted(idx, reverse=True):
+                    live.pop(i)
+            elif op == 3:
+                # an invalid free (a block with no references left) changes nothing
+                free_ids = ref.free_blocks[:1]
+                if free_ids:
+                    with pytest.raises(pk.PagedError):
+                        ours.free(free_ids)
+            assert ours.free_list() == ref.free_blocks
+            assert ours.num_free == ref.num_free()
+        for b in range(nb):
+            assert ours.refcount(b) == ref.refcount[b]
+        ours.close()
+
+
+def test_allocator_rejects_non_permutation_and_bad_ids():
+    with pytest.raises(pk.PagedError):
+        pk.BlockAllocator(3, [0, 0, 1])
+    a = pk.BlockAllocator(4)
+    with pytest.raises(pk.PagedError):
+        a.share(2)                      # free block
+    ids = a.allocate(2)
+    with pytest.raises(pk.PagedError):
+        a.free([ids[0], ids[0]])        # more drops than references: nothing changes
+    assert a.refcount(ids[0]) == 1 and a.num_free == 2
+    assert a.refcount(99) == -1
+
+
+def test_block_table_builder():
+    t = pk.build_block_table([[5, 1], [], [3, 2, 0]], 4)
+    assert t.tolist() == [[5, 1, -1, -1], [-1, -1, -1, -1], [3, 2, 0, -1]]
+    with pytest.raises(pk.PagedError):
+        pk.build_block_table([[1, 2, 3]], 2)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+def test_slot_mapping_matches_oracle(cfg):
+    sp = wl.spec(cfg, small=cfg != 1)
+    st = wl.structure(sp)
+    ours = pk.build_slot_mapping(st.block_tables, st.positions, sp.block_size)
+    ref = oracle.slot_mapping(st.block_tables, st.positions, sp.block_size)
+    assert np.array_equal(ours, ref)
+    # every position of every sequence, with explicit sequence ids
+    seq = np.concatenate([np.full(n, s, np.int32) for s, n in enumerate(sp.context_lens)])
+    pos = np.concatenate([np.arange(n, dtype=np.int32) for n in sp.context_lens])
+    pos[::7] = -1
+    assert np.array_equal(pk.build_slot_mapping(st.block_tables, pos, sp.block_size, seq),
+                          oracle.slot_mapping(st.block_tables, pos, sp.block_size, seq))
+
+
+def test_slot_mapping_errors():
+    t = np.array([[4, -1]], np.int32)
+    with pytest.raises(pk.PagedError) as e:
+        pk.build_slot_mapping(t, [20], 16)
+    assert e.value.status == _native.PA_ERR_BAD_TABLE
+    with pytest.raises(pk.PagedError):
+        pk.build_slot_mapping(t, [40], 16)
+    assert pk.build_slot_mapping(t, [-3, 3], 16, seq_ids=[0, 0]).tolist() == [-1, 67]
+
+
+# --------------------------------------------------- host-side validation
+
+def _decode_raw(**over):
+    args = dict(out=16, query=16, kc=16, vc=16, bt=16, mbps=4, cl=16, max_ctx=64, S=2, H=8,
+                Hkv=2, D=128, BS=16, NB=10, scale=0.1, qdt=_native.PA_F16, cdt=_native.PA_F16,
+                ks=None, vs=None, part=0, ws=256, wsb=1 << 20)
+    args.update(over)
+    a = args
+    return _native.lib().pa_decode(a["out"], a["query"], a["kc"], a["vc"], a["bt"], a["mbps"],
+                                   a["cl"], a["max_ctx"], a["S"], a["H"], a["Hkv"], a["D"],
+                                   a["BS"], a["NB"], a["scale"], a["qdt"], a["cdt"], a["ks"],
+                                   a["vs"], a["part"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(H=6, Hkv=4), _native.PA_ERR_INVALID_ARG),
+    (dict(H=32, Hkv=2), _native.PA_ERR_UNSUPPORTED),        # group 16
+    (dict(D=96), _native.PA_ERR_UNSUPPORTED),
+    (dict(BS=8), _native.PA_ERR_UNSUPPORTED),
+    (dict(qdt=_native.PA_FP8_E4M3), _native.PA_ERR_UNSUPPORTED),
+    (dict(cdt=_native.PA_BF16), _native.PA_ERR_UNSUPPORTED),
+    (dict(cdt=_native.PA_FP8_E4M3), _native.PA_ERR_INVALID_ARG),  # scales missing
+    (dict(out=8), _native.PA_ERR_INVALID_ARG),                      # misaligned
+    (dict(ws=128), _native.PA_ERR_INVALID_ARG),                     # workspace alignment
+    (dict(ws=None), _native.PA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _native.PA_ERR_INVALID_ARG),
+    (dict(S=-1), _native.PA_ERR_INVALID_ARG),
+    (dict(NB=1 << 28), _native.PA_ERR_UNSUPPORTED),                 # pool rows > 2^31
+])
+def test_decode_rejects_bad_arguments_before_launch(over, status):
+    assert _decode_raw(**over) == status
+    assert _native.lib().pa_last_error()
+
+
+def test_decode_with_no_sequences_is_a_no_op():
+    assert _decode_raw(S=0, out=None, query=None) == _native.PA_OK
+
+
+def test_reshape_rejects_bad_arguments():
+    lib = _native.lib()
+    f = lib.pa_reshape_and_cache
+    ok = dict(k=16, v=16, kc=16, vc=16, sm=16, T=4, Hkv=2, D=128, BS=16, NB=4,
+              kdt=_native.PA_F16, cdt=_native.PA_F16, ks=None, vs=None)
+
+    def call(**o):
+        a = dict(ok); a.update(o)
+        return f(a["k"], a["v"], a["kc"], a["vc"], a["sm"], a["T"], a["Hkv"], a["D"], a["BS"],
+                 a["NB"], a["kdt"], a["cdt"], a["ks"], a["vs"], None)
+    assert call(D=80) == _native.PA_ERR_UNSUPPORTED
+    assert call(kdt=_native.PA_FP8_E4M3) == _native.PA_ERR_UNSUPPORTED
+    assert call(cdt=_native.PA_FP8_E4M3) == _native.PA_ERR_INVALID_ARG
+    assert call(k=24) == _native.PA_ERR_INVALID_ARG
+    assert call(T=0, k=None) == _native.PA_OK
+
+
+def test_workspace_sizes_and_partition_plan():
+    # single pass: only the 256-byte header
+    assert pk.decode_workspace_size(4, 4, 4, 64, 16, 100, 0) == 256
+    assert pk.decode_partition_tokens(4, 4, 4, 64, 16, 100, 0) >= 100
+    # forced partitions of 512 tokens over 2048: 4 partials per (seq, head)
+    n = pk.decode_workspace_size(32, 32, 32, 128, 16, 2048, 512)
+    rows = 32 * 32 * 4
+    assert n >= 256 + rows * 8 + rows * 128 * 4
+    assert pk.decode_partition_tokens(32, 32, 32, 128, 16, 2048, 512) == 512
+    # partitions are whole blocks
+    assert pk.decode_partition_tokens(2, 8, 8, 128, 32, 4096, 300) == 320
