@@ -91,7 +91,7 @@ def test_decode_step_matches_oracle(cfg, path):
     g = GpuStep(sp, st, hd)
     g.reshape()
     part = {"auto": None, "single": 1 << 20, "split": 4 * sp.block_size}[path]
-    ws = g.decode(partition_tokens=part) and None
+    g.decode(partition_tokens=part)
     torch.cuda.synchronize()
     _, _, ref = oracle_step(sp, st, hd)
     assert_close(g.out_f64(), ref, sp.cache_dtype, f"cfg{cfg}/{path}")
