@@ -154,6 +154,38 @@ PA_API pa_status pa_decode(void* out, const void* query,
                     pa_stream_t stream);
 
 /*
+ * pa_decode without a workspace argument, for callers that cannot allocate
+ * device memory: a serving loop that forbids cudaMalloc once it is running
+ * (cudaMalloc synchronises the device and stalls every stream), a process whose
+ * device memory is already claimed by another framework's caching allocator,
+ * or a host-language binding that has no device allocation API. The pages
+ * describe nothing like it; it exists only for those callers.
+ *
+ * Same arguments, meaning and results as pa_decode, minus workspace and
+ * workspace_bytes. The scratch is a 32 MiB file-scope device array inside this
+ * library, held on every GPU that loads the library until the process exits.
+ * The call allocates and frees nothing. Sizes whose partitioned path needs more
+ * than 32 MiB (pa_decode_workspace_size > 32 MiB) return PA_ERR_UNSUPPORTED
+ * without launching; use pa_decode for them.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. Every call shares the one array and leaves its contents behind:
+ * two calls whose kernels overlap on the GPU (e.g. on two streams) race on it
+ * and give wrong results, so serialise them. Nothing in it needs clearing
+ * between calls (every partial result is written before it is read). Table
+ * errors are made harmless as in pa_decode but are not reported.
+ */
+PA_API pa_status pa_decode_noalloc(void* out, const void* query,
+                    const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t max_context_len,
+                    int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                    float scale, pa_dtype q_dtype, pa_dtype cache_dtype,
+                    const float* k_scale, const float* v_scale,
+                    int32_t partition_tokens, pa_stream_t stream);
+
+/*
  * Bytes of workspace pa_decode needs for these sizes on the current device
  * (the automatic partition choice depends on the device's SM count).
  * Returns 0 for invalid sizes.

@@ -20,7 +20,8 @@ import numpy as np
 from . import _native
 from ._native import PagedError, check
 
-__all__ = ["reshape_and_cache", "decode", "decode_workspace", "decode_workspace_size",
+__all__ = ["reshape_and_cache", "decode", "decode_noalloc", "decode_workspace",
+           "decode_workspace_size",
            "decode_partition_tokens", "decode_check", "BlockAllocator", "build_block_table",
            "build_slot_mapping", "PagedError", "dtype_code"]
 
@@ -100,6 +101,22 @@ def decode(out, query, key_cache, value_cache, block_tables, context_lens, max_c
         block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, H, Hkv, D, BS, NB,
         float(scale), dtype_code(query), dtype_code(key_cache), _ptr(k_scale), _ptr(v_scale),
         int(partition_tokens), _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+    return out
+
+
+def decode_noalloc(out, query, key_cache, value_cache, block_tables, context_lens,
+                   max_context_len: int, scale: float, *, k_scale=None, v_scale=None,
+                   partition_tokens: int = 0, stream=None):
+    """decode() for callers that cannot allocate device memory: the library's
+    own static 32 MiB device scratch replaces the workspace (pa_decode_noalloc).
+    Calls that overlap on the GPU race on that scratch. Returns ``out``."""
+    S, H, D = query.shape
+    NB, BS, Hkv = key_cache.shape[:3]
+    check(_native.lib().pa_decode_noalloc(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, H, Hkv, D, BS, NB,
+        float(scale), dtype_code(query), dtype_code(key_cache), _ptr(k_scale), _ptr(v_scale),
+        int(partition_tokens), _stream_handle(stream)))
     return out
 
 
