@@ -1,5 +1,5 @@
 // Decode kernels for query dtype BF16, cache dtype BF16 (all head_dim, block_size, group).
-#include "decode_simt.cuh"
+#include "decode_dispatch.cuh"
 
 namespace paged {
 cudaError_t decode_bf16_bf16(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,

@@ -1,5 +1,5 @@
 // Decode kernels for query dtype BF16, cache dtype E4M3 (all head_dim, block_size, group).
-#include "decode_simt.cuh"
+#include "decode_dispatch.cuh"
 
 namespace paged {
 cudaError_t decode_bf16_e4m3(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,

@@ -1,5 +1,5 @@
 // Decode kernels for query dtype F16, cache dtype F16 (all head_dim, block_size, group).
-#include "decode_simt.cuh"
+#include "decode_dispatch.cuh"
 
 namespace paged {
 cudaError_t decode_f16_f16(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
