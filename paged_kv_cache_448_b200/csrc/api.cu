@@ -51,26 +51,28 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Tensor map over a cache viewed as [num_blocks*block_size rows][num_kv_heads][head_dim]
-// with a box of one kv-head's block_size rows and <=128 bytes of each row.
+// Tensor map over a cache viewed as [rows = num_blocks*block_size][num_kv_heads]
+// [segments][segment elements] (a row of head_dim elements cut into <=128-byte
+// segments): one box = 16 rows of one kv-head, whole rows, swizzled per segment.
 pa_status encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks,
                            int32_t block_size, int32_t hkv, int32_t head_dim, int elem) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int row_bytes = head_dim * elem;
-  const int bb = box_bytes(row_bytes);
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(hkv),
+  const int seg = box_bytes(row_bytes);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(seg / elem),
+                        static_cast<cuuint64_t>(row_bytes / seg), static_cast<cuuint64_t>(hkv),
                         static_cast<cuuint64_t>(num_blocks) * block_size};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes),
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(seg), static_cast<cuuint64_t>(row_bytes),
                            static_cast<cuuint64_t>(row_bytes) * hkv};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(bb / elem), 1u,
-                       static_cast<cuuint32_t>(block_size)};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  const CUtensorMapSwizzle swz = bb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                               : bb == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
-                                           : CU_TENSOR_MAP_SWIZZLE_NONE;
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(seg / elem),
+                       static_cast<cuuint32_t>(row_bytes / seg), 1u, 16u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUtensorMapSwizzle swz = seg == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                               : seg == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_NONE;
   CUresult r = enc(map, elem == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                   3, const_cast<void*>(cache), dims, strides, box, estr,
+                   4, const_cast<void*>(cache), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
@@ -93,6 +95,8 @@ struct Plan {
   int32_t max_parts;         // 1 = single pass
 };
 
+constexpr int32_t kMaxParts = 1024;  // partitions per sequence the decode kernel handles
+
 Plan make_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
                int32_t max_context_len, int32_t requested) {
   const int32_t blocks_max = std::max<int32_t>(1, (max_context_len + block_size - 1) / block_size);
@@ -101,8 +105,8 @@ Plan make_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
   if (requested > 0) {
     pb = (requested + block_size - 1) / block_size;
   } else {
-    // Enough independent work units to fill every SM several times over;
-    // otherwise cut the context into partitions (>= 256 tokens each).
+    // Enough independent work units to keep every SM busy through the end of
+    // the launch; otherwise cut the context into partitions (>= 256 tokens).
     const int64_t pairs = static_cast<int64_t>(num_seqs) * num_kv_heads;
     const int64_t want = 4LL * sm_count() * 3;
     pb = blocks_max;
@@ -117,17 +121,42 @@ Plan make_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
     }
   }
   pb = std::min(std::max(pb, 1), std::min(blocks_max, kMaxPartitionBlocks));
+  pb = std::max(pb, (blocks_max + kMaxParts - 1) / kMaxParts);
   p.partition_blocks = pb;
   p.partition_tokens = pb * block_size;
   p.max_parts = (blocks_max + pb - 1) / pb;
   return p;
 }
 
-size_t workspace_bytes_for(const Plan& p, int32_t num_seqs, int32_t num_heads, int32_t head_dim) {
-  if (p.max_parts <= 1) return kHeaderBytes;
-  const size_t rows = static_cast<size_t>(num_seqs) * num_heads * p.max_parts;
-  const size_t ml = (rows * sizeof(float2) + 255) & ~size_t(255);
-  return kHeaderBytes + ml + rows * head_dim * sizeof(float);
+// Workspace layout: [header 256 B: error word, work counter, unit total]
+// [slice starts, max_parts+1 int32] [sequence order, S int2]
+// then, with partitions: [arrival counters, S*Hkv int32]
+// [partial (m, l), S*H*max_parts float2] [partial o, S*H*max_parts*D float].
+struct Layout {
+  size_t slice, order, arrive, ml, o, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Layout layout_for(const Plan& p, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                  int32_t head_dim) {
+  Layout l{};
+  size_t at = kHeaderBytes;
+  l.slice = at;
+  at = align256(at + 4 * static_cast<size_t>(p.max_parts + 1));
+  l.order = at;
+  at = align256(at + 8 * static_cast<size_t>(num_seqs));
+  if (p.max_parts > 1) {
+    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * p.max_parts;
+    l.arrive = at;
+    at = align256(at + 4 * static_cast<size_t>(num_seqs) * num_kv_heads);
+    l.ml = at;
+    at = align256(at + rows * sizeof(float2));
+    l.o = at;
+    at += rows * head_dim * sizeof(float);
+  }
+  l.total = at;
+  return l;
 }
 
 bool shape_supported(int32_t head_dim, int32_t block_size) {
@@ -192,7 +221,7 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int3
       max_context_len < 0)
     return 0;
   Plan p = make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
-  return workspace_bytes_for(p, num_seqs, num_heads, head_dim);
+  return layout_for(p, num_seqs, num_heads, num_kv_heads, head_dim).total;
 }
 
 PA_API pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_stream_t stream) {
@@ -211,9 +240,11 @@ PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream) {
   int32_t word = 0;
   cudaError_t e = cudaStreamSynchronize(st);
   if (e == cudaSuccess) e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
-  if (e == cudaSuccess && word != 0) e = cudaMemset(workspace, 0, sizeof(word));
+  if (e == cudaSuccess && word != 0) e = cudaMemset(workspace, 0, 64);  // error + failure record
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode_check: %s", cudaGetErrorString(e));
-  if (word & kErrWaitTimeout) return fail(PA_ERR_CUDA, "decode: a pipeline wait timed out");
+  if (word & (kErrWaitTimeout | kErrBadPlan))
+    return fail(PA_ERR_CUDA, "decode: %s", (word & kErrBadPlan) ? "a work unit outside the plan"
+                                                                : "a pipeline wait timed out");
   if (word & (kErrBadBlockId | kErrContextClipped))
     return fail(PA_ERR_BAD_TABLE, "decode: %s%s",
                 (word & kErrBadBlockId) ? "block-table entry outside the pool; " : "",
@@ -264,10 +295,11 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
 
   const Plan plan =
       make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
-  if (num_seqs > 65535 || plan.max_parts > 65535)
-    return fail(PA_ERR_UNSUPPORTED, "decode: %d sequences x %d partitions exceed the grid",
-                num_seqs, plan.max_parts);
-  const size_t need = workspace_bytes_for(plan, num_seqs, num_heads, head_dim);
+  if (plan.max_parts > kMaxParts || num_kv_heads > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "decode: %d partitions / %d kv-heads exceed the plan",
+                plan.max_parts, num_kv_heads);
+  const Layout lay = layout_for(plan, num_seqs, num_heads, num_kv_heads, head_dim);
+  const size_t need = lay.total;
   if (workspace_bytes < need)
     return fail(PA_ERR_INVALID_ARG, "decode: workspace %zu bytes < %zu needed", workspace_bytes,
                 need);
@@ -289,12 +321,15 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
   a.k_scale = k_scale;
   a.v_scale = v_scale;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  a.err = reinterpret_cast<int32_t*>(ws);
+  a.err = reinterpret_cast<int32_t*>(ws) + kWordError;
+  a.counters = reinterpret_cast<int32_t*>(ws);
+  a.diag = reinterpret_cast<int32_t*>(ws) + kWordDiag;
+  a.slice_start = reinterpret_cast<const int32_t*>(ws + lay.slice);
+  a.order = reinterpret_cast<const int2*>(ws + lay.order);
   if (plan.max_parts > 1) {
-    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * plan.max_parts;
-    a.ws_ml = reinterpret_cast<float2*>(ws + kHeaderBytes);
-    a.ws_o = reinterpret_cast<float*>(ws + kHeaderBytes +
-                                      ((rows * sizeof(float2) + 255) & ~size_t(255)));
+    a.arrive = reinterpret_cast<int32_t*>(ws + lay.arrive);
+    a.ws_ml = reinterpret_cast<float2*>(ws + lay.ml);
+    a.ws_o = reinterpret_cast<float*>(ws + lay.o);
   }
   a.num_blocks = num_blocks;
   a.max_blocks_per_seq = max_blocks_per_seq;
@@ -306,14 +341,30 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
   a.partition_blocks = plan.partition_blocks;
   a.max_parts = plan.max_parts;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.num_sms = sm_count();
+  a.block_size = block_size;
+
+  PlanArgs pa{};
+  pa.context_lens = context_lens;
+  pa.err = a.err;
+  pa.counters = a.counters;
+  pa.slice_start = reinterpret_cast<int32_t*>(ws + lay.slice);
+  pa.order = reinterpret_cast<int2*>(ws + lay.order);
+  pa.arrive = a.arrive;
+  pa.num_seqs = num_seqs;
+  pa.num_kv_heads = num_kv_heads;
+  pa.block_size = block_size;
+  pa.partition_blocks = plan.partition_blocks;
+  pa.max_parts = plan.max_parts;
+  pa.ctx_limit = a.ctx_limit;
 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   DecodeFn fn = nullptr;
   if (q_dtype == PA_F16) fn = fp8 ? decode_f16_e4m3 : decode_f16_f16;
   else fn = fp8 ? decode_bf16_e4m3 : decode_bf16_bf16;
-  st = cuda_status(fn(a, kmap, vmap, head_dim, block_size, group, cs), "decode");
-  if (st != PA_OK || plan.max_parts <= 1) return st;
-  return cuda_status(launch_reduce(a, q_dtype, head_dim, block_size, cs), "decode reduce");
+  st = cuda_status(launch_plan(pa, cs), "decode plan");
+  if (st != PA_OK) return st;
+  return cuda_status(fn(a, kmap, vmap, head_dim, group, cs), "decode");
 }
 
 }  // extern "C"

@@ -82,17 +82,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   }
 }
 
-template <class QF_, class CF_, int D_, int BS_, int G_>
+template <class QF_, class CF_, int D_, int G_>
 struct MmaConsumer {
   using QF = QF_;
   using CF = CF_;
-  using Tile = paged::Tile<CF, D_, BS_>;
-  static constexpr int D = D_, BS = BS_, G = G_;
+  using Tile = paged::Tile<CF, D_>;
+  static constexpr int D = D_, BS = Tile::BS, G = G_;
   static constexpr bool FP8 = CF::kBytes == 1;
   static constexpr bool BF = !FP8 && std::is_same<CF, BF16>::value;  // MMA input type
-  static constexpr int NW = 4;
-  static constexpr int R_RAW = 65536 / (NW * 2 * Tile::BYTES);
-  static constexpr int R = R_RAW < 1 ? 1 : (R_RAW > 4 ? 4 : R_RAW);
   static constexpr int KS = D / 16;   // k-steps of Q.K^T (head_dim)
   static constexpr int NS = BS / 8;   // n-tiles of S (tokens)
   static constexpr int KP = BS / 16;  // k-steps of P.V (tokens)
@@ -104,14 +101,15 @@ struct MmaConsumer {
   float m, l, qscale;
   int r, c;
 
-  __device__ __forceinline__ void init(const DecodeArgs& a, int s, int kvh, int lane) {
+  // qrows: the G query rows of this kv-head ([G][D], q dtype; global or shared).
+  __device__ __forceinline__ void init(const DecodeArgs& a, const void* qrows, int kvh, int lane) {
     r = lane >> 2;
     c = lane & 3;
     const bool live = r < G;
-    const int64_t qrow = (static_cast<int64_t>(s) * a.num_heads + kvh * G + (live ? r : 0)) * D;
+    const int qrow = (live ? r : 0) * D;
     qscale = a.scale_log2;
     if constexpr (!FP8) {
-      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(a.query);
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrows);
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
         qa[kk][0] = live ? q32[(qrow + 16 * kk + 2 * c) / 2] : 0u;
@@ -124,7 +122,7 @@ struct MmaConsumer {
       for (int kk = 0; kk < KS; ++kk)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          qv[kk][j] = live ? load_in(QF{}, a.query, qrow + 16 * kk + 4 * c + j) : 0.f;
+          qv[kk][j] = live ? load_in(QF{}, qrows, qrow + 16 * kk + 4 * c + j) : 0.f;
           mx = fmaxf(mx, fabsf(qv[kk][j]));
         }
 #pragma unroll

@@ -14,16 +14,13 @@
 
 namespace paged {
 
-template <class QF_, class CF_, int D_, int BS_, int G_>
+template <class QF_, class CF_, int D_, int G_>
 struct SimtConsumer {
   using QF = QF_;
   using CF = CF_;
-  using Tile = paged::Tile<CF, D_, BS_>;
-  static constexpr int D = D_, BS = BS_, G = G_;
+  using Tile = paged::Tile<CF, D_>;
+  static constexpr int D = D_, BS = Tile::BS, G = G_;
   static constexpr int EB = CF::kBytes, RB = Tile::RB;
-  static constexpr int NW = 4;
-  static constexpr int R_RAW = 65536 / (NW * 2 * Tile::BYTES);
-  static constexpr int R = R_RAW < 1 ? 1 : (R_RAW > 4 ? 4 : R_RAW);
   static constexpr int TPT_RAW = G * D / 16;
   static constexpr int TPT = TPT_RAW < 8 ? 8 : (TPT_RAW > 32 ? 32 : TPT_RAW);
   static constexpr int NTG = 32 / TPT;           // token groups per warp
@@ -87,16 +84,16 @@ struct SimtConsumer {
     }
   }
 
-  __device__ __forceinline__ void init(const DecodeArgs& a, int s, int kvh, int lane) {
+  // qrows: the G query rows of this kv-head ([G][D], q dtype; global or shared).
+  __device__ __forceinline__ void init(const DecodeArgs& a, const void* qrows, int kvh, int lane) {
     tg = lane / TPT;
     li = lane % TPT;
     float qs = a.scale_log2;
     if (a.k_scale) qs *= a.k_scale[kvh];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const int64_t qrow = (static_cast<int64_t>(s) * a.num_heads + kvh * G + g) * D;
 #pragma unroll
-      for (int e = 0; e < NE; ++e) qf[g][e] = load_in(QF{}, a.query, qrow + lane_dim(li, e)) * qs;
+      for (int e = 0; e < NE; ++e) qf[g][e] = load_in(QF{}, qrows, g * D + lane_dim(li, e)) * qs;
       m[g] = -CUDART_INF_F;
       l[g] = 0.f;
 #pragma unroll

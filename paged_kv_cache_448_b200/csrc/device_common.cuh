@@ -13,10 +13,16 @@
 
 namespace paged {
 
-// Upper bound on mbarrier polls before a wait gives up and reports
-// kErrWaitTimeout (each try_wait blocks for a hardware-defined slice; this
-// bound is many seconds, far above any real TMA latency).
-constexpr uint32_t kMaxWaitPolls = 1u << 26;
+// Wall-clock bound of every pipeline wait: far above any real TMA or
+// hand-over latency, yet a wait that can never complete ends in about a second
+// (the kernel then reports kErrWaitTimeout instead of hanging).
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -42,6 +48,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Plain bulk copy global -> shared (16-byte aligned addresses, size a multiple
+// of 16), completion counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -54,33 +75,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for phase `parity` of `bar`; false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kMaxWaitPolls; ++i)
+// Wait for phase `parity` of `bar` to complete. Gives up (returns false) after
+// kWaitLimitNs of wall time, or at once when *abort is set (another warp of the
+// CTA has given up already).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          const volatile int* abort = nullptr) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-  return false;
+    if (abort && *abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
 }
 
-// 3-D tiled TMA load global -> shared, completion counted on `bar` (bytes).
-// Coordinates are innermost first. Out-of-range boxes are zero-filled.
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t y, int32_t z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
-      : "memory");
+// First failure of a launch: where it happened and the state there, written
+// once (words: site, then up to 7 values) to the diagnostic words.
+__device__ __forceinline__ void record_failure(int32_t* diag, int32_t site, int32_t v0,
+                                               int32_t v1, int32_t v2, int32_t v3, int32_t v4,
+                                               int32_t v5, int32_t v6) {
+  if (!diag || atomicCAS(diag, 0, site) != 0) return;
+  diag[1] = v0; diag[2] = v1; diag[3] = v2; diag[4] = v3;
+  diag[5] = v4; diag[6] = v5; diag[7] = v6;
 }
 
-// Same, with an L2 cache-eviction policy (e.g. evict-first for streamed data).
-__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                                 int32_t x, int32_t y, int32_t z,
-                                                 uint64_t policy) {
+// 4-D tiled TMA load global -> shared with an L2 cache-eviction policy,
+// completion counted on `bar` in bytes. Coordinates are innermost first;
+// boxes reaching outside the tensor are zero-filled there.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3,
+                                            uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)),
-      "l"(policy)
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(smem_addr(bar)), "l"(policy)
       : "memory");
 }
 

@@ -24,6 +24,9 @@ __global__ void __launch_bounds__(256)
                    const int32_t* __restrict__ slots, int32_t num_tokens, int32_t hkv,
                    int64_t pool_slots, int32_t* err) {
   constexpr int CPR = D / 8;  // 16-byte chunks per head row
+  // The next kernel may be scheduled now; one that reads the cache waits for
+  // this grid's completion (griddepcontrol.wait) before it does.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t per_token = static_cast<int64_t>(hkv) * CPR;
   if (i >= num_tokens * per_token) return;
@@ -47,6 +50,7 @@ __global__ void __launch_bounds__(256)
                        int64_t pool_slots, const float* __restrict__ k_scale,
                        const float* __restrict__ v_scale, int32_t* err) {
   constexpr int CPR = D / 8;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t per_token = static_cast<int64_t>(hkv) * CPR;
   if (i >= num_tokens * per_token) return;

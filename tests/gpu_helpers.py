@@ -81,10 +81,18 @@ class GpuStep:
                              v_scale=self.vs)
 
     def decode(self, partition_tokens=None, workspace=None):
-        p = self.sp.partition_tokens if partition_tokens is None else partition_tokens
-        return pk.decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, self.max_ctx,
-                         self.sp.scale, k_scale=self.ks, v_scale=self.vs, partition_tokens=p,
-                         workspace=workspace)
+        """One decode; afterwards the workspace's error word must be clear (a
+        table error or a pipeline wait that gave up raises PagedError)."""
+        sp = self.sp
+        p = sp.partition_tokens if partition_tokens is None else partition_tokens
+        if workspace is None:
+            workspace = pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads,
+                                            sp.head_dim, sp.block_size, self.max_ctx, p)
+        out = pk.decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, self.max_ctx,
+                        sp.scale, k_scale=self.ks, v_scale=self.vs, partition_tokens=p,
+                        workspace=workspace)
+        pk.decode_check(workspace)
+        return out
 
     def out_f64(self) -> np.ndarray:
         return self.out.double().cpu().numpy()
