@@ -95,7 +95,7 @@ struct Plan {
   int32_t max_parts;         // 1 = single pass
 };
 
-constexpr int32_t kMaxParts = 1024;  // partitions per sequence the decode kernel handles
+constexpr int32_t kMaxParts = 65535;  // partitions per sequence (grid z extent)
 
 Plan make_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
                int32_t max_context_len, int32_t requested) {
@@ -128,28 +128,19 @@ Plan make_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
   return p;
 }
 
-// Workspace layout: [header 256 B: error word, work counter, unit total]
-// [slice starts, max_parts+1 int32] [sequence order, S int2]
-// then, with partitions: [arrival counters, S*Hkv int32]
-// [partial (m, l), S*H*max_parts float2] [partial o, S*H*max_parts*D float].
+// Workspace layout: [header 256 B: error word, failure record] then, with
+// partitions: [partial (m, l), S*H*max_parts float2] [partial o, S*H*max_parts*D float].
 struct Layout {
-  size_t slice, order, arrive, ml, o, total;
+  size_t ml, o, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-Layout layout_for(const Plan& p, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
-                  int32_t head_dim) {
+Layout layout_for(const Plan& p, int32_t num_seqs, int32_t num_heads, int32_t head_dim) {
   Layout l{};
   size_t at = kHeaderBytes;
-  l.slice = at;
-  at = align256(at + 4 * static_cast<size_t>(p.max_parts + 1));
-  l.order = at;
-  at = align256(at + 8 * static_cast<size_t>(num_seqs));
   if (p.max_parts > 1) {
     const size_t rows = static_cast<size_t>(num_seqs) * num_heads * p.max_parts;
-    l.arrive = at;
-    at = align256(at + 4 * static_cast<size_t>(num_seqs) * num_kv_heads);
     l.ml = at;
     at = align256(at + rows * sizeof(float2));
     l.o = at;
@@ -221,7 +212,8 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int3
       max_context_len < 0)
     return 0;
   Plan p = make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
-  return layout_for(p, num_seqs, num_heads, num_kv_heads, head_dim).total;
+  (void)num_kv_heads;
+  return layout_for(p, num_seqs, num_heads, head_dim).total;
 }
 
 PA_API pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_stream_t stream) {
@@ -242,9 +234,7 @@ PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream) {
   if (e == cudaSuccess) e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && word != 0) e = cudaMemset(workspace, 0, 64);  // error + failure record
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode_check: %s", cudaGetErrorString(e));
-  if (word & (kErrWaitTimeout | kErrBadPlan))
-    return fail(PA_ERR_CUDA, "decode: %s", (word & kErrBadPlan) ? "a work unit outside the plan"
-                                                                : "a pipeline wait timed out");
+  if (word & kErrWaitTimeout) return fail(PA_ERR_CUDA, "decode: a pipeline wait timed out");
   if (word & (kErrBadBlockId | kErrContextClipped))
     return fail(PA_ERR_BAD_TABLE, "decode: %s%s",
                 (word & kErrBadBlockId) ? "block-table entry outside the pool; " : "",
@@ -295,10 +285,10 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
 
   const Plan plan =
       make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
-  if (plan.max_parts > kMaxParts || num_kv_heads > 65535)
-    return fail(PA_ERR_UNSUPPORTED, "decode: %d partitions / %d kv-heads exceed the plan",
-                plan.max_parts, num_kv_heads);
-  const Layout lay = layout_for(plan, num_seqs, num_heads, num_kv_heads, head_dim);
+  if (num_seqs > 65535 || plan.max_parts > kMaxParts)
+    return fail(PA_ERR_UNSUPPORTED, "decode: %d sequences x %d partitions exceed the grid",
+                num_seqs, plan.max_parts);
+  const Layout lay = layout_for(plan, num_seqs, num_heads, head_dim);
   const size_t need = lay.total;
   if (workspace_bytes < need)
     return fail(PA_ERR_INVALID_ARG, "decode: workspace %zu bytes < %zu needed", workspace_bytes,
@@ -322,12 +312,8 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
   a.v_scale = v_scale;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.err = reinterpret_cast<int32_t*>(ws) + kWordError;
-  a.counters = reinterpret_cast<int32_t*>(ws);
   a.diag = reinterpret_cast<int32_t*>(ws) + kWordDiag;
-  a.slice_start = reinterpret_cast<const int32_t*>(ws + lay.slice);
-  a.order = reinterpret_cast<const int2*>(ws + lay.order);
   if (plan.max_parts > 1) {
-    a.arrive = reinterpret_cast<int32_t*>(ws + lay.arrive);
     a.ws_ml = reinterpret_cast<float2*>(ws + lay.ml);
     a.ws_o = reinterpret_cast<float*>(ws + lay.o);
   }
@@ -341,30 +327,15 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
   a.partition_blocks = plan.partition_blocks;
   a.max_parts = plan.max_parts;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.num_sms = sm_count();
   a.block_size = block_size;
-
-  PlanArgs pa{};
-  pa.context_lens = context_lens;
-  pa.err = a.err;
-  pa.counters = a.counters;
-  pa.slice_start = reinterpret_cast<int32_t*>(ws + lay.slice);
-  pa.order = reinterpret_cast<int2*>(ws + lay.order);
-  pa.arrive = a.arrive;
-  pa.num_seqs = num_seqs;
-  pa.num_kv_heads = num_kv_heads;
-  pa.block_size = block_size;
-  pa.partition_blocks = plan.partition_blocks;
-  pa.max_parts = plan.max_parts;
-  pa.ctx_limit = a.ctx_limit;
 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   DecodeFn fn = nullptr;
   if (q_dtype == PA_F16) fn = fp8 ? decode_f16_e4m3 : decode_f16_f16;
   else fn = fp8 ? decode_bf16_e4m3 : decode_bf16_bf16;
-  st = cuda_status(launch_plan(pa, cs), "decode plan");
-  if (st != PA_OK) return st;
-  return cuda_status(fn(a, kmap, vmap, head_dim, group, cs), "decode");
+  st = cuda_status(fn(a, kmap, vmap, head_dim, group, cs), "decode");
+  if (st != PA_OK || plan.max_parts <= 1) return st;
+  return cuda_status(launch_reduce(a, q_dtype, head_dim, cs), "decode combine");
 }
 
 }  // extern "C"

@@ -15,21 +15,16 @@ enum : int32_t {
   kErrContextClipped = 2,  // a context length above what the launch covers
   kErrWaitTimeout = 4,     // a pipeline wait gave up (never expected)
   kErrBadSlot = 8,         // reshape_and_cache: a slot outside the pool
-  kErrBadPlan = 16,        // a work unit outside the plan (never expected)
 };
 
 // Failure sites recorded in the diagnostic words.
 enum : int32_t {
-  kSiteSlotFree = 1,    // scheduler: unit slot never released
-  kSiteUnit = 2,        // consumer: next unit never published
-  kSiteUnitAhead = 3,   // consumer issue cursor: a later unit never published
-  kSiteTile = 4,        // consumer: a tile's loads never completed
-  kSiteBadUnit = 5,     // scheduler: a ticket decoded to an impossible unit
+  kSiteTile = 4,        // a tile's loads never completed
 };
 
-// Words of the workspace header (int32): the error word and the counters of
-// one decode launch.
-enum : int { kWordError = 0, kCounterWork = 1, kCounterTotal = 2, kWordDiag = 8 };
+// Words of the workspace header (int32): the error word and, from kWordDiag,
+// the record of the first failure of a launch.
+enum : int { kWordError = 0, kWordDiag = 8 };
 
 
 struct DecodeArgs {
@@ -42,11 +37,7 @@ struct DecodeArgs {
   float* ws_o;                  // [S, H, max_parts, D] partial outputs (split mode)
   float2* ws_ml;                // [S, H, max_parts] (running max, sum) in log2 units
   int32_t* err;                 // error word (bits of the kErr* enum)
-  int32_t* counters;            // header words: work counter, total units
   int32_t* diag;                // header words kWordDiag..+7: first failure record
-  const int32_t* slice_start;   // [max_parts + 1] units before each partition slice
-  const int2* order;            // [S] (sequence, blocks), longest first
-  int32_t* arrive;              // [S * Hkv] partials written so far (split mode)
   int64_t num_blocks;
   int32_t max_blocks_per_seq;
   int32_t ctx_limit;            // min(max_context_len, max_blocks_per_seq * block_size)
@@ -56,19 +47,7 @@ struct DecodeArgs {
   int32_t partition_blocks;     // blocks per partition (single pass: covers max context)
   int32_t max_parts;            // partitions per sequence in the launch (1 = single pass)
   float scale_log2;             // softmax scale * log2(e)
-  int32_t num_sms;              // SMs of the device (persistent grid size)
   int32_t block_size;           // tokens per cache block (a multiple of 16)
-};
-
-// Arguments of the plan kernel (decode_plan.cu).
-struct PlanArgs {
-  const int32_t* context_lens;
-  int32_t* err;
-  int32_t* counters;
-  int32_t* slice_start;
-  int2* order;
-  int32_t* arrive;  // null in single-pass mode
-  int32_t num_seqs, num_kv_heads, block_size, partition_blocks, max_parts, ctx_limit;
 };
 
 // Per (q dtype, cache dtype) dispatchers, defined in decode_<q>_<c>.cu.
@@ -85,7 +64,7 @@ cudaError_t decode_f16_e4m3(const DecodeArgs&, const CUtensorMap&, const CUtenso
 cudaError_t decode_bf16_e4m3(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int, int,
                              cudaStream_t);
 
-cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream);
+cudaError_t launch_reduce(const DecodeArgs& a, int q_dtype, int head_dim, cudaStream_t stream);
 
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
                                      void* value_cache, const int32_t* slot_mapping,

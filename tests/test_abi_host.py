@@ -183,8 +183,8 @@ def test_reshape_rejects_bad_arguments():
 
 
 def test_workspace_sizes_and_partition_plan():
-    # single pass: header, plan slices and sequence order only
-    assert 256 < pk.decode_workspace_size(4, 4, 4, 64, 16, 100, 0) <= 1024
+    # single pass: only the 256-byte header (error word and failure record)
+    assert pk.decode_workspace_size(4, 4, 4, 64, 16, 100, 0) == 256
     assert pk.decode_partition_tokens(4, 4, 4, 64, 16, 100, 0) >= 100
     # forced partitions of 512 tokens over 2048: 4 partials per (seq, head)
     n = pk.decode_workspace_size(32, 32, 32, 128, 16, 2048, 512)
