@@ -233,6 +233,28 @@ def run_reference(args, sp, st):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------- rank logic
+
+def rank_seed(sp: wl.Spec, rank: int) -> int:
+    """Each rank decodes its own batch of the same shape (weak scaling)."""
+    return sp.seed + 97 * rank
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise maximum over all ranks (the slowest rank sets the time)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput_gbs(world: int, bytes_per_rank: int, ms: float) -> float:
+    """Whole-job GB/s: the bytes all ranks processed over the slowest rank's time."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def main():
@@ -257,7 +279,7 @@ def main():
                                 device_id=dev)
 
     part = sp.partition_tokens if args.partition < 0 else args.partition
-    sp_r = dataclasses.replace(sp, seed=sp.seed + 97 * rank)
+    sp_r = dataclasses.replace(sp, seed=rank_seed(sp, rank))
     d = wl.device_data(sp_r, st, device=dev)
     slots = pk.build_slot_mapping(st.block_tables, st.positions, sp.block_size)
     bt = torch.from_numpy(st.block_tables).to(dev)
@@ -349,17 +371,13 @@ def main():
         e2e = {"ms_per_step": e2e_ms, "h2d": h2d, "d2h": d2h}
 
     # max over ranks
-    step_ms = elapsed_ms / args.steps
-    vals = torch.tensor([step_ms, dec_ms, e2e["ms_per_step"] if e2e else 0.0],
-                        dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    step_ms, dec_ms, e2e_ms = vals.tolist()
+    step_ms, dec_ms, e2e_ms = max_over_ranks(
+        [elapsed_ms / args.steps, dec_ms, e2e["ms_per_step"] if e2e else 0.0], world, dev)
 
     if rank == 0:
         dbytes = wl.decode_bytes(sp, st)
         peak, peak_kind = measured_peaks()
-        value = world * dbytes / (step_ms * 1e-3) / 1e9
+        value = job_throughput_gbs(world, dbytes, step_ms)
         achieved = dbytes / (dec_ms * 1e-3) / 1e9
         traffic = recorded_traffic(sp.name)
         line = {
@@ -387,7 +405,7 @@ def main():
             "clocks": clocks,
         }
         if e2e:
-            line["e2e"] = {"value": round(world * dbytes / (e2e_ms * 1e-3) / 1e9, 2),
+            line["e2e"] = {"value": round(job_throughput_gbs(world, dbytes, e2e_ms), 2),
                            "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
                            "d2h_bytes_per_step": e2e["d2h"],
                            "ms_per_step": round(e2e_ms, 5)}
