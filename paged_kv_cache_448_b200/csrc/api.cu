@@ -53,20 +53,23 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // Tensor map over a cache viewed as [rows = num_blocks*block_size][num_kv_heads]
 // [segments][segment elements] (a row of head_dim elements cut into <=128-byte
-// segments): one box = 16 rows of one kv-head, whole rows, swizzled per segment.
+// segments): one box = 16 rows of one kv-head, whole rows, swizzled per segment,
+// stored in shared memory segment-major (all rows' first segment, then the next).
 pa_status encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks,
                            int32_t block_size, int32_t hkv, int32_t head_dim, int elem) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int row_bytes = head_dim * elem;
   const int seg = box_bytes(row_bytes);
+  // dims: elements of a segment, token slots, kv-heads, segments of a row.
+  // The box is one kv-head x 16 slots x all segments, segment outermost.
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(seg / elem),
-                        static_cast<cuuint64_t>(row_bytes / seg), static_cast<cuuint64_t>(hkv),
-                        static_cast<cuuint64_t>(num_blocks) * block_size};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(seg), static_cast<cuuint64_t>(row_bytes),
-                           static_cast<cuuint64_t>(row_bytes) * hkv};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(seg / elem),
-                       static_cast<cuuint32_t>(row_bytes / seg), 1u, 16u};
+                        static_cast<cuuint64_t>(num_blocks) * block_size,
+                        static_cast<cuuint64_t>(hkv), static_cast<cuuint64_t>(row_bytes / seg)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(row_bytes) * hkv,
+                           static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(seg)};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(seg / elem), 16u, 1u,
+                       static_cast<cuuint32_t>(row_bytes / seg)};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   const CUtensorMapSwizzle swz = seg == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                : seg == 64  ? CU_TENSOR_MAP_SWIZZLE_64B

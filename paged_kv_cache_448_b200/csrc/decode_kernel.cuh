@@ -18,7 +18,7 @@
 // Tiles are 16 tokens of one kv-head (a 32-token block is two tiles). Each of
 // the NW warps owns every NW-th tile of the unit and runs its own R-deep ring:
 // its lane 0 issues one 4-D TMA box for the K tile and one for the V tile
-// (whole rows, swizzled) and the warp waits on the stage's mbarrier. No
+// (whole rows, segment-major, swizzled) and the warp waits on the stage's mbarrier. No
 // barrier is shared between warps until the final merge. Every wait is bounded
 // by wall time; a wait that gives up makes the CTA stop and report.
 #pragma once
@@ -39,8 +39,12 @@ constexpr int kTileRows = 16;         // tokens per pipeline tile
 constexpr int kMaxUnitBlocks = 1024;  // blocks of one work unit (ids staged in shared memory)
 
 // Shared-memory geometry of one staged K (or V) tile: kTileRows token rows of
-// one kv-head, RB bytes each, stored back to back; the TMA swizzles the 16-byte
-// chunks inside every BOXB-byte segment (128B or 64B pattern).
+// one kv-head, RB bytes each. A row longer than the swizzle span (BOXB = 128
+// or 64 bytes) is split into NBOX segments, and the TMA box puts the segment
+// outermost: all rows' segment 0, then all rows' segment 1. Consecutive
+// tokens of one segment thus sit in consecutive BOXB-byte lines, whose 16-byte
+// chunks the TMA swizzles (128B or 64B pattern), so 8 rows read at the same
+// logical column fall in 8 different bank groups.
 template <class CF, int D_>
 struct Tile {
   static constexpr int D = D_, BS = kTileRows;
@@ -52,7 +56,7 @@ struct Tile {
   static constexpr int BYTES = BS * RB;
   // Byte offset of logical byte `o` of row `r`.
   static __device__ __forceinline__ uint32_t off(int r, int o) {
-    const int lin = r * RB + o;
+    const int lin = ((o / BOXB) * BS + r) * BOXB + o % BOXB;
     return lin ^ ((lin >> 3) & SWZ);
   }
 };
@@ -143,8 +147,8 @@ __global__ void __launch_bounds__(GridCfg<Consumer>::NW * 32)
     const int32_t row0 = bid >= 0 ? bid * a.block_size + (t % tpb) * TR : -TR;
     uint8_t* kt = my_stages + stage * STAGE;
     mbar_arrive_expect_tx(&my_bars[stage], STAGE);
-    tma_load_4d(kt, &kmap, &my_bars[stage], 0, 0, kvh, row0, policy);
-    tma_load_4d(kt + T::BYTES, &vmap, &my_bars[stage], 0, 0, kvh, row0, policy);
+    tma_load_4d(kt, &kmap, &my_bars[stage], 0, row0, kvh, 0, policy);
+    tma_load_4d(kt + T::BYTES, &vmap, &my_bars[stage], 0, row0, kvh, 0, policy);
   };
   if (lane == 0) {
     for (int k = 0; k < min(R, my_count); ++k) issue(k);
