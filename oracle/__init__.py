@@ -15,7 +15,12 @@ Functions mirror the pages' problem statement:
 * ``slot_mapping`` — the address translation of [P3] "Paged KVCache：大模型推理
   显存管理优化方案" §2.3, page size counted in tokens.
 * ``BlockManager`` (``oracle.block_manager``) — the free list of [P2] §2.2 with
-  the reference counts of [P4] "大模型推理KV Cache内存管理与PagedAttention分页显存实战".
+  the reference counts of [P4] "大模型推理KV Cache内存管理与PagedAttention分页显存实战",
+  and copy-on-write of a shared block before a write.
+* ``copy_blocks`` — whole-block copies between or within caches: the private
+  copy of a shared block ([P4]'s reference-counted sharing) and the migration
+  of blocks between GPU memory and host memory ([P3] §5, Hybrid Cache; [P4]'s
+  ``swap_space``).
 
 Parity status: every function here is pinned by the ``-m "not gpu"`` tests
 (format decoders exhaustively against numpy/torch, the E4M3 encoder against a
@@ -207,3 +212,22 @@ def round_to(values: np.ndarray, dt: str) -> np.ndarray:
     fn = {"f16": lib.orc_encode_f16, "bf16": lib.orc_encode_bf16}[dt]
     flat = np.asarray(values, dtype=np.float64).reshape(-1)
     return np.array([fn(float(v)) for v in flat], dtype=np.uint16).reshape(np.shape(values))
+
+
+def copy_blocks(src_cache: np.ndarray, dst_cache: np.ndarray, pairs) -> None:
+    """Copy whole blocks: ``dst_cache[d] = src_cache[s]`` for every (s, d) in
+    ``pairs`` (block index along axis 0; the bytes are copied unchanged).
+
+    The destinations must be distinct, and when both caches are the same array
+    no destination may also be a source (each pair then reads a block no pair
+    writes, so the order of the copies does not matter). Modifies ``dst_cache``.
+    """
+    pairs = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
+    dsts = pairs[:, 1].tolist()
+    assert len(set(dsts)) == len(dsts), "duplicate destination block"
+    if src_cache is dst_cache:
+        assert not set(dsts) & set(pairs[:, 0].tolist()), "a destination is also a source"
+    for s, d in pairs.tolist():
+        assert 0 <= s < src_cache.shape[0] and 0 <= d < dst_cache.shape[0], "block id out of range"
+        dst_cache[d] = src_cache[s].copy()
+

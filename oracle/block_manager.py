@@ -64,5 +64,25 @@ class BlockManager:
             if self.refcount[b] == 0:
                 self.free_blocks.append(b)
 
+    def copy_on_write(self, block_id: int):
+        """Make ``block_id`` private to the holder that is about to write into it.
+
+        [P4] lets several block tables reference one physical block, with a
+        reference count for its lifetime, but says nothing about writing into
+        such a block. The reading taken here: a holder that must write into a
+        block with refcount > 1 first takes a fresh block (allocated like any
+        other: the head of the free list), moves its reference there and
+        copies the contents; a block with refcount 1 is written in place.
+        Returns ``(block_to_write, must_copy)``; on OutOfBlocks nothing changes.
+        """
+        b = int(block_id)
+        if not (0 <= b < self.num_blocks) or self.refcount[b] == 0:
+            raise ValueError("copy_on_write of a free or unknown block")
+        if self.refcount[b] == 1:
+            return b, False
+        (new,) = self.allocate(1)
+        self.refcount[b] -= 1
+        return new, True
+
     def num_free(self) -> int:
         return len(self.free_blocks)

@@ -536,6 +536,108 @@ def test_block_manager_refcounted_sharing():
     assert bm.num_free() == 4
 
 
+def test_block_manager_copy_on_write():
+    bm = BlockManager(5, initial_free_order=[3, 0, 4, 1, 2])
+    a, b = bm.allocate(2)                  # 3, 0
+    assert bm.copy_on_write(a) == (a, False)          # sole holder writes in place
+    bm.share(b); bm.share(b)               # three holders
+    new, copy = bm.copy_on_write(b)
+    assert (new, copy) == (4, True)        # head of the free list
+    assert bm.refcount[b] == 2 and bm.refcount[new] == 1 and bm.free_blocks == [1, 2]
+    bm.allocate(2)
+    with pytest.raises(OutOfBlocks):
+        bm.copy_on_write(b)                # nothing changes on failure
+    assert bm.refcount[b] == 2 and bm.free_blocks == []
+    with pytest.raises(ValueError):
+        BlockManager(2).copy_on_write(0)   # a free block has no holder
+
+
+def test_copy_blocks_hand_example():
+    src = np.arange(4 * 3, dtype=np.uint16).reshape(4, 3)
+    dst = np.full((5, 3), 7, np.uint16)
+    oracle.copy_blocks(src, dst, [(0, 2), (3, 0)])
+    assert dst.tolist() == [[9, 10, 11], [7, 7, 7], [0, 1, 2], [7, 7, 7], [7, 7, 7]]
+    with pytest.raises(AssertionError):
+        oracle.copy_blocks(src, src, [(0, 1), (1, 2)])   # 1 is read and written
+    with pytest.raises(AssertionError):
+        oracle.copy_blocks(src, dst, [(0, 1), (2, 1)])   # two writers of block 1
+
+
+def _manager_for(st, sp):
+    """A BlockManager driven through the same allocations as the workload
+    structure (prefix blocks once per group, then shared by every member)."""
+    bm = BlockManager(st.num_blocks, initial_free_order=st.free_order)
+    tables = []
+    pblk = sp.prefix_tokens // sp.block_size
+    per = sp.num_seqs // sp.shared_groups
+    for g in range(sp.shared_groups):
+        prefix = bm.allocate(pblk)
+        for _ in range(per - 1):
+            for b in prefix:
+                bm.share(b)
+        for j in range(per):
+            s = g * per + j
+            tables.append(prefix + bm.allocate(len(st.seq_block_ids[s]) - pblk))
+    return bm, tables
+
+
+def test_copy_on_write_gives_the_writer_a_private_block():
+    """[P4]: a physical block may back the logical blocks of several
+    sequences. After copy-on-write of one shared prefix block for one
+    sequence and a write into the copy, every other sequence's output is
+    unchanged bit for bit, and so is the writer's until the write."""
+    sp, st, hd = _small_workload(5)
+    bm, tables = _manager_for(st, sp)
+    assert [t for t in tables] == [list(x) for x in st.seq_block_ids]
+    assert bm.refcount == st.refcounts.tolist()
+    base = _decode(sp, st, hd)
+    s0, j = 5, 2                                   # second member of group 1, prefix block 2
+    old = int(st.block_tables[s0, j])
+    free_before = bm.num_free()
+    new, must_copy = bm.copy_on_write(old)
+    assert must_copy and bm.refcount[old] == 3 and bm.num_free() == free_before - 1
+    kc, vc = hd.key_cache.copy(), hd.value_cache.copy()
+    oracle.copy_blocks(kc, kc, [(old, new)])
+    oracle.copy_blocks(vc, vc, [(old, new)])
+    table = st.block_tables.copy()
+    table[s0, j] = new
+    assert np.array_equal(_decode(sp, st, hd, table=table, kc=kc, vc=vc), base)
+    # overwrite token 3 of the copy (e4m3 codes) for s0 only
+    kc[new, 3] = 0x38                              # 1.0 in every dimension
+    vc[new, 3] = 0xB8                              # -1.0
+    after = _decode(sp, st, hd, table=table, kc=kc, vc=vc)
+    others = [s for s in range(sp.num_seqs) if s != s0]
+    assert np.array_equal(after[others], base[others])
+    assert not np.array_equal(after[s0], base[s0])
+
+
+def test_swap_out_and_back_in_keeps_outputs():
+    """[P3] §5: blocks migrate to host memory and back. A sequence whose
+    blocks go to a host pool, whose device blocks are then overwritten, and
+    which comes back into other device blocks (table rewritten) attends
+    exactly as before."""
+    sp, st, hd = _small_workload(3)
+    base = _decode(sp, st, hd)
+    s0 = int(np.argmax(sp.context_lens))
+    ids = list(st.seq_block_ids[s0])
+    others = {b for s, x in enumerate(st.seq_block_ids) if s != s0 for b in x}
+    host_k = np.zeros((len(ids) + 2,) + hd.key_cache.shape[1:], hd.key_cache.dtype)
+    host_v = np.zeros_like(host_k)
+    kc, vc = hd.key_cache.copy(), hd.value_cache.copy()
+    out_pairs = [(b, i + 2) for i, b in enumerate(ids)]
+    oracle.copy_blocks(kc, host_k, out_pairs)
+    oracle.copy_blocks(vc, host_v, out_pairs)
+    kc[ids] = 0x7FC0; vc[ids] = 0x7FC0             # reused by someone else (NaN codes)
+    targets = [b for b in np.random.default_rng(2).permutation(st.num_blocks).tolist()
+               if b not in others][:len(ids)]
+    in_pairs = [(i + 2, t) for i, t in enumerate(targets)]
+    oracle.copy_blocks(host_k, kc, in_pairs)
+    oracle.copy_blocks(host_v, vc, in_pairs)
+    table = st.block_tables.copy()
+    table[s0, :len(ids)] = targets
+    assert np.array_equal(_decode(sp, st, hd, table=table, kc=kc, vc=vc), base)
+
+
 def test_blocks_for_prompt_and_waste_bound():
     facts = load_golden("page_facts.json")
     bs = facts["block_size_tokens"]["value"]
