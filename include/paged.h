@@ -215,6 +215,37 @@ PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream);
  */
 PA_API pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_stream_t stream);
 
+/*
+ * Copy whole blocks: for each pair i, block block_pairs[2i] of the source
+ * caches is copied byte for byte to block block_pairs[2i+1] of the destination
+ * caches (K, and V when the value caches are given). One block of one cache is
+ * block_bytes contiguous bytes (block_size * num_kv_heads * head_dim * elem).
+ * Two uses:
+ *  - copy-on-write of a shared block (source and destination in the same
+ *    cache), after pa_alloc_copy_on_write; [P4] shares prefix blocks among
+ *    requests under a reference count;
+ *  - migration between GPU memory and a host pool ([P3] "Paged KVCache：大模型
+ *    推理显存管理优化方案" §5 Hybrid Cache: GPU memory, then CPU memory, then
+ *    disk; [P4]'s swap_space): one side may be pinned host memory
+ *    (cudaHostAlloc / cudaHostRegister), which the kernel reads or writes through
+ *    its mapped device address. Pageable host memory is rejected.
+ * src_key_cache, src_value_cache  [num_src_blocks, ...] device or pinned host
+ * dst_key_cache, dst_value_cache  [num_dst_blocks, ...] device or pinned host
+ *                 (value caches: both NULL to copy the key cache only)
+ * block_pairs     int32 [num_pairs][2], device or pinned host; destination ids
+ *                 distinct; with the same cache on both sides no destination
+ *                 may also be a source (else the result is unspecified).
+ * error_word      optional device int32: a pair with an id outside its pool is
+ *                 skipped (nothing is read or written for it) and bit 1 is set.
+ * block_bytes must be a positive multiple of 16 and every pointer 16-byte
+ * aligned (4 for block_pairs / error_word). Asynchronous on `stream`.
+ */
+PA_API pa_status pa_copy_blocks(const void* src_key_cache, const void* src_value_cache,
+                                void* dst_key_cache, void* dst_value_cache,
+                                const int32_t* block_pairs, int32_t num_pairs, int64_t block_bytes,
+                                int64_t num_src_blocks, int64_t num_dst_blocks,
+                                int32_t* error_word, pa_stream_t stream);
+
 /* ------------------------------------------------------------------------- */
 /* Host block allocator (no device memory; produces integer tables only).      */
 /* ------------------------------------------------------------------------- */
@@ -240,6 +271,16 @@ PA_API pa_status pa_alloc_share(pa_alloc* a, int32_t id);
  * free or listed more often than its refcount gives PA_ERR_INVALID_ARG and
  * changes nothing). */
 PA_API pa_status pa_alloc_free(pa_alloc* a, const int32_t* ids, int32_t n);
+/* Before a write into block `id`: with refcount 1, *id_out = id and
+ * *must_copy = 0 (write in place). With refcount > 1 (shared), a fresh block
+ * is taken from the head of the free list, one reference moves to it,
+ * *id_out = that block and *must_copy = 1: the caller copies the contents
+ * (pa_copy_blocks) and points its table entry at *id_out. The pages share
+ * blocks under a reference count ([P4]) but give no write rule; this is the
+ * reading taken. PA_ERR_OOM (nothing changes) when no block is free;
+ * PA_ERR_INVALID_ARG for a free or unknown id. */
+PA_API pa_status pa_alloc_copy_on_write(pa_alloc* a, int32_t id, int32_t* id_out,
+                                        int32_t* must_copy);
 PA_API int64_t pa_alloc_num_free(const pa_alloc* a);
 PA_API int64_t pa_alloc_num_blocks(const pa_alloc* a);
 /* Reference count of a block (0 = free), -1 for an id out of range. */

@@ -22,7 +22,8 @@ from ._native import PagedError, check
 
 __all__ = ["reshape_and_cache", "decode", "decode_noalloc", "decode_workspace",
            "decode_workspace_size",
-           "decode_partition_tokens", "decode_check", "BlockAllocator", "build_block_table",
+           "decode_partition_tokens", "decode_check", "copy_blocks", "BlockAllocator",
+           "build_block_table",
            "build_slot_mapping", "PagedError", "dtype_code"]
 
 
@@ -131,6 +132,30 @@ def _i32(a) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=np.int32)
 
 
+def copy_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache, block_pairs, *,
+                error_word=None, stream=None):
+    """Copy whole blocks src[pairs[i, 0]] -> dst[pairs[i, 1]] (pa_copy_blocks).
+
+    Caches are [num_blocks, ...] tensors on the GPU or in pinned host memory
+    (value caches may both be None); block_pairs is an int32 [n, 2] tensor on
+    the GPU or pinned. A block is one row along axis 0 of each cache.
+    """
+    n = int(block_pairs.shape[0]) if block_pairs.dim() == 2 else 0
+    if block_pairs.dim() != 2 or block_pairs.shape[1] != 2 or not block_pairs.is_contiguous():
+        raise ValueError("block_pairs must be a contiguous int32 [n, 2] tensor")
+    bb = src_key_cache[0].numel() * src_key_cache.element_size()
+    if dst_key_cache[0].numel() * dst_key_cache.element_size() != bb:
+        raise ValueError("source and destination blocks differ in size")
+    if src_value_cache is not None and (
+            src_value_cache[0].numel() * src_value_cache.element_size() != bb or
+            dst_value_cache[0].numel() * dst_value_cache.element_size() != bb):
+        raise ValueError("value blocks differ in size from key blocks")
+    check(_native.lib().pa_copy_blocks(
+        _ptr(src_key_cache), _ptr(src_value_cache), _ptr(dst_key_cache), _ptr(dst_value_cache),
+        _ptr(block_pairs), n, bb, src_key_cache.shape[0], dst_key_cache.shape[0],
+        _ptr(error_word), _stream_handle(stream)))
+
+
 class BlockAllocator:
     """Host free list with refcounts (pa_alloc_*)."""
 
@@ -161,6 +186,14 @@ class BlockAllocator:
     def free(self, ids) -> None:
         a = _i32(ids)
         check(self._lib.pa_alloc_free(self._h, a.ctypes.data if a.size else None, a.size))
+
+    def copy_on_write(self, block_id: int):
+        """(block to write, must_copy): a shared block is replaced by a fresh one
+        that the caller fills with copy_blocks (pa_alloc_copy_on_write)."""
+        out, copy = ctypes.c_int32(), ctypes.c_int32()
+        check(self._lib.pa_alloc_copy_on_write(self._h, int(block_id), ctypes.byref(out),
+                                               ctypes.byref(copy)))
+        return int(out.value), bool(copy.value)
 
     @property
     def num_free(self) -> int:

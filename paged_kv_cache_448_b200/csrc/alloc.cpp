@@ -96,6 +96,31 @@ PA_API pa_status pa_alloc_free(pa_alloc* a, const int32_t* ids, int32_t n) {
   return PA_OK;
 }
 
+// A holder about to write into a block with refcount > 1 moves its reference
+// to a fresh block (the head of the free list) and copies the contents there;
+// with refcount 1 it writes in place. The pages give refcounted sharing but no
+// write rule: this is the plainest reading that keeps other holders intact.
+PA_API pa_status pa_alloc_copy_on_write(pa_alloc* a, int32_t id, int32_t* id_out,
+                                        int32_t* must_copy) {
+  clear_error();
+  if (!a || !id_out || !must_copy) return fail(PA_ERR_INVALID_ARG, "alloc_copy_on_write: bad args");
+  if (id < 0 || static_cast<size_t>(id) >= a->refcount.size() || a->refcount[id] == 0)
+    return fail(PA_ERR_INVALID_ARG, "alloc_copy_on_write: block %d is not allocated", id);
+  if (a->refcount[id] == 1) {
+    *id_out = id;
+    *must_copy = 0;
+    return PA_OK;
+  }
+  if (a->free_list.empty()) return fail(PA_ERR_OOM, "Need 1 block, only 0 available");
+  const int32_t fresh = a->free_list.front();
+  a->free_list.pop_front();
+  a->refcount[fresh] = 1;
+  --a->refcount[id];
+  *id_out = fresh;
+  *must_copy = 1;
+  return PA_OK;
+}
+
 PA_API int64_t pa_alloc_num_free(const pa_alloc* a) {
   return a ? static_cast<int64_t>(a->free_list.size()) : -1;
 }

@@ -20,6 +20,11 @@ namespace {
 constexpr size_t kHeaderBytes = 256;          // error word + padding
 constexpr int32_t kMaxPartitionBlocks = 1024; // block ids staged in shared memory per CTA
 constexpr int32_t kMinAutoPartition = 256;    // tokens
+// Partitions of at most this many tokens run on the 2-warp CTA: six of them
+// per SM overlap their start-up (table read, first loads) and the end of
+// their unit better than three 4-warp CTAs (~7% on 512-token partitions of a
+// 64-sequence, 8-kv-head batch); longer units keep the 4-warp CTA.
+constexpr int32_t kNarrowTokens = 512;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -151,6 +156,27 @@ Layout layout_for(const Plan& p, int32_t num_seqs, int32_t num_heads, int32_t he
   }
   l.total = at;
   return l;
+}
+
+// The address kernels use for a buffer: device (or managed) memory as is;
+// pinned host memory through its mapped device address. Pageable host memory
+// has none and is rejected.
+pa_status device_view(const void* p, const void** out, const char* what) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(PA_ERR_INVALID_ARG, "copy_blocks: %s is not a CUDA-visible pointer", what);
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+    *out = p;
+    return PA_OK;
+  }
+  if (at.type == cudaMemoryTypeHost && at.devicePointer) {
+    *out = at.devicePointer;
+    return PA_OK;
+  }
+  return fail(PA_ERR_INVALID_ARG,
+              "copy_blocks: %s is pageable host memory (pin it, e.g. cudaHostAlloc)", what);
 }
 
 bool shape_supported(int32_t head_dim, int32_t block_size) {
@@ -336,9 +362,52 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
   DecodeFn fn = nullptr;
   if (q_dtype == PA_F16) fn = fp8 ? decode_f16_e4m3 : decode_f16_f16;
   else fn = fp8 ? decode_bf16_e4m3 : decode_bf16_bf16;
-  st = cuda_status(fn(a, kmap, vmap, head_dim, group, cs), "decode");
+  const int warps = plan.max_parts > 1 && plan.partition_tokens <= kNarrowTokens ? 2 : 4;
+  st = cuda_status(fn(a, kmap, vmap, head_dim, group, warps, cs), "decode");
   if (st != PA_OK || plan.max_parts <= 1) return st;
   return cuda_status(launch_reduce(a, q_dtype, head_dim, cs), "decode combine");
+}
+
+PA_API pa_status pa_copy_blocks(const void* src_key_cache, const void* src_value_cache,
+                                void* dst_key_cache, void* dst_value_cache,
+                                const int32_t* block_pairs, int32_t num_pairs, int64_t block_bytes,
+                                int64_t num_src_blocks, int64_t num_dst_blocks,
+                                int32_t* error_word, pa_stream_t stream) {
+  clear_error();
+  if (num_pairs < 0 || block_bytes <= 0 || block_bytes % 16 != 0 || num_src_blocks <= 0 ||
+      num_dst_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "copy_blocks: bad sizes (block_bytes a positive multiple of 16)");
+  if (!src_key_cache || !dst_key_cache || !block_pairs)
+    return fail(PA_ERR_INVALID_ARG, "copy_blocks: null pointer");
+  if ((src_value_cache == nullptr) != (dst_value_cache == nullptr))
+    return fail(PA_ERR_INVALID_ARG, "copy_blocks: give both value caches or neither");
+  if (!aligned(src_key_cache, 16) || !aligned(dst_key_cache, 16) ||
+      !aligned(src_value_cache, 16) || !aligned(dst_value_cache, 16) || !aligned(block_pairs, 4) ||
+      !aligned(error_word, 4))
+    return fail(PA_ERR_INVALID_ARG, "copy_blocks: misaligned pointer");
+  if (num_pairs == 0) return PA_OK;
+  const void* views[5] = {};
+  const void* ptrs[5] = {src_key_cache, dst_key_cache, src_value_cache, dst_value_cache,
+                         block_pairs};
+  const char* names[5] = {"src_key_cache", "dst_key_cache", "src_value_cache",
+                          "dst_value_cache", "block_pairs"};
+  for (int i = 0; i < 5; ++i) {
+    if (!ptrs[i]) continue;
+    pa_status st = device_view(ptrs[i], &views[i], names[i]);
+    if (st != PA_OK) return st;
+  }
+  int32_t* err = nullptr;
+  if (error_word) {
+    const void* v = nullptr;
+    pa_status st = device_view(error_word, &v, "error_word");
+    if (st != PA_OK) return st;
+    err = const_cast<int32_t*>(static_cast<const int32_t*>(v));
+  }
+  cudaError_t e = launch_copy_blocks(
+      views[0], views[2], const_cast<void*>(views[1]), const_cast<void*>(views[3]),
+      static_cast<const int32_t*>(views[4]), num_pairs, block_bytes, num_src_blocks,
+      num_dst_blocks, err, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e, "copy_blocks");
 }
 
 }  // extern "C"

@@ -51,18 +51,19 @@ struct DecodeArgs {
 };
 
 // Per (q dtype, cache dtype) dispatchers, defined in decode_<q>_<c>.cu.
-// Return cudaErrorNotSupported for a (head_dim, block_size, group) they lack.
+// `warps` is the CTA width (2 or 4 warps). Return cudaErrorNotSupported for a
+// (head_dim, group, width) they lack.
 using DecodeFn = cudaError_t (*)(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&,
-                                 int head_dim, int group, cudaStream_t);
+                                 int head_dim, int group, int warps, cudaStream_t);
 
 cudaError_t decode_f16_f16(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int, int,
-                           cudaStream_t);
+                           int, cudaStream_t);
 cudaError_t decode_bf16_bf16(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int, int,
-                             cudaStream_t);
+                             int, cudaStream_t);
 cudaError_t decode_f16_e4m3(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int, int,
-                            cudaStream_t);
+                            int, cudaStream_t);
 cudaError_t decode_bf16_e4m3(const DecodeArgs&, const CUtensorMap&, const CUtensorMap&, int, int,
-                             cudaStream_t);
+                             int, cudaStream_t);
 
 cudaError_t launch_reduce(const DecodeArgs& a, int q_dtype, int head_dim, cudaStream_t stream);
 
@@ -72,6 +73,11 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k
                                      int32_t block_size, int64_t num_blocks, int kv_dtype,
                                      int cache_dtype, const float* k_scale, const float* v_scale,
                                      int32_t* err, cudaStream_t stream);
+
+cudaError_t launch_copy_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                               const int32_t* pairs, int64_t num_pairs, int64_t block_bytes,
+                               int64_t num_src_blocks, int64_t num_dst_blocks, int32_t* err,
+                               int sm_count, cudaStream_t stream);
 
 // Box geometry shared by the host tensor-map encoder and the kernels: a row
 // of head_dim elements is cut into segments of at most 128 bytes (the widest

@@ -1,9 +1,9 @@
-// Decode kernels for query dtype F16, cache dtype E4M3 (all head_dim and query groups).
+// Decode kernels for query dtype F16, cache dtype E4M3 (all head_dim, query groups and CTA widths).
 #include "decode_dispatch.cuh"
 
 namespace paged {
 cudaError_t decode_f16_e4m3(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                        int head_dim, int group, cudaStream_t stream) {
-  return dispatch_decode<F16, E4M3>(a, kmap, vmap, head_dim, group, stream);
+                        int head_dim, int group, int warps, cudaStream_t stream) {
+  return dispatch_decode<F16, E4M3>(a, kmap, vmap, head_dim, group, warps, stream);
 }
 }  // namespace paged

@@ -61,25 +61,25 @@ struct Tile {
   }
 };
 
-// Per-CTA shape: NW warps with R-deep rings of ~64 KB in total, so that three
-// CTAs fit on an SM.
-template <class Consumer>
+// Per-CTA shape: NW warps whose R-deep rings take 16 KB per warp (64 KB for
+// the 4-warp CTA, so that three CTAs fit on an SM; six of the 2-warp CTA).
+template <class Consumer, int NW_>
 struct GridCfg {
   using T = typename Consumer::Tile;
   static constexpr int G = Consumer::G, D = T::D;
-  static constexpr int NW = 4;
+  static constexpr int NW = NW_;
   static constexpr int STAGE = 2 * T::BYTES;                 // K and V tiles
-  static constexpr int R_RAW = 65536 / (NW * STAGE);
+  static constexpr int R_RAW = 16384 / STAGE;
   static constexpr int R = R_RAW < 1 ? 1 : (R_RAW > 8 ? 8 : R_RAW);
   static constexpr int STAGES_BYTES = NW * R * STAGE;
   static_assert(NW * G * (D + 2) * 4 <= STAGES_BYTES, "merge buffer fits in the stages");
 };
 
-template <class Consumer>
-__global__ void __launch_bounds__(GridCfg<Consumer>::NW * 32)
+template <class Consumer, int NW_>
+__global__ void __launch_bounds__(NW_ * 32)
     paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap) {
-  using C = GridCfg<Consumer>;
+  using C = GridCfg<Consumer, NW_>;
   using T = typename Consumer::Tile;
   constexpr int D = T::D, G = Consumer::G, NW = C::NW, R = C::R, STAGE = C::STAGE;
   constexpr int TR = kTileRows;
@@ -259,15 +259,15 @@ cudaError_t launch_pdl(Kernel kern, dim3 grid, int threads, size_t smem, cudaStr
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <class Consumer>
+template <class Consumer, int NW>
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           cudaStream_t stream) {
-  using C = GridCfg<Consumer>;
+  using C = GridCfg<Consumer, NW>;
   if (a.partition_blocks > kMaxUnitBlocks || a.block_size % kTileRows != 0)
     return cudaErrorNotSupported;
   const size_t smem = 1024 + C::STAGES_BYTES + 8 * C::NW * C::R +
                       4 * static_cast<size_t>(a.partition_blocks);
-  auto kern = paged_decode_kernel<Consumer>;
+  auto kern = paged_decode_kernel<Consumer, NW>;
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(a.num_kv_heads, a.num_seqs, a.max_parts), C::NW * 32, smem,

@@ -46,7 +46,7 @@ def test_allocator_matches_oracle_model_on_random_ops():
         ref = BlockManager(nb, order)
         live = []                      # references held (block ids, with repeats)
         for _ in range(300):
-            op = rng.integers(0, 4)
+            op = rng.integers(0, 5)
             if op == 0:
                 n = int(rng.integers(0, 12))
                 try:
@@ -75,6 +75,18 @@ def test_allocator_matches_oracle_model_on_random_ops():
                 if free_ids:
                     with pytest.raises(pk.PagedError):
                         ours.free(free_ids)
+            elif op == 4 and live:
+                # copy-on-write of a held reference
+                i = int(rng.integers(0, len(live)))
+                try:
+                    expect = ref.copy_on_write(live[i])
+                except OutOfBlocks:
+                    with pytest.raises(pk.PagedError) as ei:
+                        ours.copy_on_write(live[i])
+                    assert ei.value.status == _native.PA_ERR_OOM
+                    continue
+                assert ours.copy_on_write(live[i]) == expect
+                live[i] = expect[0]
             assert ours.free_list() == ref.free_blocks
             assert ours.num_free == ref.num_free()
         for b in range(nb):
@@ -180,6 +192,24 @@ def test_reshape_rejects_bad_arguments():
     assert call(cdt=_native.PA_FP8_E4M3) == _native.PA_ERR_INVALID_ARG
     assert call(k=24) == _native.PA_ERR_INVALID_ARG
     assert call(T=0, k=None) == _native.PA_OK
+
+
+def test_copy_blocks_rejects_bad_arguments_before_launch():
+    lib = _native.lib()
+    P = 1 << 20                                 # any 16-byte aligned address; never touched
+    def call(src=P, sv=None, dst=P, dv=None, pairs=P, n=1, bb=4096, ns=4, nd=4, err=None):
+        return lib.pa_copy_blocks(src, sv, dst, dv, pairs, n, bb, ns, nd, err, None)
+    bad = _native.PA_ERR_INVALID_ARG
+    assert call(n=-1) == bad
+    assert call(bb=24) == bad                   # not a multiple of 16
+    assert call(bb=0) == bad
+    assert call(ns=0) == bad
+    assert call(src=None) == bad
+    assert call(pairs=None) == bad
+    assert call(sv=P) == bad                    # one value cache without the other
+    assert call(dst=P + 8) == bad               # misaligned
+    assert call(pairs=P + 2) == bad
+    assert call(n=0) == _native.PA_OK           # nothing to do, no device call
 
 
 def test_workspace_sizes_and_partition_plan():

@@ -126,6 +126,69 @@ def test_decode_edge_sweep(qdt, cdt, G, D, bs):
     assert np.all(g.out_f64()[0] == 0.0)          # context 0 -> zeros
 
 
+@pytest.mark.parametrize("qdt,cdt", [("f16", "f16"), ("bf16", "bf16"), ("bf16", "e4m3")])
+@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_decode_long_partitions(qdt, cdt, G, bs):
+    """Partitions longer than 512 tokens (the 4-warp CTA) with ragged tails,
+    and more partitions per sequence than the short-partition sweep reaches."""
+    Hkv = 2
+    sp, st, hd = custom([0, 1, 600, 1100, 2049, 1056], Hkv * G, Hkv, 128, bs, qdt, cdt,
+                        seed=77 + G + bs)
+    _, _, ref = oracle_step(sp, st, hd)
+    g = GpuStep(sp, st, hd)
+    g.reshape()
+    for part in (33 * bs, 48 * bs, 3 * bs):
+        g.out.fill_(float("nan"))
+        g.decode(partition_tokens=part)
+        torch.cuda.synchronize()
+        assert_close(g.out_f64(), ref, cdt, f"{qdt}/{cdt} G{G} bs{bs} part{part}")
+
+
+def test_workspace_reused_across_shapes_with_garbage_partials():
+    """One workspace, initialised once, then used by two partitioned launches
+    of different sizes; everything past the header is garbage beforehand."""
+    shapes = [custom([900, 33, 1500], 16, 2, 128, 16, "bf16", "bf16", seed=31),
+              custom([700, 2000, 5, 64, 1200], 8, 8, 128, 32, "f16", "f16", seed=32)]
+    ws = max((pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                                  sp.block_size, int(sp.context_lens.max()), 128)
+              for sp, _, _ in shapes), key=lambda t: t.numel())
+    ws[256:].fill_(0xFF)
+    for sp, st, hd in shapes:
+        _, _, ref = oracle_step(sp, st, hd)
+        g = GpuStep(sp, st, hd)
+        g.reshape()
+        g.decode(partition_tokens=128, workspace=ws)
+        torch.cuda.synchronize()
+        assert_close(g.out_f64(), ref, sp.cache_dtype, f"reuse {sp.num_seqs} seqs")
+
+
+def test_decode_graph_replay_is_bit_identical():
+    """A captured partitioned decode (decode kernel + combine kernel, chained by
+    programmatic dependent launch) replays with the same bits as the eager call."""
+    sp, st, hd = small(4)
+    g = GpuStep(sp, st, hd)
+    g.reshape()
+    ws = pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                             sp.block_size, g.max_ctx, 2 * sp.block_size)
+    g.decode(partition_tokens=2 * sp.block_size, workspace=ws)
+    torch.cuda.synchronize()
+    eager = host_codes(g.out).copy()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        pk.decode(g.out, g.q, g.kc, g.vc, g.bt, g.cl, g.max_ctx, sp.scale, k_scale=g.ks,
+                  v_scale=g.vs, partition_tokens=2 * sp.block_size, workspace=ws)
+    for _ in range(3):
+        g.out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(host_codes(g.out), eager)
+    pk.decode_check(ws)
+    del graph
+
+
 def test_decode_ignores_poisoned_slots_past_context():
     sp, st, hd = custom([5, 17, 40, 100], 8, 2, 128, 16, "bf16", "bf16", seed=9)
     for s, n in enumerate(sp.context_lens):
