@@ -13,12 +13,41 @@ increments it and a block goes back to the free list only when ``free``
 brings it to zero. The page does not say what the initial free-list order
 is; it starts as ``list(range(num_blocks))`` there, and a caller may pass a
 permutation instead (a seeded shuffle is an input, not part of the method).
+
+Prefix caching ([P4] "Prefix Caching": KV blocks of a shared prompt prefix
+are reused across requests and found by hash matching) keeps a map from
+block content hash to block, with the policy of ``acquire_prefix``.
 """
 from __future__ import annotations
 
 
+import hashlib
+
+import numpy as np
+
+
 class OutOfBlocks(Exception):
     pass
+
+
+def block_hash(parent, tokens) -> bytes:
+    """Content hash of one full block for prefix caching ([P4], Prefix
+    Caching: shareable prefix blocks are found by hash matching; the page
+    names no hash). SHA-256 of the parent block's 32-byte hash (32 zero bytes
+    for a prompt's first block) followed by the token ids as little-endian
+    int32 (hashlib's SHA-256 is the library step)."""
+    head = bytes(32) if parent is None else bytes(parent)
+    assert len(head) == 32
+    return hashlib.sha256(head + np.asarray(tokens, dtype="<i4").tobytes()).digest()
+
+
+def prompt_block_hashes(tokens, block_size: int) -> list:
+    """Chained hashes of the full blocks of a prompt (a partial last block has none)."""
+    out, parent = [], None
+    for j in range(len(tokens) // block_size):
+        parent = block_hash(parent, tokens[j * block_size:(j + 1) * block_size])
+        out.append(parent)
+    return out
 
 
 class BlockManager:
@@ -32,6 +61,8 @@ class BlockManager:
                 raise ValueError("initial order must be a permutation of range(num_blocks)")
             self.free_blocks = order
         self.refcount = [0] * num_blocks
+        self.by_hash = {}          # prefix caching: hash -> block
+        self.hash_of = {}          # block -> hash
 
     def allocate(self, n: int) -> list:
         if n < 0:
@@ -42,7 +73,66 @@ class BlockManager:
         self.free_blocks = self.free_blocks[n:]
         for b in taken:
             self.refcount[b] = 1
+            self._drop_hash(b)     # new content: a cached hash no longer holds
         return taken
+
+    def _drop_hash(self, b):
+        h = self.hash_of.pop(b, None)
+        if h is not None:
+            del self.by_hash[h]
+
+    def acquire_prefix(self, hashes):
+        """Blocks for a prompt's full-block hashes, in order ([P4] Prefix
+        Caching). A hash naming a cached block takes a reference to it (a
+        cached block with no references left is taken back out of the free
+        list); every other hash gets the head of the free list, registered
+        under the hash. Cached blocks are taken before any fresh one, so a
+        fresh allocation never evicts a block this request reuses. A block
+        keeps its hash after it is freed and loses it when handed out again.
+        Returns (ids, hits); OutOfBlocks leaves everything unchanged."""
+        hashes = [bytes(h) for h in hashes]
+        new_hashes = {h for h in hashes if h not in self.by_hash}
+        revived = {self.by_hash[h] for h in hashes
+                   if h in self.by_hash and self.refcount[self.by_hash[h]] == 0}
+        if len(new_hashes) > len(self.free_blocks) - len(revived):
+            raise OutOfBlocks(f"Need {len(new_hashes)} new blocks")
+        ids, hits = [None] * len(hashes), 0
+        for i, h in enumerate(hashes):
+            if h in self.by_hash:
+                b = self.by_hash[h]
+                if self.refcount[b] == 0:
+                    self.free_blocks.remove(b)
+                self.refcount[b] += 1
+                ids[i] = b
+                hits += 1
+        for i, h in enumerate(hashes):
+            if ids[i] is not None:
+                continue
+            if h in self.by_hash:          # an earlier block of this request
+                b = self.by_hash[h]
+                self.refcount[b] += 1
+                hits += 1
+            else:
+                (b,) = self.allocate(1)
+                self.by_hash[h] = b
+                self.hash_of[b] = h
+            ids[i] = b
+        return ids, hits
+
+    def register_hash(self, block_id: int, h) -> None:
+        """Give an allocated block (that just became full) its content hash;
+        nothing happens if the hash names a block already."""
+        b, h = int(block_id), bytes(h)
+        if not (0 <= b < self.num_blocks) or self.refcount[b] == 0:
+            raise ValueError("register_hash of a free or unknown block")
+        if h in self.by_hash:
+            return
+        self._drop_hash(b)
+        self.by_hash[h] = b
+        self.hash_of[b] = h
+
+    def lookup(self, h) -> int:
+        return self.by_hash.get(bytes(h), -1)
 
     def share(self, block_id: int) -> None:
         if not (0 <= block_id < self.num_blocks) or self.refcount[block_id] == 0:
