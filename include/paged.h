@@ -247,6 +247,24 @@ PA_API pa_status pa_copy_blocks(const void* src_key_cache, const void* src_value
                                 int32_t* error_word, pa_stream_t stream);
 
 /* ------------------------------------------------------------------------- */
+/* Block content hashes for prefix caching (host only).                        */
+/* ------------------------------------------------------------------------- */
+
+/* SHA-256 (FIPS 180-4) of n bytes. */
+PA_API pa_status pa_sha256(const void* data, int64_t n, uint8_t out[32]);
+/* Hash of one block: SHA-256 of the parent block's 32-byte hash (32 zero bytes
+ * when parent is NULL: the first block of a prompt) followed by the block's
+ * num_tokens token ids as little-endian int32. [P4] recognises shareable
+ * prefix blocks by hash matching without naming a hash; chaining through the
+ * parent makes equal hashes mean equal whole prefixes. */
+PA_API pa_status pa_block_hash(const uint8_t* parent, const int32_t* tokens, int32_t num_tokens,
+                               uint8_t out[32]);
+/* Chained hashes of the floor(num_tokens / block_size) full blocks of a
+ * prompt into hashes_out[32 * j]; a partial last block has none. */
+PA_API pa_status pa_prompt_block_hashes(const int32_t* tokens, int64_t num_tokens,
+                                        int32_t block_size, uint8_t* hashes_out);
+
+/* ------------------------------------------------------------------------- */
 /* Host block allocator (no device memory; produces integer tables only).      */
 /* ------------------------------------------------------------------------- */
 /*
@@ -281,6 +299,24 @@ PA_API pa_status pa_alloc_free(pa_alloc* a, const int32_t* ids, int32_t n);
  * PA_ERR_INVALID_ARG for a free or unknown id. */
 PA_API pa_status pa_alloc_copy_on_write(pa_alloc* a, int32_t id, int32_t* id_out,
                                         int32_t* must_copy);
+/* Prefix caching ([P4] Prefix Caching: prefix blocks are reused across
+ * requests, recognised by hash matching). hashes: n 32-byte block hashes
+ * (pa_prompt_block_hashes), in prompt order. Each hash that names a cached
+ * block takes a reference to it (a cached block whose references were all
+ * freed is taken back out of the free list); every other hash gets a fresh
+ * block from the head of the free list, registered under that hash (the
+ * caller then fills it). ids_out[i] is the block of hash i; *num_hits counts
+ * the hashes that found a block. PA_ERR_OOM (nothing changes) when the fresh
+ * blocks do not fit. A block keeps its hash after it is freed and loses it
+ * when it is handed out again from the head of the free list. */
+PA_API pa_status pa_alloc_acquire_prefix(pa_alloc* a, const uint8_t* hashes, int32_t n,
+                                         int32_t* ids_out, int32_t* num_hits);
+/* Register the hash of an allocated block that has just become full (e.g. a
+ * decode step filled it), replacing any hash it had. Nothing happens when the
+ * hash names a block already. PA_ERR_INVALID_ARG for a free or unknown id. */
+PA_API pa_status pa_alloc_register_hash(pa_alloc* a, int32_t id, const uint8_t* hash);
+/* The block registered under a hash, or -1. */
+PA_API int32_t pa_alloc_lookup(const pa_alloc* a, const uint8_t* hash);
 PA_API int64_t pa_alloc_num_free(const pa_alloc* a);
 PA_API int64_t pa_alloc_num_blocks(const pa_alloc* a);
 /* Reference count of a block (0 = free), -1 for an id out of range. */

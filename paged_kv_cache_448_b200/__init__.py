@@ -22,7 +22,8 @@ from ._native import PagedError, check
 
 __all__ = ["reshape_and_cache", "decode", "decode_noalloc", "decode_workspace",
            "decode_workspace_size",
-           "decode_partition_tokens", "decode_check", "copy_blocks", "BlockAllocator",
+           "decode_partition_tokens", "decode_check", "copy_blocks", "sha256", "block_hash",
+           "prompt_block_hashes", "BlockAllocator",
            "build_block_table",
            "build_slot_mapping", "PagedError", "dtype_code"]
 
@@ -156,6 +157,33 @@ def copy_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache, 
         _ptr(error_word), _stream_handle(stream)))
 
 
+def sha256(data: bytes) -> bytes:
+    """SHA-256 of a byte string (pa_sha256)."""
+    buf = ctypes.create_string_buffer(bytes(data), max(len(data), 1))
+    out = ctypes.create_string_buffer(32)
+    check(_native.lib().pa_sha256(buf, len(data), out))
+    return out.raw
+
+
+def block_hash(parent, tokens) -> bytes:
+    """Hash of one block chained to its parent's (None for a prompt's first)."""
+    t = _i32(tokens)
+    par = None if parent is None else ctypes.create_string_buffer(bytes(parent), 32)
+    out = ctypes.create_string_buffer(32)
+    check(_native.lib().pa_block_hash(par, t.ctypes.data if t.size else None, t.size, out))
+    return out.raw
+
+
+def prompt_block_hashes(tokens, block_size: int) -> np.ndarray:
+    """uint8 [len(tokens) // block_size, 32]: chained hashes of the full blocks."""
+    t = _i32(tokens)
+    n = t.size // block_size
+    out = np.empty((max(n, 1), 32), np.uint8)
+    check(_native.lib().pa_prompt_block_hashes(t.ctypes.data if t.size else None, t.size,
+                                               block_size, out.ctypes.data))
+    return out[:n]
+
+
 class BlockAllocator:
     """Host free list with refcounts (pa_alloc_*)."""
 
@@ -194,6 +222,24 @@ class BlockAllocator:
         check(self._lib.pa_alloc_copy_on_write(self._h, int(block_id), ctypes.byref(out),
                                                ctypes.byref(copy)))
         return int(out.value), bool(copy.value)
+
+    def acquire_prefix(self, hashes):
+        """Blocks for a prompt's full-block hashes ([n, 32] uint8): cached ones
+        are shared, the rest allocated and registered. Returns (ids, hits)."""
+        h = np.ascontiguousarray(hashes, dtype=np.uint8).reshape(-1, 32)
+        ids = np.empty(max(len(h), 1), np.int32)
+        hits = ctypes.c_int32()
+        check(self._lib.pa_alloc_acquire_prefix(self._h, h.ctypes.data if len(h) else None,
+                                                len(h), ids.ctypes.data, ctypes.byref(hits)))
+        return [int(i) for i in ids[:len(h)]], int(hits.value)
+
+    def register_hash(self, block_id: int, h) -> None:
+        b = np.ascontiguousarray(np.frombuffer(bytes(h), np.uint8))
+        check(self._lib.pa_alloc_register_hash(self._h, int(block_id), b.ctypes.data))
+
+    def lookup(self, h) -> int:
+        b = np.ascontiguousarray(np.frombuffer(bytes(h), np.uint8))
+        return int(self._lib.pa_alloc_lookup(self._h, b.ctypes.data))
 
     @property
     def num_free(self) -> int:

@@ -34,12 +34,18 @@ SIGNATURES = [
     ("pa_decode_check", _st, [_P, _P]),
     ("pa_workspace_init", _st, [_P, _sz, _P]),
     ("pa_copy_blocks", _st, [_P, _P, _P, _P, _P, _i32, _i64, _i64, _i64, _P, _P]),
+    ("pa_sha256", _st, [_P, _i64, _P]),
+    ("pa_block_hash", _st, [_P, _P, _i32, _P]),
+    ("pa_prompt_block_hashes", _st, [_P, _i64, _i32, _P]),
     ("pa_alloc_create", _st, [_i64, _P, ctypes.POINTER(_P)]),
     ("pa_alloc_destroy", None, [_P]),
     ("pa_alloc_allocate", _st, [_P, _i32, _P]),
     ("pa_alloc_share", _st, [_P, _i32]),
     ("pa_alloc_free", _st, [_P, _P, _i32]),
     ("pa_alloc_copy_on_write", _st, [_P, _i32, ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
+    ("pa_alloc_acquire_prefix", _st, [_P, _P, _i32, _P, ctypes.POINTER(_i32)]),
+    ("pa_alloc_register_hash", _st, [_P, _i32, _P]),
+    ("pa_alloc_lookup", _i32, [_P, _P]),
     ("pa_alloc_num_free", _i64, [_P]),
     ("pa_alloc_num_blocks", _i64, [_P]),
     ("pa_alloc_refcount", _i32, [_P, _i32]),

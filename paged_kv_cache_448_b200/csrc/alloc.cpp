@@ -7,7 +7,17 @@
 // ("大模型推理KV Cache内存管理与PagedAttention分页显存实战": several sampling
 // requests of one prompt share the prefix blocks, their lifetime managed by a
 // reference count). Host memory only; no device calls.
-#include <deque>
+//
+// Prefix caching ("大模型推理KV Cache内存管理与PagedAttention分页显存实战",
+// Prefix Caching: prefix blocks are reused across requests, found by hash
+// matching): a full block may carry the content hash of prefix_hash.cpp. A
+// block keeps its hash after its last reference is freed, so a later request
+// with the same prefix can take it back from the free list; the hash is
+// dropped only when the block is handed out for other content (it reaches
+// the head of the free list), i.e. cached blocks are evicted oldest-freed first.
+#include <array>
+#include <cstring>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -15,9 +25,44 @@
 #include "paged.h"
 #include "status.h"
 
+namespace {
+using Hash = std::array<uint8_t, 32>;
+struct HashKey {
+  size_t operator()(const Hash& h) const {
+    size_t v;
+    std::memcpy(&v, h.data(), sizeof(v));
+    return v;
+  }
+};
+Hash to_hash(const uint8_t* p) {
+  Hash h;
+  std::memcpy(h.data(), p, 32);
+  return h;
+}
+}  // namespace
+
 struct pa_alloc {
-  std::deque<int32_t> free_list;
+  std::list<int32_t> free_list;
+  std::vector<std::list<int32_t>::iterator> where;  // position in free_list when free
   std::vector<int32_t> refcount;
+  std::vector<char> hashed;
+  std::vector<Hash> hash_of;
+  std::unordered_map<Hash, int32_t, HashKey> by_hash;
+
+  void push_free(int32_t id) { where[id] = free_list.insert(free_list.end(), id); }
+  void drop_hash(int32_t id) {
+    if (!hashed[id]) return;
+    by_hash.erase(hash_of[id]);
+    hashed[id] = 0;
+  }
+  // The head of the free list, for new content: its cached hash goes.
+  int32_t pop_free() {
+    const int32_t id = free_list.front();
+    free_list.pop_front();
+    drop_hash(id);
+    refcount[id] = 1;
+    return id;
+  }
 };
 
 using paged::clear_error;
@@ -35,6 +80,9 @@ PA_API pa_status pa_alloc_create(int64_t num_blocks, const int32_t* initial_free
   pa_alloc* a = new (std::nothrow) pa_alloc;
   if (!a) return fail(PA_ERR_OOM, "alloc_create: host allocation failed");
   a->refcount.assign(static_cast<size_t>(num_blocks), 0);
+  a->where.resize(static_cast<size_t>(num_blocks));
+  a->hashed.assign(static_cast<size_t>(num_blocks), 0);
+  a->hash_of.resize(static_cast<size_t>(num_blocks));
   if (initial_free_order) {
     std::vector<char> seen(static_cast<size_t>(num_blocks), 0);
     for (int64_t i = 0; i < num_blocks; ++i) {
@@ -44,10 +92,10 @@ PA_API pa_status pa_alloc_create(int64_t num_blocks, const int32_t* initial_free
         return fail(PA_ERR_INVALID_ARG, "alloc_create: initial order is not a permutation");
       }
       seen[id] = 1;
-      a->free_list.push_back(id);
+      a->push_free(id);
     }
   } else {
-    for (int64_t i = 0; i < num_blocks; ++i) a->free_list.push_back(static_cast<int32_t>(i));
+    for (int64_t i = 0; i < num_blocks; ++i) a->push_free(static_cast<int32_t>(i));
   }
   *out = a;
   return PA_OK;
@@ -60,12 +108,7 @@ PA_API pa_status pa_alloc_allocate(pa_alloc* a, int32_t n, int32_t* ids_out) {
   if (!a || n < 0 || (n > 0 && !ids_out)) return fail(PA_ERR_INVALID_ARG, "alloc_allocate: bad args");
   if (static_cast<size_t>(n) > a->free_list.size())
     return fail(PA_ERR_OOM, "Need %d blocks, only %zu available", n, a->free_list.size());
-  for (int32_t i = 0; i < n; ++i) {
-    const int32_t id = a->free_list.front();
-    a->free_list.pop_front();
-    a->refcount[id] = 1;
-    ids_out[i] = id;
-  }
+  for (int32_t i = 0; i < n; ++i) ids_out[i] = a->pop_free();
   return PA_OK;
 }
 
@@ -91,7 +134,7 @@ PA_API pa_status pa_alloc_free(pa_alloc* a, const int32_t* ids, int32_t n) {
   }
   for (int32_t i = 0; i < n; ++i) {
     const int32_t id = ids[i];
-    if (--a->refcount[id] == 0) a->free_list.push_back(id);
+    if (--a->refcount[id] == 0) a->push_free(id);
   }
   return PA_OK;
 }
@@ -112,13 +155,94 @@ PA_API pa_status pa_alloc_copy_on_write(pa_alloc* a, int32_t id, int32_t* id_out
     return PA_OK;
   }
   if (a->free_list.empty()) return fail(PA_ERR_OOM, "Need 1 block, only 0 available");
-  const int32_t fresh = a->free_list.front();
-  a->free_list.pop_front();
-  a->refcount[fresh] = 1;
+  const int32_t fresh = a->pop_free();
   --a->refcount[id];
   *id_out = fresh;
   *must_copy = 1;
   return PA_OK;
+}
+
+PA_API pa_status pa_alloc_acquire_prefix(pa_alloc* a, const uint8_t* hashes, int32_t n,
+                                         int32_t* ids_out, int32_t* num_hits) {
+  clear_error();
+  if (!a || n < 0 || (n > 0 && (!hashes || !ids_out)) || !num_hits)
+    return fail(PA_ERR_INVALID_ARG, "alloc_acquire_prefix: bad args");
+  // Feasibility first (nothing changes on PA_ERR_OOM): cached blocks that sit
+  // in the free list leave it, and every other hash needs a fresh block.
+  int64_t free_hits = 0, misses = 0;
+  std::unordered_map<Hash, int32_t, HashKey> fresh;  // hashes first seen in this request
+  for (int32_t i = 0; i < n; ++i) {
+    const Hash h = to_hash(hashes + 32 * static_cast<int64_t>(i));
+    auto it = a->by_hash.find(h);
+    if (it != a->by_hash.end()) {
+      if (a->refcount[it->second] == 0 && !fresh.count(h)) {
+        fresh.emplace(h, -1);  // revived once
+        ++free_hits;
+      }
+    } else if (fresh.emplace(h, -1).second) {
+      ++misses;
+    }
+  }
+  if (misses > static_cast<int64_t>(a->free_list.size()) - free_hits)
+    return fail(PA_ERR_OOM, "Need %lld new blocks, only %lld available",
+                static_cast<long long>(misses),
+                static_cast<long long>(a->free_list.size()) - free_hits);
+  // Cached blocks first, so that no fresh allocation evicts one of them.
+  int32_t hits = 0;
+  std::vector<char> done(static_cast<size_t>(n), 0);
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = a->by_hash.find(to_hash(hashes + 32 * static_cast<int64_t>(i)));
+    if (it == a->by_hash.end()) continue;
+    const int32_t id = it->second;
+    if (a->refcount[id] == 0) {
+      a->free_list.erase(a->where[id]);
+      a->refcount[id] = 1;
+    } else {
+      ++a->refcount[id];
+    }
+    ids_out[i] = id;
+    done[i] = 1;
+    ++hits;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    if (done[i]) continue;
+    const Hash h = to_hash(hashes + 32 * static_cast<int64_t>(i));
+    auto it = a->by_hash.find(h);
+    if (it != a->by_hash.end()) {  // registered by an earlier block of this request
+      ++a->refcount[it->second];
+      ids_out[i] = it->second;
+      ++hits;
+      continue;
+    }
+    const int32_t id = a->pop_free();
+    a->hashed[id] = 1;
+    a->hash_of[id] = h;
+    a->by_hash.emplace(h, id);
+    ids_out[i] = id;
+  }
+  *num_hits = hits;
+  return PA_OK;
+}
+
+PA_API pa_status pa_alloc_register_hash(pa_alloc* a, int32_t id, const uint8_t* hash) {
+  clear_error();
+  if (!a || !hash || id < 0 || static_cast<size_t>(id) >= a->refcount.size() ||
+      a->refcount[id] == 0)
+    return fail(PA_ERR_INVALID_ARG, "alloc_register_hash: block %d is not allocated", id);
+  const Hash h = to_hash(hash);
+  auto it = a->by_hash.find(h);
+  if (it != a->by_hash.end()) return PA_OK;  // that content is cached already (maybe here)
+  a->drop_hash(id);
+  a->hashed[id] = 1;
+  a->hash_of[id] = h;
+  a->by_hash.emplace(h, id);
+  return PA_OK;
+}
+
+PA_API int32_t pa_alloc_lookup(const pa_alloc* a, const uint8_t* hash) {
+  if (!a || !hash) return -1;
+  auto it = a->by_hash.find(to_hash(hash));
+  return it == a->by_hash.end() ? -1 : it->second;
 }
 
 PA_API int64_t pa_alloc_num_free(const pa_alloc* a) {

@@ -5,6 +5,8 @@ import ctypes
 import os
 import re
 
+import hashlib
+
 import numpy as np
 import pytest
 
@@ -192,6 +194,75 @@ def test_reshape_rejects_bad_arguments():
     assert call(cdt=_native.PA_FP8_E4M3) == _native.PA_ERR_INVALID_ARG
     assert call(k=24) == _native.PA_ERR_INVALID_ARG
     assert call(T=0, k=None) == _native.PA_OK
+
+
+def test_sha256_matches_fips_examples():
+    import json, os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "sha256_fips180.json")) as f:
+        vecs = json.load(f)["vectors"]
+    for v in vecs:
+        m = b"a" * 1000000 if v["message"] == "a*1000000" else v["message"].encode()
+        assert pk.sha256(m).hex() == v["sha256"], v["cite"]
+    assert pk.sha256(b"").hex() == hashlib.sha256(b"").hexdigest()
+    rng = np.random.default_rng(1)
+    for n in [1, 55, 56, 63, 64, 65, 119, 120, 128, 1000]:   # padding boundaries
+        m = rng.integers(0, 256, n).astype(np.uint8).tobytes()
+        assert pk.sha256(m) == hashlib.sha256(m).digest(), n
+
+
+def test_block_hashes_match_oracle():
+    from oracle.block_manager import block_hash, prompt_block_hashes
+    rng = np.random.default_rng(2)
+    for trial in range(20):
+        bs = int(rng.choice([16, 32]))
+        toks = rng.integers(-5, 200000, int(rng.integers(0, 400))).astype(np.int32)
+        ours = pk.prompt_block_hashes(toks, bs)
+        ref = prompt_block_hashes(toks.tolist(), bs)
+        assert [bytes(r) for r in ours] == ref
+    parent = bytes(rng.integers(0, 256, 32).astype(np.uint8))
+    assert pk.block_hash(parent, [3, 4, 5]) == block_hash(parent, [3, 4, 5])
+    assert pk.block_hash(None, []) == block_hash(None, [])
+
+
+def test_prefix_cache_matches_oracle_model_on_random_requests():
+    from oracle.block_manager import prompt_block_hashes
+    rng = np.random.default_rng(23)
+    prefixes = [rng.integers(0, 1000, 16 * int(rng.integers(1, 5))).tolist() for _ in range(4)]
+    for trial in range(10):
+        nb = int(rng.integers(4, 60))
+        order = rng.permutation(nb).astype(np.int32)
+        ours, ref = pk.BlockAllocator(nb, order), BlockManager(nb, order)
+        held = []                          # block lists of live requests
+        for _ in range(200):
+            op = rng.integers(0, 4)
+            if op <= 1:                    # a request: shared prefix + own tokens
+                toks = prefixes[int(rng.integers(0, 4))] + \
+                    rng.integers(0, 3, 16 * int(rng.integers(0, 3))).tolist()
+                hs = prompt_block_hashes(toks, 16)
+                try:
+                    expect = ref.acquire_prefix(hs)
+                except OutOfBlocks:
+                    with pytest.raises(pk.PagedError) as ei:
+                        ours.acquire_prefix(np.frombuffer(b"".join(hs), np.uint8))
+                    assert ei.value.status == _native.PA_ERR_OOM
+                    continue
+                got = ours.acquire_prefix(np.frombuffer(b"".join(hs), np.uint8).reshape(-1, 32))
+                assert got == expect
+                held.append(expect[0])
+            elif op == 2 and held:         # a request ends
+                ids = held.pop(int(rng.integers(0, len(held))))
+                ref.free(ids); ours.free(ids)
+            elif op == 3 and held:         # a decode step fills a block: register it
+                ids = held[int(rng.integers(0, len(held)))]
+                if ids:
+                    h = bytes(rng.integers(0, 256, 32).astype(np.uint8))
+                    b = ids[int(rng.integers(0, len(ids)))]
+                    ref.register_hash(b, h); ours.register_hash(b, h)
+            assert ours.free_list() == ref.free_blocks
+            for b in range(nb):
+                assert ours.refcount(b) == ref.refcount[b]
+            for h, b in list(ref.by_hash.items())[:8]:
+                assert ours.lookup(h) == b
 
 
 def test_copy_blocks_rejects_bad_arguments_before_launch():
