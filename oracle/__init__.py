@@ -12,6 +12,8 @@ Functions mirror the pages' problem statement:
   (attention over the blocks a block table names) with the logical->physical
   translation of [P1] "vLLM框架中的KV cache优化与PagedAttention机制详解" §5.1.
 * ``reshape_and_cache`` — writes rows into the cache layout of [P2] §2.2.
+* ``chunked_prefill`` — the same attention for several query tokens per
+  sequence (its last positions), each seeing itself and earlier tokens.
 * ``slot_mapping`` — the address translation of [P3] "Paged KVCache：大模型推理
   显存管理优化方案" §2.3, page size counted in tokens.
 * ``BlockManager`` (``oracle.block_manager``) — the free list of [P2] §2.2 with
@@ -82,6 +84,9 @@ def _load():
         lib.orc_decode.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64, f32,
                                    ctypes.c_int, ctypes.c_int, P, P, i32]
         lib.orc_decode.restype = ctypes.c_int
+        lib.orc_chunked_prefill.argtypes = [P, P, P, i32, P, P, P, i32, P, i32, i32, i32, i32,
+                                            i32, i64, f32, ctypes.c_int, ctypes.c_int, P, P]
+        lib.orc_chunked_prefill.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -203,6 +208,36 @@ def decode(query, key_cache, value_cache, block_tables, context_lens, *, scale: 
                             int(partition_tokens))
     if rc != 0:
         raise ValueError(f"oracle decode failed (rc={rc})")
+    return out
+
+
+def chunked_prefill(query, key_cache, value_cache, block_tables, context_lens, cu_query_lens, *,
+                    scale: float, q_dtype: str, cache_dtype: str, k_scale=None,
+                    v_scale=None) -> np.ndarray:
+    """fp64 output [T, H, D] of a multi-token query: rows cu_query_lens[s] ..
+    cu_query_lens[s+1]-1 of query (raw codes [T, H, D]) are the last positions
+    of sequence s and attend causally to its cached tokens (orc_chunked_prefill)."""
+    q = _raw(query, q_dtype)
+    kc = _raw(key_cache, cache_dtype)
+    vc = _raw(value_cache, cache_dtype)
+    if not (kc.flags.c_contiguous and vc.flags.c_contiguous):
+        raise ValueError("caches must be C-contiguous")
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    cu = np.ascontiguousarray(cu_query_lens, dtype=np.int32)
+    T, H, D = q.shape
+    NB, BS, Hkv, D2 = kc.shape
+    S = cl.shape[0]
+    assert D2 == D and bt.shape[0] == S and cu.shape[0] == S + 1
+    ks = None if k_scale is None else np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = None if v_scale is None else np.ascontiguousarray(v_scale, dtype=np.float32)
+    out = np.zeros((T, H, D), dtype=np.float64)
+    rc = _load().orc_chunked_prefill(_ptr(out), _ptr(q), _ptr(cu), T, _ptr(kc), _ptr(vc),
+                                     _ptr(bt), bt.shape[1], _ptr(cl), S, H, Hkv, D, BS, NB,
+                                     float(scale), DTYPE_CODES[q_dtype], DTYPE_CODES[cache_dtype],
+                                     _ptr(ks), _ptr(vs))
+    if rc != 0:
+        raise ValueError(f"oracle chunked_prefill failed (rc={rc})")
     return out
 
 

@@ -370,3 +370,62 @@ int orc_decode(double* out, const void* query, const void* key_cache, const void
   }
   return 0;
 }
+
+/*
+ * Multi-token query over the paged cache (chunked prefill, verification of
+ * several draft tokens). [P2] §2.3's interface takes a query tensor; here it
+ * has more rows than sequences: the q_len_s = cu_q[s+1] - cu_q[s] rows
+ * query[cu_q[s] ..] are the last q_len_s positions of sequence s,
+ * p_i = context_lens[s] - q_len_s + i, whose keys and values are already in
+ * the cache. Row i attends to the tokens t <= p_i of its sequence (the
+ * causal rule of autoregressive attention: a token sees itself and its
+ * past), through block_tables as in orc_decode. out is fp64
+ * [num_tokens, num_heads, head_dim]. Returns 0; -1 on a bad table entry;
+ * -2 on bad sizes; -3 when q_len_s > context_lens[s].
+ */
+int orc_chunked_prefill(double* out, const void* query, const int32_t* cu_q, int32_t num_tokens,
+                        const void* key_cache, const void* value_cache,
+                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                        const int32_t* context_lens, int32_t num_seqs, int32_t num_heads,
+                        int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                        int64_t num_blocks, float scale, int q_dtype, int cache_dtype,
+                        const float* k_scale, const float* v_scale) {
+  if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0 ||
+      cu_q[0] != 0 || cu_q[num_seqs] != num_tokens)
+    return -2;
+  int32_t group = num_heads / num_kv_heads;
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    int32_t n = context_lens[s];
+    int32_t qlen = cu_q[s + 1] - cu_q[s];
+    if (n < 0 || qlen < 0 || (n + block_size - 1) / block_size > max_blocks_per_seq) return -2;
+    if (qlen > n) return -3;
+    const int32_t* row = block_tables + (size_t)s * max_blocks_per_seq;
+    double* K = (double*)malloc(sizeof(double) * ((size_t)n * head_dim + 1));
+    double* V = (double*)malloc(sizeof(double) * ((size_t)n * head_dim + 1));
+    double* q = (double*)malloc(sizeof(double) * (size_t)head_dim);
+    int rc = 0;
+    for (int32_t kvh = 0; kvh < num_kv_heads && rc == 0; ++kvh) {
+      double ks = (cache_dtype == ORC_E4M3) ? (double)k_scale[kvh] : 1.0;
+      double vs = (cache_dtype == ORC_E4M3) ? (double)v_scale[kvh] : 1.0;
+      rc = gather_sequence(key_cache, cache_dtype, ks, row, n, kvh, num_kv_heads, head_dim,
+                           block_size, num_blocks, K);
+      if (rc == 0)
+        rc = gather_sequence(value_cache, cache_dtype, vs, row, n, kvh, num_kv_heads, head_dim,
+                             block_size, num_blocks, V);
+      if (rc != 0) break;
+      for (int32_t i = 0; i < qlen; ++i) {
+        int32_t pos = n - qlen + i;
+        for (int32_t j = 0; j < group; ++j) {
+          int32_t h = kvh * group + j;
+          size_t qoff = ((size_t)(cu_q[s] + i) * num_heads + h) * head_dim;
+          for (int32_t d = 0; d < head_dim; ++d) q[d] = load_elem(query, qoff + d, q_dtype);
+          double m, l;
+          attend_rows(q, K, V, 0, pos + 1, head_dim, (double)scale, out + qoff, &m, &l);
+        }
+      }
+    }
+    free(K); free(V); free(q);
+    if (rc != 0) return rc;
+  }
+  return 0;
+}

@@ -362,6 +362,86 @@ def test_decode_equals_unpaged_sdpa(qdt, cdt, H, Hkv, D, bs, ctxs):
     np.testing.assert_allclose(ours, ref, rtol=1e-12, atol=1e-13)
 
 
+PREFILL_CASES = [
+    # (q/cache dtype, H, Hkv, D, bs, contexts, query lengths)
+    ("f16", "f16", 4, 4, 64, 16, [17, 40, 5, 33], [17, 9, 1, 16]),
+    ("bf16", "bf16", 8, 2, 128, 32, [64, 100, 70], [64, 3, 33]),
+    ("bf16", "e4m3", 8, 1, 64, 16, [50, 20], [7, 20]),
+]
+
+
+def _prefill_inputs(qdt, cdt, H, Hkv, D, bs, ctxs, qlens, seed):
+    rng = np.random.default_rng(seed)
+    T = sum(qlens)
+    q = from_f32(rng.standard_normal((T, H, D)), qdt)
+    if cdt == "e4m3":
+        Kc = [random_e4m3_codes(rng, (n, Hkv, D)) for n in ctxs]
+        Vc = [random_e4m3_codes(rng, (n, Hkv, D)) for n in ctxs]
+        ks = rng.uniform(0.001, 0.01, Hkv).astype(np.float32)
+        vs = rng.uniform(0.001, 0.01, Hkv).astype(np.float32)
+    else:
+        Kc = [from_f32(rng.standard_normal((n, Hkv, D)), cdt) for n in ctxs]
+        Vc = [from_f32(rng.standard_normal((n, Hkv, D)), cdt) for n in ctxs]
+        ks = vs = None
+    kc, vc, table = build_paged(rng, Kc, Vc, ctxs, bs)
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    return q, Kc, Vc, ks, vs, kc, vc, table, cu
+
+
+@pytest.mark.parametrize("qdt,cdt,H,Hkv,D,bs,ctxs,qlens", PREFILL_CASES)
+def test_chunked_prefill_equals_masked_sdpa(qdt, cdt, H, Hkv, D, bs, ctxs, qlens):
+    """Against fp64 torch SDPA on the contiguous K/V with an explicit boolean
+    mask (row i of sequence s sees keys 0 .. ctx - qlen + i); where the chunk
+    is the whole context, against SDPA's own is_causal rule as well."""
+    q, Kc, Vc, ks, vs, kc, vc, table, cu = _prefill_inputs(qdt, cdt, H, Hkv, D, bs, ctxs, qlens,
+                                                          seed=H + D + bs)
+    scale = float(np.float32(1.0 / math.sqrt(D)))
+    ours = oracle.chunked_prefill(q, kc, vc, table, np.array(ctxs, np.int32), cu,
+                                  scale=np.float32(scale), q_dtype=qdt, cache_dtype=cdt,
+                                  k_scale=ks, v_scale=vs)
+    G = H // Hkv
+    qf = to_f64(q, qdt)
+    for s, (n, ql) in enumerate(zip(ctxs, qlens)):
+        K = to_f64(Kc[s], cdt) * (1.0 if ks is None else ks.astype(np.float64)[None, :, None])
+        V = to_f64(Vc[s], cdt) * (1.0 if vs is None else vs.astype(np.float64)[None, :, None])
+        k = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(G, 0)     # [H, n, D]
+        v = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(G, 0)
+        qs = torch.from_numpy(qf[cu[s]:cu[s + 1]]).permute(1, 0, 2)         # [H, ql, D]
+        pos = torch.arange(n - ql, n)[:, None]
+        mask = torch.arange(n)[None, :] <= pos                               # [ql, n]
+        ref = torch.nn.functional.scaled_dot_product_attention(qs, k, v, attn_mask=mask,
+                                                               scale=scale)
+        np.testing.assert_allclose(ours[cu[s]:cu[s + 1]], ref.permute(1, 0, 2).numpy(),
+                                   rtol=1e-12, atol=1e-13)
+        if ql == n:
+            causal = torch.nn.functional.scaled_dot_product_attention(qs, k, v, is_causal=True,
+                                                                      scale=scale)
+            np.testing.assert_allclose(ours[cu[s]:cu[s + 1]], causal.permute(1, 0, 2).numpy(),
+                                       rtol=1e-12, atol=1e-13)
+
+
+def test_chunked_prefill_with_one_token_per_sequence_is_decode():
+    q, Kc, Vc, ks, vs, kc, vc, table, cu = _prefill_inputs("bf16", "bf16", 8, 2, 128, 16,
+                                                          [1, 30, 77], [1, 1, 1], seed=4)
+    ctx = np.array([1, 30, 77], np.int32)
+    a = oracle.chunked_prefill(q, kc, vc, table, ctx, cu, scale=np.float32(0.1), q_dtype="bf16",
+                               cache_dtype="bf16")
+    b = oracle.decode(q, kc, vc, table, ctx, scale=np.float32(0.1), q_dtype="bf16",
+                      cache_dtype="bf16")
+    assert np.array_equal(a, b)
+
+
+def test_chunked_prefill_first_row_of_a_full_chunk_returns_v0():
+    q, Kc, Vc, ks, vs, kc, vc, table, cu = _prefill_inputs("f16", "f16", 4, 4, 64, 16,
+                                                          [20], [20], seed=8)
+    out = oracle.chunked_prefill(q, kc, vc, table, np.array([20], np.int32), cu,
+                                 scale=np.float32(0.125), q_dtype="f16", cache_dtype="f16")
+    assert np.array_equal(out[0], to_f64(Vc[0][0], "f16"))     # sees only token 0
+    with pytest.raises(ValueError):                              # chunk longer than context
+        oracle.chunked_prefill(q, kc, vc, table, np.array([19], np.int32), cu,
+                               scale=np.float32(0.125), q_dtype="f16", cache_dtype="f16")
+
+
 def _small_workload(cfg):
     sp = wl.spec(cfg, small=True)
     st = wl.structure(sp)
