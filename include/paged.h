@@ -186,6 +186,41 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* query,
                     int32_t partition_tokens, pa_stream_t stream);
 
 /*
+ * Attention of several query tokens per sequence over the paged cache
+ * (chunked prefill; verification of several draft tokens). [P2] §2.3's
+ * interface takes a query tensor; here it has more rows than sequences:
+ * rows cu_query_lens[s] .. cu_query_lens[s+1]-1 of query are the last
+ * q_len_s = cu_query_lens[s+1] - cu_query_lens[s] positions of sequence s,
+ * p_i = context_lens[s] - q_len_s + i, whose keys and values are already in
+ * the cache (pa_reshape_and_cache). Row i attends to the tokens t <= p_i of
+ * its sequence (the causal rule of autoregressive attention), query head h
+ * to kv-head h / (num_heads / num_kv_heads), with softmax scale `scale`.
+ * out, query      device [num_tokens, num_heads, head_dim] of `dtype`
+ *                 (f16 or bf16; the cache has the same dtype).
+ * cu_query_lens   device int32 [num_seqs + 1], cu[0] = 0, cu[num_seqs] = num_tokens.
+ * max_query_len   host int >= every q_len_s; sizes the launch.
+ * key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens,
+ * max_context_len, num_blocks: as in pa_decode (context_lens include the
+ * query tokens).
+ * workspace       >= 256 bytes, 256-byte aligned, zeroed once (pa_workspace_init);
+ *                 its error word reports, through pa_decode_check, table
+ *                 entries outside the pool (read as zeros), clipped context
+ *                 lengths, and a query longer than its context (bit 16; those
+ *                 rows are written as zeros).
+ * Supported: head_dim in {64, 128}; block_size in {16, 32}; group in {1, 2, 4, 8};
+ *            at most 65535 sequences and kv-heads.
+ */
+PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t* cu_query_lens,
+                                    int32_t num_tokens, int32_t max_query_len,
+                                    const void* key_cache, const void* value_cache,
+                                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                    const int32_t* context_lens, int32_t max_context_len,
+                                    int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                    int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                                    float scale, pa_dtype dtype, void* workspace,
+                                    size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * Bytes of workspace pa_decode needs for these sizes on the current device
  * (the automatic partition choice depends on the device's SM count).
  * Returns 0 for invalid sizes.
@@ -204,8 +239,10 @@ PA_API int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads, i
 
 /*
  * Synchronises `stream`, reads and clears the error word of `workspace`.
- * Returns PA_OK, or PA_ERR_BAD_TABLE if a previous pa_decode on this workspace
- * met an out-of-range table entry or context length, or PA_ERR_CUDA.
+ * Returns PA_OK, or PA_ERR_BAD_TABLE if a previous pa_decode or
+ * pa_chunked_prefill on this workspace met an out-of-range table entry or
+ * context length or a query longer than its context, or PA_ERR_CUDA (a wait
+ * that gave up, or a CUDA error).
  */
 PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream);
 

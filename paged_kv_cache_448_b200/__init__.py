@@ -22,7 +22,7 @@ from ._native import PagedError, check
 
 __all__ = ["reshape_and_cache", "decode", "decode_noalloc", "decode_workspace",
            "decode_workspace_size",
-           "decode_partition_tokens", "decode_check", "copy_blocks", "sha256", "block_hash",
+           "decode_partition_tokens", "decode_check", "chunked_prefill", "copy_blocks", "sha256", "block_hash",
            "prompt_block_hashes", "BlockAllocator",
            "build_block_table",
            "build_slot_mapping", "PagedError", "dtype_code"]
@@ -131,6 +131,25 @@ def decode_check(workspace, stream=None) -> None:
 
 def _i32(a) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def chunked_prefill(out, query, cu_query_lens, max_query_len: int, key_cache, value_cache,
+                    block_tables, context_lens, max_context_len: int, scale: float, *,
+                    workspace=None, stream=None):
+    """Several query tokens per sequence (its last positions), causal
+    (pa_chunked_prefill). out/query [T, H, D] f16|bf16 (cache of the same
+    dtype); cu_query_lens int32 [S+1]; context_lens include the query tokens."""
+    T, H, D = query.shape
+    NB, BS, Hkv = key_cache.shape[:3]
+    S = context_lens.shape[0]
+    if workspace is None:
+        workspace = decode_workspace(1, 1, 1, D, BS, 0, 0, device=query.device, stream=stream)
+    check(_native.lib().pa_chunked_prefill(
+        _ptr(out), _ptr(query), _ptr(cu_query_lens), T, int(max_query_len), _ptr(key_cache),
+        _ptr(value_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+        int(max_context_len), S, H, Hkv, D, BS, NB, float(scale), dtype_code(query),
+        _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+    return out
 
 
 def copy_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache, block_pairs, *,

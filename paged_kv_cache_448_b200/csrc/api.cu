@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "decode_args.h"
+#include "prefill_args.h"
 #include "paged.h"
 #include "status.h"
 
@@ -264,10 +265,12 @@ PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream) {
   if (e == cudaSuccess && word != 0) e = cudaMemset(workspace, 0, 64);  // error + failure record
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode_check: %s", cudaGetErrorString(e));
   if (word & kErrWaitTimeout) return fail(PA_ERR_CUDA, "decode: a pipeline wait timed out");
-  if (word & (kErrBadBlockId | kErrContextClipped))
-    return fail(PA_ERR_BAD_TABLE, "decode: %s%s",
+  if (word & (kErrBadBlockId | kErrContextClipped | kErrQueryLonger))
+    return fail(PA_ERR_BAD_TABLE, "decode: %s%s%s",
                 (word & kErrBadBlockId) ? "block-table entry outside the pool; " : "",
-                (word & kErrContextClipped) ? "context length beyond the launch; clipped" : "");
+                (word & kErrContextClipped) ? "context length beyond the launch; clipped; " : "",
+                (word & kErrQueryLonger) ? "query longer than its context; rows zeroed" : "");
+  if (word) return fail(PA_ERR_CUDA, "decode: error word 0x%x", word);
   return PA_OK;
 }
 
@@ -408,6 +411,73 @@ PA_API pa_status pa_copy_blocks(const void* src_key_cache, const void* src_value
       static_cast<const int32_t*>(views[4]), num_pairs, block_bytes, num_src_blocks,
       num_dst_blocks, err, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   return cuda_status(e, "copy_blocks");
+}
+
+PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t* cu_query_lens,
+                                    int32_t num_tokens, int32_t max_query_len,
+                                    const void* key_cache, const void* value_cache,
+                                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                    const int32_t* context_lens, int32_t max_context_len,
+                                    int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                    int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                                    float scale, pa_dtype dtype, void* workspace,
+                                    size_t workspace_bytes, pa_stream_t stream) {
+  clear_error();
+  if (num_tokens < 0 || max_query_len < 0 || num_seqs < 0 || num_heads <= 0 ||
+      num_kv_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || num_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "chunked_prefill: negative or zero size");
+  if (num_heads % num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "chunked_prefill: num_heads %% num_kv_heads != 0");
+  const int32_t group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: query group %d not in {1,2,4,8}", group);
+  if (!shape_supported(head_dim, block_size))
+    return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: head_dim %d / block_size %d unsupported",
+                head_dim, block_size);
+  if (dtype != PA_F16 && dtype != PA_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: query and cache must be f16 or bf16");
+  if (num_blocks * block_size > INT32_MAX)
+    return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: pool rows exceed 2^31");
+  if (num_seqs > 65535 || num_kv_heads > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: more than 65535 sequences or kv-heads");
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "chunked_prefill: scale is not finite");
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < kHeaderBytes)
+    return fail(PA_ERR_INVALID_ARG, "chunked_prefill: workspace missing, small or misaligned");
+  if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens ||
+      !cu_query_lens)
+    return fail(PA_ERR_INVALID_ARG, "chunked_prefill: null pointer");
+  if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) ||
+      !aligned(value_cache, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4) ||
+      !aligned(cu_query_lens, 4))
+    return fail(PA_ERR_INVALID_ARG, "chunked_prefill: misaligned pointer");
+
+  CUtensorMap kmap, vmap;
+  pa_status st = encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads,
+                                  head_dim, 2);
+  if (st == PA_OK)
+    st = encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, 2);
+  if (st != PA_OK) return st;
+  PrefillArgs a{};
+  a.out = out;
+  a.query = query;
+  a.cu_query_lens = cu_query_lens;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.err = reinterpret_cast<int32_t*>(workspace) + kWordError;
+  a.diag = reinterpret_cast<int32_t*>(workspace) + kWordDiag;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.ctx_limit = std::min<int64_t>(max_context_len,
+                                  static_cast<int64_t>(max_blocks_per_seq) * block_size);
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.block_size = block_size;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  return cuda_status(launch_prefill(a, kmap, vmap, dtype == PA_F16 ? kF16 : kBF16, head_dim, group,
+                                    max_query_len, reinterpret_cast<cudaStream_t>(stream)),
+                     "chunked_prefill");
 }
 
 }  // extern "C"

@@ -15,6 +15,7 @@ enum : int32_t {
   kErrContextClipped = 2,  // a context length above what the launch covers
   kErrWaitTimeout = 4,     // a pipeline wait gave up (never expected)
   kErrBadSlot = 8,         // reshape_and_cache: a slot outside the pool
+  kErrQueryLonger = 16,    // multi-token query: more query rows than context (rows are zeros)
 };
 
 // Failure sites recorded in the diagnostic words.

@@ -1,0 +1,38 @@
+// prefill_args.h — host/device argument block of the multi-token query kernel.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace paged {
+
+struct PrefillArgs {
+  void* out;                     // [T, H, D] q dtype
+  const void* query;             // [T, H, D] q dtype
+  const int32_t* cu_query_lens;  // [S + 1]: rows of sequence s are cu[s] .. cu[s+1]-1
+  const int32_t* block_tables;   // [S, max_blocks_per_seq]
+  const int32_t* context_lens;   // [S], including the query tokens
+  int32_t* err;                  // error word
+  int32_t* diag;                 // failure record
+  int64_t num_blocks;
+  int32_t max_blocks_per_seq;
+  int32_t ctx_limit;             // min(max_context_len, max_blocks_per_seq * block_size)
+  int32_t num_seqs;
+  int32_t num_heads;
+  int32_t num_kv_heads;
+  int32_t block_size;
+  float scale_log2;              // softmax scale * log2(e)
+};
+
+// Failure site of a prefill wait that gave up.
+enum : int32_t { kSitePrefill = 5 };
+
+// Launch for one (q dtype == cache dtype) pair; q_tiles = ceil(max_query_len
+// / tokens per CTA) is computed inside. cudaErrorNotSupported for shapes
+// without a kernel.
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                           int q_dtype, int head_dim, int group, int32_t max_query_len,
+                           cudaStream_t stream);
+
+}  // namespace paged

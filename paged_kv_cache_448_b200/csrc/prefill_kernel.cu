@@ -1,0 +1,347 @@
+// prefill_kernel.cu — attention of several query tokens per sequence over the
+// paged cache (chunked prefill, verification of draft tokens).
+//
+// The q_len_s query rows of sequence s are its last positions,
+// p_i = ctx_s - q_len_s + i; row i attends to the tokens t <= p_i of the
+// sequence, found through its block table ("vLLM推理引擎架构：PagedAttention
+// 机制与高吞吐推理" §2.3: attention over the blocks a block table names, here
+// with a query tensor of more rows than sequences, and the causal rule of
+// autoregressive attention).
+//
+// Unlike decode this is a dense contraction: a CTA owns 64 rows, a row being
+// one (query token, head of the kv-head's group), i.e. 64/G consecutive query
+// tokens of one (sequence, kv-head); each of its 4 warps owns 16 rows. The
+// K/V tiles of that kv-head (16 tokens, the decode kernel's TMA box and
+// swizzled layout) stream through an R-stage ring shared by the CTA: one
+// thread issues the TMA loads (full barriers with transaction counts), every
+// warp reads every tile and releases it (empty barriers, one arrival per
+// warp). Per tile a warp computes S = Q K^T (16 x 16, mma.sync m16n8k16,
+// fp32 accumulators; K as the B operand by ldmatrix), masks tokens after each
+// row's position, runs the online softmax in base 2 and accumulates
+// O += P V with P re-packed from the S accumulators as the A operand and V
+// transposed by ldmatrix.trans. Every wait is bounded by wall time.
+#include <math_constants.h>
+
+#include "consumer_mma.cuh"
+#include "decode_args.h"
+#include "decode_kernel.cuh"
+#include "device_common.cuh"
+#include "prefill_args.h"
+
+namespace paged {
+namespace {
+
+constexpr int kPrefillWarps = 4;
+constexpr int kPrefillRows = 16 * kPrefillWarps;  // rows (token x head) per CTA
+constexpr int kPrefillStages = 6;
+
+// D[16 x 8] += A[16 x 16] . B[16 x 8] (all 16 rows live).
+template <bool BF>
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  if constexpr (BF) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+template <class QF, int D, int G>
+__global__ void __launch_bounds__(kPrefillWarps * 32)
+    paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap kmap,
+                         const __grid_constant__ CUtensorMap vmap) {
+  using T = Tile<QF, D>;
+  constexpr bool BF = std::is_same<QF, BF16>::value;
+  constexpr int R = kPrefillStages, NW = kPrefillWarps, TR = kTileRows;
+  constexpr int QT = kPrefillRows / G;  // query tokens per CTA
+  constexpr int KS = D / 16, NO = D / 8;
+  constexpr int STAGE = 2 * T::BYTES;
+  constexpr unsigned FULL = 0xffffffffu;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + R * STAGE);
+  uint64_t* empty = full + R;
+  __shared__ int aborted;
+
+  const int z = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int r = 0; r < R; ++r) {
+      mbar_init(&full[r], 1);
+      mbar_init(&empty[r], NW);
+    }
+    fence_mbar_init();
+    aborted = 0;
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  __syncthreads();
+  // Everything below reads data of earlier kernels in the stream.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  const int q0 = a.cu_query_lens[s];
+  const int qlen = a.cu_query_lens[s + 1] - q0;
+  int ctx = a.context_lens[s];
+  if (ctx > a.ctx_limit || ctx < 0) {
+    if (threadIdx.x == 0 && z == 0 && kvh == 0) report(a.err, kErrContextClipped);
+    ctx = ctx < 0 ? 0 : a.ctx_limit;
+  }
+  const int tok0 = z * QT;
+  if (tok0 >= qlen) return;  // ragged chunk lengths: nothing for this CTA
+  const int ntok = min(QT, qlen - tok0);
+
+  // rows of this lane: r_lo and r_lo + 8 of the warp's 16; row = token * G + head
+  const int c = lane & 3;
+  const int r_lo = warp * 16 + (lane >> 2), r_hi = r_lo + 8;
+  const int tk_lo = r_lo / G, tk_hi = r_hi / G;
+  const bool v_lo = tk_lo < ntok, v_hi = tk_hi < ntok;
+  const int64_t row_lo = (static_cast<int64_t>(q0 + tok0 + tk_lo) * a.num_heads + kvh * G +
+                          r_lo % G) * D;
+  const int64_t row_hi = (static_cast<int64_t>(q0 + tok0 + tk_hi) * a.num_heads + kvh * G +
+                          r_hi % G) * D;
+
+  if (qlen > ctx) {  // a query longer than its context: rows become zeros
+    if (threadIdx.x == 0 && z == 0 && kvh == 0) report(a.err, kErrQueryLonger);
+    uint32_t* out32 = static_cast<uint32_t*>(a.out);
+    for (int j = 0; j < NO; ++j) {
+      if (v_lo) out32[(row_lo + j * 8 + 2 * c) / 2] = 0u;
+      if (v_hi) out32[(row_hi + j * 8 + 2 * c) / 2] = 0u;
+    }
+    return;
+  }
+  const int pos0 = ctx - qlen + tok0;       // position of the CTA's first query token
+  const int ntiles = (pos0 + ntok - 1) / TR + 1;
+  const int p_lo = v_lo ? pos0 + tk_lo : -1, p_hi = v_hi ? pos0 + tk_hi : -1;
+  const int p_min = min(p_lo, p_hi);
+
+  const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
+  const uint64_t policy = l2_policy_evict_last();  // the other query tiles read them too
+  const bool producer = threadIdx.x == 0;
+  auto issue = [&](int t) {
+    const int stage = t % R;
+    int32_t bid = table[(t * TR) / a.block_size];
+    if (bid < 0 || bid >= a.num_blocks) {
+      report(a.err, kErrBadBlockId);
+      bid = -1;  // read as a box outside the pool: zero-filled
+    }
+    const int32_t row0 = bid >= 0 ? bid * a.block_size + (t * TR) % a.block_size : -TR;
+    uint8_t* kt = smem + stage * STAGE;
+    mbar_arrive_expect_tx(&full[stage], STAGE);
+    tma_load_4d(kt, &kmap, &full[stage], 0, row0, kvh, 0, policy);
+    tma_load_4d(kt + T::BYTES, &vmap, &full[stage], 0, row0, kvh, 0, policy);
+  };
+  int issued = 0;
+  if (producer) {
+    for (; issued < min(R - 1, ntiles); ++issued) issue(issued);
+  }
+
+  // Q fragments (A operand, rows r_lo / r_hi, k-steps of 16 dims)
+  uint32_t qa[KS][4];
+  {
+    const uint32_t* q32 = static_cast<const uint32_t*>(a.query);
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      qa[kk][0] = v_lo ? q32[(row_lo + kk * 16 + 2 * c) / 2] : 0u;
+      qa[kk][1] = v_hi ? q32[(row_hi + kk * 16 + 2 * c) / 2] : 0u;
+      qa[kk][2] = v_lo ? q32[(row_lo + kk * 16 + 8 + 2 * c) / 2] : 0u;
+      qa[kk][3] = v_hi ? q32[(row_hi + kk * 16 + 8 + 2 * c) / 2] : 0u;
+    }
+  }
+  float o[NO][4];
+#pragma unroll
+  for (int j = 0; j < NO; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_lo = -CUDART_INF_F, m_hi = -CUDART_INF_F, l_lo = 0.f, l_hi = 0.f;
+  const float qscale = a.scale_log2;
+
+  int t = 0;
+  for (; t < ntiles; ++t) {
+    if (producer && issued < ntiles) {
+      // refill the stage tile t-1 used once every warp has released it
+      if (t >= 1 && !mbar_wait(&empty[(t - 1) % R], ((t - 1) / R) & 1, &aborted)) {
+        aborted = 1;
+        record_failure(a.diag, kSitePrefill, blockIdx.x, blockIdx.y, blockIdx.z, t, issued,
+                       ntiles, 1);
+      } else if (!aborted) {
+        issue(issued++);
+      }
+    }
+    const int stage = t % R;
+    if (!__all_sync(FULL, mbar_wait(&full[stage], (t / R) & 1, &aborted))) break;
+    const uint8_t* kt = smem + stage * STAGE;
+    uint8_t* vt = smem + stage * STAGE + T::BYTES;
+
+    // ---- S = Q K^T over this tile's 16 tokens
+    float sacc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+      const int row = nt * 8 + (lane & 7);
+#pragma unroll
+      for (int kk = 0; kk < KS; kk += 2) {
+        uint32_t b[4];
+        ldsm_x4(kt + T::off(row, (2 * kk + (lane >> 3)) * 16), b);
+        mma_16816<BF>(sacc[nt], qa[kk], b[0], b[1]);
+        mma_16816<BF>(sacc[nt], qa[kk + 1], b[2], b[3]);
+      }
+    }
+    // ---- causal mask (tokens after a row's position), scale, online softmax
+    const int tok_base = t * TR;
+    const bool masked = tok_base + TR - 1 > p_min;
+    float mx_lo = -CUDART_INF_F, mx_hi = -CUDART_INF_F;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tok = tok_base + nt * 8 + 2 * c + (i & 1);
+        const int p = i < 2 ? p_lo : p_hi;
+        const float x = (!masked || tok <= p) ? sacc[nt][i] * qscale : -CUDART_INF_F;
+        sacc[nt][i] = x;
+        if (i < 2) mx_lo = fmaxf(mx_lo, x);
+        else mx_hi = fmaxf(mx_hi, x);
+      }
+    mx_lo = fmaxf(mx_lo, __shfl_xor_sync(FULL, mx_lo, 1));
+    mx_lo = fmaxf(mx_lo, __shfl_xor_sync(FULL, mx_lo, 2));
+    mx_hi = fmaxf(mx_hi, __shfl_xor_sync(FULL, mx_hi, 1));
+    mx_hi = fmaxf(mx_hi, __shfl_xor_sync(FULL, mx_hi, 2));
+    const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
+    const float mu_lo = mn_lo == -CUDART_INF_F ? 0.f : mn_lo;
+    const float mu_hi = mn_hi == -CUDART_INF_F ? 0.f : mn_hi;
+    const float al_lo = exp2f(m_lo - mu_lo), al_hi = exp2f(m_hi - mu_hi);
+    m_lo = mn_lo;
+    m_hi = mn_hi;
+    float ps_lo = 0.f, ps_hi = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      sacc[nt][0] = exp2f(sacc[nt][0] - mu_lo);
+      sacc[nt][1] = exp2f(sacc[nt][1] - mu_lo);
+      sacc[nt][2] = exp2f(sacc[nt][2] - mu_hi);
+      sacc[nt][3] = exp2f(sacc[nt][3] - mu_hi);
+      ps_lo += sacc[nt][0] + sacc[nt][1];
+      ps_hi += sacc[nt][2] + sacc[nt][3];
+    }
+    l_lo = l_lo * al_lo + ps_lo;
+    l_hi = l_hi * al_hi + ps_hi;
+#pragma unroll
+    for (int j = 0; j < NO; ++j) {
+      o[j][0] *= al_lo;
+      o[j][1] *= al_lo;
+      o[j][2] *= al_hi;
+      o[j][3] *= al_hi;
+    }
+    // Rows of the tile past the context may hold anything (even NaN) and
+    // 0 * NaN is NaN inside the MMA: each warp clears them in its view of the
+    // stage before reading V (every warp writes the same zeros; the stage is
+    // not refilled after the last tile).
+    if (tok_base + TR > ctx) {
+      constexpr int CPR = T::RB / 16;
+      const int first = max(0, ctx - tok_base);
+      for (int i = lane; i < (TR - first) * CPR; i += 32)
+        *reinterpret_cast<uint4*>(vt + T::off(first + i / CPR, (i % CPR) * 16)) =
+            make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+    }
+    // ---- O += P V (P from the S accumulators, as the A operand). bf16 keeps
+    // only 8 significant bits, too few for rows that see a handful of tokens;
+    // there P = P_hi + P_lo, both bf16, in two MMAs (about 16 bits).
+    uint32_t pa[4], pl[4];
+    pa[0] = pack2<BF>(sacc[0][0], sacc[0][1]);
+    pa[1] = pack2<BF>(sacc[0][2], sacc[0][3]);
+    pa[2] = pack2<BF>(sacc[1][0], sacc[1][1]);
+    pa[3] = pack2<BF>(sacc[1][2], sacc[1][3]);
+    if constexpr (BF) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float* src = sacc[k >> 1] + 2 * (k & 1);
+        pl[k] = pack2<true>(src[0] - __uint_as_float(pa[k] << 16),
+                            src[1] - __uint_as_float(pa[k] & 0xffff0000u));
+      }
+    }
+    const int vrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int dn = 0; dn < NO; dn += 2) {
+      uint32_t b[4];
+      ldsm_x4_trans(vt + T::off(vrow, (dn + (lane >> 4)) * 16), b);
+      mma_16816<BF>(o[dn], pa, b[0], b[1]);
+      mma_16816<BF>(o[dn + 1], pa, b[2], b[3]);
+      if constexpr (BF) {
+        mma_16816<BF>(o[dn], pl, b[0], b[1]);
+        mma_16816<BF>(o[dn + 1], pl, b[2], b[3]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+  }
+  if (t < ntiles) {
+    // A wait gave up (never expected): record it and let the loads this CTA
+    // issued land (bounded) before its shared memory goes away.
+    if (lane == 0) {
+      aborted = 1;
+      record_failure(a.diag, kSitePrefill, blockIdx.x, blockIdx.y, blockIdx.z, warp, t, ntiles,
+                     0);
+      report(a.err, kErrWaitTimeout);
+    }
+    if (producer)
+      for (int k = t; k < issued; ++k) mbar_wait(&full[k % R], (k / R) & 1);
+    return;
+  }
+
+  // ---- epilogue: out = O / l, rounded to the q dtype
+  l_lo += __shfl_xor_sync(FULL, l_lo, 1);
+  l_lo += __shfl_xor_sync(FULL, l_lo, 2);
+  l_hi += __shfl_xor_sync(FULL, l_hi, 1);
+  l_hi += __shfl_xor_sync(FULL, l_hi, 2);
+  const float i_lo = l_lo > 0.f ? 1.f / l_lo : 0.f, i_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
+  uint32_t* out32 = static_cast<uint32_t*>(a.out);
+#pragma unroll
+  for (int j = 0; j < NO; ++j) {
+    if (v_lo) out32[(row_lo + j * 8 + 2 * c) / 2] = pack2<BF>(o[j][0] * i_lo, o[j][1] * i_lo);
+    if (v_hi) out32[(row_hi + j * 8 + 2 * c) / 2] = pack2<BF>(o[j][2] * i_hi, o[j][3] * i_hi);
+  }
+}
+
+template <class QF, int D, int G>
+cudaError_t launch_one(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                       int32_t max_query_len, cudaStream_t stream) {
+  constexpr int QT = kPrefillRows / G;
+  constexpr int STAGE = 2 * Tile<QF, D>::BYTES;
+  const size_t smem = 1024 + kPrefillStages * STAGE + 16 * kPrefillStages;
+  auto kern = paged_prefill_kernel<QF, D, G>;
+  cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  const unsigned tiles = static_cast<unsigned>((max_query_len + QT - 1) / QT);
+  return launch_pdl(kern, dim3(tiles, a.num_kv_heads, a.num_seqs), kPrefillWarps * 32, smem,
+                    stream, a, kmap, vmap);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                           int q_dtype, int head_dim, int group, int32_t max_query_len,
+                           cudaStream_t stream) {
+#define PAGED_PREFILL(QF, d, g) \
+  if (head_dim == d && group == g) return launch_one<QF, d, g>(a, kmap, vmap, max_query_len, stream);
+#define PAGED_PREFILL_ALL(QF)                                                   \
+  PAGED_PREFILL(QF, 64, 1) PAGED_PREFILL(QF, 64, 2) PAGED_PREFILL(QF, 64, 4)     \
+  PAGED_PREFILL(QF, 64, 8) PAGED_PREFILL(QF, 128, 1) PAGED_PREFILL(QF, 128, 2)   \
+  PAGED_PREFILL(QF, 128, 4) PAGED_PREFILL(QF, 128, 8)
+  if (q_dtype == kF16) {
+    PAGED_PREFILL_ALL(F16)
+  } else if (q_dtype == kBF16) {
+    PAGED_PREFILL_ALL(BF16)
+  }
+#undef PAGED_PREFILL_ALL
+#undef PAGED_PREFILL
+  return cudaErrorNotSupported;
+}
+
+}  // namespace paged

@@ -112,6 +112,78 @@ def spec(config: int, seed: int | None = None, *, small: bool = False) -> Spec:
     raise ValueError(f"unknown config {config}")
 
 
+# ---------------------------------------------------- multi-token queries
+
+PREFILL_NAMES = ("chunk_llama7b", "chunk_gqa70b", "verify_gqa70b")
+
+
+def prefill_spec(name: str, seed: int | None = None, *, small: bool = False):
+    """(Spec, query_lens) of a multi-token query workload. context_lens include
+    the query tokens (its last positions); shapes follow the decode workloads:
+
+    * ``chunk_llama7b``  chunked prefill on the LLaMA-7B shape: 16 sequences,
+      a 512-token chunk after a prior context uniform in [0, 3584]; 32 heads,
+      head_dim 128, block_size 16, fp16.
+    * ``chunk_gqa70b``   chunked prefill on the 70B GQA shape: 16 sequences, a
+      256-token chunk after a log-uniform prior context in [1024, 8192];
+      64 query / 8 kv heads, block_size 32, bf16.
+    * ``verify_gqa70b``  verification of 8 draft tokens for 64 sequences with
+      prior contexts uniform in [1024, 4096]; 64 / 8 heads, block_size 16, bf16.
+    """
+    if seed is None:
+        seed = 2000 + PREFILL_NAMES.index(name)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    if name == "chunk_llama7b":
+        S, chunk, lo, hi, H, Hkv, bs, dt = (3, 40, 0, 100, 4, 4, 16, "f16") if small else \
+            (16, 512, 0, 3584, 32, 32, 16, "f16")
+        prior = _uniform_ints(rng, lo, hi, S)
+    elif name == "chunk_gqa70b":
+        S, chunk, lo, hi, H, Hkv, bs, dt = (3, 33, 10, 150, 16, 2, 32, "bf16") if small else \
+            (16, 256, 1024, 8192, 64, 8, 32, "bf16")
+        prior = np.round(np.exp(rng.uniform(math.log(lo), math.log(hi), size=S))).astype(np.int32)
+    elif name == "verify_gqa70b":
+        S, chunk, lo, hi, H, Hkv, bs, dt = (5, 8, 5, 100, 16, 2, 16, "bf16") if small else \
+            (64, 8, 1024, 4096, 64, 8, 16, "bf16")
+        prior = _uniform_ints(rng, lo, hi, S)
+    else:
+        raise ValueError(f"unknown multi-token workload {name}")
+    qlens = np.full(S, chunk, np.int32)
+    sp = Spec(name, S, H, Hkv, 128, bs, dt, dt, 1.0 / math.sqrt(128),
+              (prior + qlens).astype(np.int32), seed=seed)
+    return sp, qlens
+
+
+def prefill_queries_host(sp: Spec, qlens: np.ndarray) -> np.ndarray:
+    """Raw codes [sum(qlens), H, D] of N(0,1) query rows."""
+    rng = np.random.Generator(np.random.PCG64(sp.seed + 17))
+    q = rng.standard_normal((int(qlens.sum()), sp.num_heads, sp.head_dim), dtype=np.float32)
+    return _f32_to_codes(q, sp.q_dtype)
+
+
+def prefill_queries_device(sp: Spec, qlens: np.ndarray, device="cuda"):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(sp.seed + 19)
+    return torch.randn((int(qlens.sum()), sp.num_heads, sp.head_dim), generator=g, device=device,
+                       dtype=torch.float32).to(torch_dtype(sp.q_dtype))
+
+
+def prefill_flops(sp: Spec, qlens: np.ndarray) -> int:
+    """Algorithmic FLOPs: every query row and head against each visible key,
+    2 * head_dim for q.k and 2 * head_dim for p.v."""
+    ctx = sp.context_lens.astype(np.int64)
+    q = qlens.astype(np.int64)
+    visible = (ctx * q - q * (q - 1) // 2).sum()    # sum over rows of (position + 1)
+    return int(visible) * sp.num_heads * sp.head_dim * 4
+
+
+def prefill_bytes(sp: Spec, qlens: np.ndarray) -> int:
+    """Algorithmic bytes: K/V of every context token once per kv-head, the
+    query rows and the output rows."""
+    rows = int(qlens.sum()) * sp.num_heads * sp.head_dim * 2
+    return kv_bytes(sp) + 2 * rows
+
+
 def structure(sp: Spec) -> Structure:
     """Block tables from a seeded permutation of the pool: ids are handed out
     in permutation order, sequence by sequence (shared prefixes once per

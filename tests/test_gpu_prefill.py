@@ -1,0 +1,155 @@
+"""GPU parity of the multi-token query path (pa_chunked_prefill) against the
+oracle: the three multi-token workloads at reduced size, an edge sweep over
+chunk / context lengths, head_dim, block_size, query group and dtype, a
+one-token-per-sequence case against decode, error reporting, and the
+full-size workloads in the launch configuration the benchmark times,
+compared on sampled sequences."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_448_b200 as pk
+from paged_kv_cache_448_b200 import workloads as wl
+from gpu_helpers import assert_close, dev, host_codes, i32
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(sp, st, hd, q, qlens, table=None, ctx=None):
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    ctx = sp.context_lens if ctx is None else ctx
+    table = st.block_tables if table is None else table
+    gq = dev(q, sp.q_dtype)
+    out = torch.full_like(gq, float("nan"))
+    ws = pk.decode_workspace(1, 1, 1, sp.head_dim, sp.block_size, 0, 0)
+    pk.chunked_prefill(out, gq, i32(cu), int(qlens.max()), dev(hd.key_cache, sp.cache_dtype),
+                       dev(hd.value_cache, sp.cache_dtype), i32(table), i32(ctx),
+                       int(np.max(ctx)), sp.scale, workspace=ws)
+    return out, ws, cu
+
+
+def run_oracle(sp, st, hd, q, cu, table=None, ctx=None):
+    return oracle.chunked_prefill(q, hd.key_cache, hd.value_cache,
+                                  st.block_tables if table is None else table,
+                                  sp.context_lens if ctx is None else ctx, cu,
+                                  scale=np.float32(sp.scale), q_dtype=sp.q_dtype,
+                                  cache_dtype=sp.cache_dtype)
+
+
+@pytest.mark.parametrize("name", wl.PREFILL_NAMES)
+def test_multi_token_workloads_small(name):
+    sp, qlens = wl.prefill_spec(name, small=True)
+    st = wl.structure(sp)
+    hd = wl.host_data(sp, st)
+    q = wl.prefill_queries_host(sp, qlens)
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), sp.cache_dtype, name)
+
+
+def custom(ctxs, qlens, H, Hkv, D, bs, dt, seed):
+    sp = wl.Spec("custom", len(ctxs), H, Hkv, D, bs, dt, dt, 1.0 / math.sqrt(D),
+                 np.array(ctxs, np.int32), spare_blocks=3, seed=seed)
+    st = wl.structure(sp)
+    hd = wl.host_data(sp, st)
+    q = wl.prefill_queries_host(sp, np.array(qlens, np.int32))
+    return sp, st, hd, q, np.array(qlens, np.int32)
+
+
+# chunk lengths cross CTA tiles (64 / G tokens) and K tiles (16 tokens), with a
+# full prefill (q_len == ctx), single tokens, and a context of one token
+EDGE = ([1, 17, 40, 100, 33, 130], [1, 17, 9, 70, 1, 65])
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_multi_token_edge_sweep(dt, G, D, bs):
+    sp, st, hd, q, qlens = custom(*EDGE, 2 * G, 2, D, bs, dt, seed=G * 100 + D + bs)
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), dt,
+                 f"{dt} G{G} D{D} bs{bs}")
+
+
+def test_one_token_per_sequence_matches_decode_and_oracle():
+    sp, st, hd, q, qlens = custom([5, 64, 300, 1], [1, 1, 1, 1], 16, 2, 128, 16, "bf16", seed=5)
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens)
+    ref = run_oracle(sp, st, hd, q, cu)
+    assert_close(out.double().cpu().numpy(), ref, "bf16", "one token")
+    dout = torch.empty_like(out)
+    pk.decode(dout, dev(q, "bf16"), dev(hd.key_cache, "bf16"), dev(hd.value_cache, "bf16"),
+              i32(st.block_tables), i32(sp.context_lens), int(sp.context_lens.max()), sp.scale)
+    assert_close(dout.double().cpu().numpy(), ref, "bf16", "decode")
+
+
+def test_errors_are_reported_not_faulted():
+    sp, st, hd, q, qlens = custom([40, 70], [40, 10], 8, 2, 128, 16, "f16", seed=6)
+    bad = st.block_tables.copy()
+    bad[1, 1] = st.num_blocks + 9                 # outside the pool: read as zeros
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens, table=bad)
+    with pytest.raises(pk.PagedError) as e:
+        pk.decode_check(ws)
+    assert e.value.status == 5
+    assert torch.isfinite(out.float()).all()
+    # a chunk longer than its context: its rows are zeros, the rest is right
+    ctx = np.array([30, 70], np.int32)
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens, ctx=ctx)
+    with pytest.raises(pk.PagedError):
+        pk.decode_check(ws)
+    o = out.double().cpu().numpy()
+    assert np.all(o[:40] == 0.0)
+    ref = oracle.chunked_prefill(q[40:], hd.key_cache, hd.value_cache, st.block_tables[1:],
+                                 ctx[1:], np.array([0, 10], np.int32), scale=np.float32(sp.scale),
+                                 q_dtype="f16", cache_dtype="f16")
+    assert_close(o[40:], ref, "f16", "second sequence")
+
+
+def test_block_permutation_keeps_the_bits():
+    sp, st, hd, q, qlens = custom([90, 45], [50, 45], 8, 8, 64, 16, "bf16", seed=7)
+    base, _, cu = run_gpu(sp, st, hd, q, qlens)
+    pi = np.random.default_rng(1).permutation(st.num_blocks)
+    kc = np.empty_like(hd.key_cache); vc = np.empty_like(hd.value_cache)
+    kc[pi] = hd.key_cache; vc[pi] = hd.value_cache
+    table = np.where(st.block_tables >= 0, pi[np.maximum(st.block_tables, 0)], -1)
+    hd2 = wl.HostData(hd.query, kc, vc, hd.new_key, hd.new_value, None, None)
+    out, _, _ = run_gpu(sp, st, hd2, q, qlens, table=table.astype(np.int32))
+    assert np.array_equal(host_codes(out), host_codes(base))
+
+
+@pytest.mark.parametrize("name", wl.PREFILL_NAMES)
+def test_multi_token_full_size_sampled(name):
+    """Full-size workload in the benchmark's launch configuration; the oracle
+    checks the shortest sequence's rows (and the longest's last chunk rows
+    for the verification workload, whose chunks are short)."""
+    sp, qlens = wl.prefill_spec(name)
+    st = wl.structure(sp)
+    d = wl.device_data(sp, st)
+    q = wl.prefill_queries_device(sp, qlens)
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    out = torch.empty_like(q)
+    ws = pk.decode_workspace(1, 1, 1, sp.head_dim, sp.block_size, 0, 0)
+    pk.chunked_prefill(out, q, i32(cu), int(qlens.max()), d["key_cache"], d["value_cache"],
+                       i32(st.block_tables), i32(sp.context_lens), int(sp.context_lens.max()),
+                       sp.scale, workspace=ws)
+    pk.decode_check(ws)
+    assert torch.isfinite(out.float()).all()
+    picks = [int(np.argmin(sp.context_lens))]
+    if name == "verify_gqa70b":
+        picks.append(int(np.argmax(sp.context_lens)))
+    for s in picks:
+        ids = st.seq_block_ids[s]
+        sel = torch.tensor(ids, device="cuda")
+        kc = host_codes(d["key_cache"].index_select(0, sel))
+        vc = host_codes(d["value_cache"].index_select(0, sel))
+        table = np.arange(len(ids), dtype=np.int32)[None, :]
+        qs = host_codes(q[cu[s]:cu[s + 1]])
+        ref = oracle.chunked_prefill(qs, kc, vc, table, sp.context_lens[[s]],
+                                     np.array([0, qlens[s]], np.int32), scale=np.float32(sp.scale),
+                                     q_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype)
+        assert_close(out[cu[s]:cu[s + 1]].double().cpu().numpy(), ref, sp.cache_dtype,
+                     f"{name} seq {s}")
