@@ -44,6 +44,7 @@ from paged_kv_cache_448_b200 import workloads as wl  # noqa: E402
 METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode tokens/s per layer"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def log(*a):
@@ -59,6 +60,12 @@ def parse():
     ap.add_argument("--config", type=int, default=2, help="workload 1..5 (2 = headline)")
     ap.add_argument("--partition", type=int, default=-1,
                     help="decode partition tokens (-1: the workload's setting, 0: automatic)")
+    ap.add_argument("--op", choices=["decode", "prefill", "copy_blocks", "swap"],
+                    default="decode",
+                    help="decode: the headline step; the others time the multi-token query "
+                         "path or the block-copy kernel on their own workloads")
+    ap.add_argument("--workload", default="chunk_llama7b",
+                    help="multi-token workload for --op prefill: " + ", ".join(wl.PREFILL_NAMES))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -73,6 +80,15 @@ def measured_peaks():
             j = json.load(f)
         return float(j["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor TFLOP/s (burst: a kernel timed alone)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def sources_digest() -> str:
@@ -257,8 +273,182 @@ def job_throughput_gbs(world: int, bytes_per_rank: int, ms: float) -> float:
 
 # ------------------------------------------------------------------ GPU arm
 
+# ------------------------------------------------ other rows of the hot path
+
+def _time_device(fn, steps, warmup):
+    """Mean ms per call over `steps` calls (CUDA events on the current stream)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def prefill_oracle_sample(sp, qlens, budget_s):
+    """Oracle timing on the first sequences of the multi-token workload (all
+    heads, full contexts), as many as fit about `budget_s` seconds."""
+    import oracle
+    oracle.build()
+    done, t_total, flops = 0, 0.0, 0
+    while done < sp.num_seqs and t_total < budget_s:
+        sub = dataclasses.replace(sp, num_seqs=1, context_lens=sp.context_lens[done:done + 1].copy(),
+                                  spare_blocks=0)
+        st = wl.structure(sub)
+        hd = wl.host_data(sub, st)
+        ql = qlens[done:done + 1]
+        q = wl.prefill_queries_host(sub, ql)
+        t0 = time.perf_counter()
+        oracle.chunked_prefill(q, hd.key_cache, hd.value_cache, st.block_tables, sub.context_lens,
+                               np.array([0, ql[0]], np.int32), scale=np.float32(sp.scale),
+                               q_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype)
+        t_total += time.perf_counter() - t0
+        flops += wl.prefill_flops(sub, ql)
+        done += 1
+    return {"value": round(flops / t_total / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"first {done} of {sp.num_seqs} sequences (all heads, whole chunks); "
+                      f"{t_total:.1f} s single-threaded fp64 C"}
+
+
+def run_prefill(args):
+    """--op prefill: the multi-token query path on one multi-token workload."""
+    import torch
+    import paged_kv_cache_448_b200 as pk
+    sp, qlens = wl.prefill_spec(args.workload)
+    flops, nbytes = wl.prefill_flops(sp, qlens), wl.prefill_bytes(sp, qlens)
+    chunk = int(qlens.max())
+    config = {"workload": f"{sp.name}: {sp.num_seqs} seqs x {chunk} query tokens, ctx "
+                          f"{int(sp.context_lens.min())}-{int(sp.context_lens.max())}, "
+                          f"{sp.num_heads} q / {sp.num_kv_heads} kv heads, head_dim {sp.head_dim}, "
+                          f"block_size {sp.block_size}, {sp.q_dtype}"}
+    # tensor-bound when the work per K/V byte is above the machine balance
+    peak_t, kind_t = measured_tensor_peak()
+    peak_b, kind_b = measured_peaks()
+    tensor_bound = flops / nbytes > peak_t * 1e12 / (peak_b * 1e9)
+    if args.impl == "reference":
+        cb = prefill_oracle_sample(sp, qlens, args.cpu_seconds)
+        print(json.dumps({"metric": "multi-token paged attention TFLOP/s", "impl": "reference",
+                          "value": cb["value"], "unit": "TFLOP/s", "n_gpus": 1,
+                          "higher_is_better": True, "config": config, "cpu_baseline": cb,
+                          "e2e": {"value": cb["value"], "unit": "TFLOP/s",
+                                  "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return
+    dev = torch.device("cuda", 0)
+    st = wl.structure(sp)
+    d = wl.device_data(sp, st, device=dev)
+    q = wl.prefill_queries_device(sp, qlens, device=dev)
+    cu = torch.from_numpy(np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)).to(dev)
+    bt = torch.from_numpy(st.block_tables).to(dev)
+    cl = torch.from_numpy(sp.context_lens).to(dev)
+    out = torch.empty_like(q)
+    ws = pk.decode_workspace(1, 1, 1, sp.head_dim, sp.block_size, 0, 0, device=dev)
+    mctx = int(sp.context_lens.max())
+    fn = lambda: pk.chunked_prefill(out, q, cu, chunk, d["key_cache"], d["value_cache"], bt, cl,
+                                    mctx, sp.scale, workspace=ws)
+    sampler = ClockSampler(0)
+    sampler.start()
+    ms = _time_device(fn, args.steps, max(3, args.warmup))
+    clocks = sampler.stop()
+    pk.decode_check(ws)
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    roof = ({"bound": "tensor", "achieved": round(tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
+             "frac": round(tflops / peak_t, 4), "peak_kind": f"{kind_t} dense bf16 (cuBLAS)"}
+            if tensor_bound else
+            {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak_b, "unit": "GB/s",
+             "frac": round(gbs / peak_b, 4), "peak_kind": f"{kind_b} HBM copy GB/s"})
+    roof.update({"traffic": None, "algorithmic_flops_per_launch": flops,
+                 "algorithmic_bytes_per_launch": nbytes, "launch_ms": round(ms, 5)})
+    line = {"metric": "multi-token paged attention TFLOP/s", "value": round(tflops, 3),
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": sp.q_dtype, "data": "synthetic", "config": config,
+            "gb_per_s": round(gbs, 2),
+            "query_tokens_per_s": round(int(qlens.sum()) / (ms * 1e-3), 1),
+            "roofline": roof, "gpu_launches": args.steps, "clocks": clocks}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_oracle_sample(sp, qlens, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def run_copy(args):
+    """--op copy_blocks: copy-on-write copies of 2048 random block pairs inside
+    the LLaMA-7B-shaped cache (K and V); --op swap: 512 of its blocks out to a
+    pinned host pool and back in."""
+    import torch
+    import paged_kv_cache_448_b200 as pk
+    dev = torch.device("cuda", 0)
+    NB, BS, H, D = 4352, 16, 32, 128
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    k = torch.randn((NB, BS, H, D), generator=g, device=dev, dtype=torch.float32).half()
+    v = torch.randn((NB, BS, H, D), generator=g, device=dev, dtype=torch.float32).half()
+    bb = BS * H * D * 2
+    rng = np.random.default_rng(1234)
+    perm = rng.permutation(NB)
+    sampler = ClockSampler(0)
+    if args.op == "copy_blocks":
+        n = 2048
+        pairs = torch.from_numpy(np.stack([perm[:n], perm[n:2 * n]], 1).astype(np.int32)).to(dev)
+        sampler.start()
+        ms = _time_device(lambda: pk.copy_blocks(k, v, k, v, pairs), args.steps,
+                          max(3, args.warmup))
+        clocks = sampler.stop()
+        moved = 2 * 2 * n * bb                                     # read + write, K and V
+        peak, kind = measured_peaks()
+        gbs = moved / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak, "unit": "GB/s",
+                "frac": round(gbs / peak, 4), "peak_kind": f"{kind} HBM copy GB/s",
+                "traffic": None, "algorithmic_bytes_per_launch": moved, "launch_ms": round(ms, 5)}
+        metric, workload = "block copy GB/s (read + write)", \
+            f"copy-on-write: {n} block pairs of a 4352-block fp16 cache (16 x 32 x 128), K and V"
+    else:
+        n = 512
+        hk = torch.empty((n, BS, H, D), dtype=torch.float16).pin_memory()
+        hv = torch.empty_like(hk).pin_memory()
+        out_p = torch.from_numpy(np.stack([perm[:n], np.arange(n)], 1).astype(np.int32)).to(dev)
+        in_p = torch.from_numpy(np.stack([np.arange(n), perm[n:2 * n]], 1).astype(np.int32)).to(dev)
+        sampler.start()
+        ms = _time_device(lambda: (pk.copy_blocks(k, v, hk, hv, out_p),
+                                   pk.copy_blocks(hk, hv, k, v, in_p)), args.steps,
+                          max(3, args.warmup))
+        clocks = sampler.stop()
+        big = torch.empty(n * bb, dtype=torch.uint8).pin_memory()
+        dbig = torch.empty(n * bb, dtype=torch.uint8, device=dev)
+        ref_ms = _time_device(lambda: (dbig.copy_(big, non_blocking=True),
+                                       big.copy_(dbig, non_blocking=True)), 5, 2)
+        moved = 2 * 2 * n * bb                                     # out and in, K and V
+        peak = round(2 * n * bb / (ref_ms * 1e-3) / 1e9, 2)
+        gbs = moved / (ms * 1e-3) / 1e9
+        roof = {"bound": "pcie", "achieved": round(gbs, 2), "peak": peak, "unit": "GB/s",
+                "frac": round(gbs / peak, 4),
+                "peak_kind": "measured in this run: contiguous pinned cudaMemcpy, one H2D + one D2H",
+                "traffic": None, "algorithmic_bytes_per_launch": moved, "launch_ms": round(ms, 5)}
+        metric, workload = "block swap GB/s (GPU <-> pinned host)", \
+            f"swap: {n} blocks of a 4352-block fp16 cache (16 x 32 x 128) out to pinned host and back, K and V"
+    print(json.dumps({"metric": metric, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": 1,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                      "dtype": "f16", "data": "synthetic", "config": {"workload": workload},
+                      "roofline": roof, "gpu_launches": args.steps * (1 if args.op == "copy_blocks" else 2),
+                      "clocks": clocks}), flush=True)
+
+
 def main():
     args = parse()
+    if args.op == "prefill":
+        run_prefill(args)
+        return
+    if args.op in ("copy_blocks", "swap"):
+        run_copy(args)
+        return
     sp = wl.spec(args.config)
     st = wl.structure(sp)
     if args.impl == "reference":

@@ -31,9 +31,17 @@
 namespace paged {
 namespace {
 
+#ifndef PAGED_PREFILL_TPS
+#define PAGED_PREFILL_TPS 1
+#endif
+#ifndef PAGED_PREFILL_RS
+#define PAGED_PREFILL_RS 4
+#endif
 constexpr int kPrefillWarps = 4;
 constexpr int kPrefillRows = 16 * kPrefillWarps;  // rows (token x head) per CTA
-constexpr int kPrefillStages = 6;
+constexpr int kPrefillTps = PAGED_PREFILL_TPS;    // 16-token tiles per softmax step
+constexpr int kPrefillRs = PAGED_PREFILL_RS;      // steps in flight in the ring
+constexpr int kPrefillStages = kPrefillRs * kPrefillTps;
 
 // D[16 x 8] += A[16 x 16] . B[16 x 8] (all 16 rows live).
 template <bool BF>
@@ -127,9 +135,8 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
   const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
   const uint64_t policy = l2_policy_evict_last();  // the other query tiles read them too
   const bool producer = threadIdx.x == 0;
-  auto issue = [&](int t) {
+  auto issue = [&](int t, int32_t bid) {
     const int stage = t % R;
-    int32_t bid = table[(t * TR) / a.block_size];
     if (bid < 0 || bid >= a.num_blocks) {
       report(a.err, kErrBadBlockId);
       bid = -1;  // read as a box outside the pool: zero-filled
@@ -140,10 +147,24 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
     tma_load_4d(kt, &kmap, &full[stage], 0, row0, kvh, 0, policy);
     tma_load_4d(kt + T::BYTES, &vmap, &full[stage], 0, row0, kvh, 0, policy);
   };
-  int issued = 0;
-  if (producer) {
-    for (; issued < min(R - 1, ntiles); ++issued) issue(issued);
-  }
+  // The producer loads the block ids of a whole step first, then issues its
+  // TMA boxes (the id loads overlap instead of preceding each box).
+  auto issue_step = [&](int k) {
+    int32_t bid[kPrefillTps];
+#pragma unroll
+    for (int j = 0; j < kPrefillTps; ++j) {
+      const int tt = k * kPrefillTps + j;
+      bid[j] = tt < ntiles ? table[(tt * TR) / a.block_size] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kPrefillTps; ++j) {
+      const int tt = k * kPrefillTps + j;
+      if (tt < ntiles) issue(tt, bid[j]);
+    }
+  };
+  const int nsteps = (ntiles + kPrefillTps - 1) / kPrefillTps;
+  if (producer)
+    for (int k = 0; k < min(kPrefillRs, nsteps); ++k) issue_step(k);
 
   // Q fragments (A operand, rows r_lo / r_hi, k-steps of 16 dims)
   uint32_t qa[KS][4];
@@ -163,52 +184,78 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
   float m_lo = -CUDART_INF_F, m_hi = -CUDART_INF_F, l_lo = 0.f, l_hi = 0.f;
   const float qscale = a.scale_log2;
 
-  int t = 0;
-  for (; t < ntiles; ++t) {
-    if (producer && issued < ntiles) {
-      // refill the stage tile t-1 used once every warp has released it
-      if (t >= 1 && !mbar_wait(&empty[(t - 1) % R], ((t - 1) / R) & 1, &aborted)) {
+  int k = 0, t = 0;  // step, and the first tile not yet received
+  bool failed = false;
+  for (; k < nsteps && !failed; ++k) {
+    const int t0 = k * kPrefillTps;
+    // refill the stages of step k-1 with step k+RS-1 once every warp released them
+    if (producer && k >= 1 && k + kPrefillRs - 1 < nsteps && !aborted) {
+      bool ok = true;
+      for (int j = 0; j < kPrefillTps && ok; ++j) {
+        const int tp = t0 - kPrefillTps + j;
+        ok = mbar_wait(&empty[tp % R], (tp / R) & 1, &aborted);
+      }
+      if (ok) {
+        issue_step(k + kPrefillRs - 1);
+      } else {
         aborted = 1;
-        record_failure(a.diag, kSitePrefill, blockIdx.x, blockIdx.y, blockIdx.z, t, issued,
-                       ntiles, 1);
-      } else if (!aborted) {
-        issue(issued++);
+        record_failure(a.diag, kSitePrefill, blockIdx.x, blockIdx.y, blockIdx.z, k, t0, ntiles,
+                       1);
       }
     }
-    const int stage = t % R;
-    if (!__all_sync(FULL, mbar_wait(&full[stage], (t / R) & 1, &aborted))) break;
-    const uint8_t* kt = smem + stage * STAGE;
-    uint8_t* vt = smem + stage * STAGE + T::BYTES;
-
-    // ---- S = Q K^T over this tile's 16 tokens
-    float sacc[2][4];
+    // ---- S = Q K^T over the step's tiles (16 tokens each)
+    float sacc[kPrefillTps][2][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-      const int row = nt * 8 + (lane & 7);
+    for (int j = 0; j < kPrefillTps; ++j) {
+      const int tt = t0 + j;
 #pragma unroll
-      for (int kk = 0; kk < KS; kk += 2) {
-        uint32_t b[4];
-        ldsm_x4(kt + T::off(row, (2 * kk + (lane >> 3)) * 16), b);
-        mma_16816<BF>(sacc[nt], qa[kk], b[0], b[1]);
-        mma_16816<BF>(sacc[nt], qa[kk + 1], b[2], b[3]);
+      for (int nt = 0; nt < 2; ++nt)
+        sacc[j][nt][0] = sacc[j][nt][1] = sacc[j][nt][2] = sacc[j][nt][3] = 0.f;
+      if (tt >= ntiles) continue;
+      if (!__all_sync(FULL, mbar_wait(&full[tt % R], (tt / R) & 1, &aborted))) {
+        failed = true;
+        break;
       }
+      t = tt + 1;
+      const uint8_t* kt = smem + (tt % R) * STAGE;
+      // even and odd k-steps in separate accumulators: two independent MMA
+      // chains per n-tile instead of one of length KS
+      float s2[2][4] = {};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int row = nt * 8 + (lane & 7);
+#pragma unroll
+        for (int kk = 0; kk < KS; kk += 2) {
+          uint32_t b[4];
+          ldsm_x4(kt + T::off(row, (2 * kk + (lane >> 3)) * 16), b);
+          mma_16816<BF>(sacc[j][nt], qa[kk], b[0], b[1]);
+          mma_16816<BF>(s2[nt], qa[kk + 1], b[2], b[3]);
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sacc[j][nt][i] += s2[nt][i];
     }
+    if (failed) break;
     // ---- causal mask (tokens after a row's position), scale, online softmax
-    const int tok_base = t * TR;
-    const bool masked = tok_base + TR - 1 > p_min;
     float mx_lo = -CUDART_INF_F, mx_hi = -CUDART_INF_F;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int j = 0; j < kPrefillTps; ++j) {
+      const int tok_base = (t0 + j) * TR;
+      const bool masked = tok_base + TR - 1 > p_min;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int tok = tok_base + nt * 8 + 2 * c + (i & 1);
-        const int p = i < 2 ? p_lo : p_hi;
-        const float x = (!masked || tok <= p) ? sacc[nt][i] * qscale : -CUDART_INF_F;
-        sacc[nt][i] = x;
-        if (i < 2) mx_lo = fmaxf(mx_lo, x);
-        else mx_hi = fmaxf(mx_hi, x);
-      }
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tok = tok_base + nt * 8 + 2 * c + (i & 1);
+          const int p = i < 2 ? p_lo : p_hi;
+          const float x = (!masked || tok <= p) ? sacc[j][nt][i] * qscale : -CUDART_INF_F;
+          sacc[j][nt][i] = x;
+          if (i < 2) mx_lo = fmaxf(mx_lo, x);
+          else mx_hi = fmaxf(mx_hi, x);
+        }
+    }
     mx_lo = fmaxf(mx_lo, __shfl_xor_sync(FULL, mx_lo, 1));
     mx_lo = fmaxf(mx_lo, __shfl_xor_sync(FULL, mx_lo, 2));
     mx_hi = fmaxf(mx_hi, __shfl_xor_sync(FULL, mx_hi, 1));
@@ -221,14 +268,16 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
     m_hi = mn_hi;
     float ps_lo = 0.f, ps_hi = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      sacc[nt][0] = exp2f(sacc[nt][0] - mu_lo);
-      sacc[nt][1] = exp2f(sacc[nt][1] - mu_lo);
-      sacc[nt][2] = exp2f(sacc[nt][2] - mu_hi);
-      sacc[nt][3] = exp2f(sacc[nt][3] - mu_hi);
-      ps_lo += sacc[nt][0] + sacc[nt][1];
-      ps_hi += sacc[nt][2] + sacc[nt][3];
-    }
+    for (int j = 0; j < kPrefillTps; ++j)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        sacc[j][nt][0] = exp2f(sacc[j][nt][0] - mu_lo);
+        sacc[j][nt][1] = exp2f(sacc[j][nt][1] - mu_lo);
+        sacc[j][nt][2] = exp2f(sacc[j][nt][2] - mu_hi);
+        sacc[j][nt][3] = exp2f(sacc[j][nt][3] - mu_hi);
+        ps_lo += sacc[j][nt][0] + sacc[j][nt][1];
+        ps_hi += sacc[j][nt][2] + sacc[j][nt][3];
+      }
     l_lo = l_lo * al_lo + ps_lo;
     l_hi = l_hi * al_hi + ps_hi;
 #pragma unroll
@@ -238,50 +287,57 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
       o[j][2] *= al_hi;
       o[j][3] *= al_hi;
     }
-    // Rows of the tile past the context may hold anything (even NaN) and
-    // 0 * NaN is NaN inside the MMA: each warp clears them in its view of the
-    // stage before reading V (every warp writes the same zeros; the stage is
-    // not refilled after the last tile).
-    if (tok_base + TR > ctx) {
-      constexpr int CPR = T::RB / 16;
-      const int first = max(0, ctx - tok_base);
-      for (int i = lane; i < (TR - first) * CPR; i += 32)
-        *reinterpret_cast<uint4*>(vt + T::off(first + i / CPR, (i % CPR) * 16)) =
-            make_uint4(0u, 0u, 0u, 0u);
-      __syncwarp();
-    }
-    // ---- O += P V (P from the S accumulators, as the A operand). bf16 keeps
-    // only 8 significant bits, too few for rows that see a handful of tokens;
-    // there P = P_hi + P_lo, both bf16, in two MMAs (about 16 bits).
-    uint32_t pa[4], pl[4];
-    pa[0] = pack2<BF>(sacc[0][0], sacc[0][1]);
-    pa[1] = pack2<BF>(sacc[0][2], sacc[0][3]);
-    pa[2] = pack2<BF>(sacc[1][0], sacc[1][1]);
-    pa[3] = pack2<BF>(sacc[1][2], sacc[1][3]);
-    if constexpr (BF) {
+    // ---- O += P V per tile (P from the S accumulators, as the A operand)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float* src = sacc[k >> 1] + 2 * (k & 1);
-        pl[k] = pack2<true>(src[0] - __uint_as_float(pa[k] << 16),
-                            src[1] - __uint_as_float(pa[k] & 0xffff0000u));
+    for (int j = 0; j < kPrefillTps; ++j) {
+      const int tt = t0 + j;
+      if (tt >= ntiles) break;
+      uint8_t* vt = smem + (tt % R) * STAGE + T::BYTES;
+      const int tok_base = tt * TR;
+      // Rows of the tile past the context may hold anything (even NaN) and
+      // 0 * NaN is NaN inside the MMA: each warp clears them in its view of
+      // the stage before reading V (every warp writes the same zeros; only
+      // the last tile can reach past the context and its stage is not refilled).
+      if (tok_base + TR > ctx) {
+        constexpr int CPR = T::RB / 16;
+        const int first = max(0, ctx - tok_base);
+        for (int i = lane; i < (TR - first) * CPR; i += 32)
+          *reinterpret_cast<uint4*>(vt + T::off(first + i / CPR, (i % CPR) * 16)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
       }
-    }
-    const int vrow = (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-    for (int dn = 0; dn < NO; dn += 2) {
-      uint32_t b[4];
-      ldsm_x4_trans(vt + T::off(vrow, (dn + (lane >> 4)) * 16), b);
-      mma_16816<BF>(o[dn], pa, b[0], b[1]);
-      mma_16816<BF>(o[dn + 1], pa, b[2], b[3]);
+      // bf16 keeps only 8 significant bits, too few for rows that see a
+      // handful of tokens; there P = P_hi + P_lo, both bf16, in two MMAs.
+      uint32_t pa[4], pl[4];
+      pa[0] = pack2<BF>(sacc[j][0][0], sacc[j][0][1]);
+      pa[1] = pack2<BF>(sacc[j][0][2], sacc[j][0][3]);
+      pa[2] = pack2<BF>(sacc[j][1][0], sacc[j][1][1]);
+      pa[3] = pack2<BF>(sacc[j][1][2], sacc[j][1][3]);
       if constexpr (BF) {
-        mma_16816<BF>(o[dn], pl, b[0], b[1]);
-        mma_16816<BF>(o[dn + 1], pl, b[2], b[3]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float* src = sacc[j][q >> 1] + 2 * (q & 1);
+          pl[q] = pack2<true>(src[0] - __uint_as_float(pa[q] << 16),
+                              src[1] - __uint_as_float(pa[q] & 0xffff0000u));
+        }
       }
+      const int vrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int dn = 0; dn < NO; dn += 2) {
+        uint32_t b[4];
+        ldsm_x4_trans(vt + T::off(vrow, (dn + (lane >> 4)) * 16), b);
+        mma_16816<BF>(o[dn], pa, b[0], b[1]);
+        mma_16816<BF>(o[dn + 1], pa, b[2], b[3]);
+        if constexpr (BF) {
+          mma_16816<BF>(o[dn], pl, b[0], b[1]);
+          mma_16816<BF>(o[dn + 1], pl, b[2], b[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[tt % R]);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
   }
-  if (t < ntiles) {
+  if (failed) {
     // A wait gave up (never expected): record it and let the loads this CTA
     // issued land (bounded) before its shared memory goes away.
     if (lane == 0) {
@@ -290,8 +346,11 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
                      0);
       report(a.err, kErrWaitTimeout);
     }
-    if (producer)
-      for (int k = t; k < issued; ++k) mbar_wait(&full[k % R], (k / R) & 1);
+    if (producer) {
+      // issued so far: steps 0 .. min(k + RS - 1, nsteps - 1) at most
+      const int last = min(ntiles, (min(k + kPrefillRs - 1, nsteps - 1) + 1) * kPrefillTps);
+      for (int tt = t; tt < last; ++tt) mbar_wait(&full[tt % R], (tt / R) & 1);
+    }
     return;
   }
 
