@@ -62,7 +62,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // segments): one box = 16 rows of one kv-head, whole rows, swizzled per segment,
 // stored in shared memory segment-major (all rows' first segment, then the next).
 pa_status encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_blocks,
-                           int32_t block_size, int32_t hkv, int32_t head_dim, int elem) {
+                           int32_t block_size, int32_t hkv, int32_t head_dim, int elem,
+                           bool one_segment = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const int row_bytes = head_dim * elem;
@@ -75,7 +76,7 @@ pa_status encode_cache_map(CUtensorMap* map, const void* cache, int64_t num_bloc
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(row_bytes) * hkv,
                            static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(seg)};
   cuuint32_t box[4] = {static_cast<cuuint32_t>(seg / elem), 16u, 1u,
-                       static_cast<cuuint32_t>(row_bytes / seg)};
+                       one_segment ? 1u : static_cast<cuuint32_t>(row_bytes / seg)};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   const CUtensorMapSwizzle swz = seg == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                : seg == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -453,10 +454,15 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
     return fail(PA_ERR_INVALID_ARG, "chunked_prefill: misaligned pointer");
 
   CUtensorMap kmap, vmap;
+  // Chunks that fill the 128 rows of a tensor-memory CTA (query tokens x heads
+  // of a kv-head's group) run on tcgen05; shorter ones (a few draft tokens)
+  // on the 64-row mma.sync kernel, which wastes fewer rows.
+  const bool tc = static_cast<int64_t>(max_query_len) * group >= 128;
   pa_status st = encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads,
-                                  head_dim, 2);
+                                  head_dim, 2, tc);
   if (st == PA_OK)
-    st = encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, 2);
+    st = encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, 2,
+                          tc);
   if (st != PA_OK) return st;
   PrefillArgs a{};
   a.out = out;
@@ -475,8 +481,9 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
   a.num_kv_heads = num_kv_heads;
   a.block_size = block_size;
   a.scale_log2 = scale * 1.4426950408889634f;
-  return cuda_status(launch_prefill(a, kmap, vmap, dtype == PA_F16 ? kF16 : kBF16, head_dim, group,
-                                    max_query_len, reinterpret_cast<cudaStream_t>(stream)),
+  auto launch = tc ? launch_prefill_tc : launch_prefill;
+  return cuda_status(launch(a, kmap, vmap, dtype == PA_F16 ? kF16 : kBF16, head_dim, group,
+                            max_query_len, reinterpret_cast<cudaStream_t>(stream)),
                      "chunked_prefill");
 }
 

@@ -35,4 +35,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& kmap, const 
                            int q_dtype, int head_dim, int group, int32_t max_query_len,
                            cudaStream_t stream);
 
+// The same on the 5th-generation tensor cores (tcgen05, tensor memory); the
+// tensor maps are the one-segment boxes of encode_cache_map(..., 1 segment).
+cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& kmap,
+                              const CUtensorMap& vmap, int q_dtype, int head_dim, int group,
+                              int32_t max_query_len, cudaStream_t stream);
+
 }  // namespace paged

@@ -1,0 +1,450 @@
+// prefill_tc.cu — the multi-token query on the 5th-generation tensor cores.
+//
+// Same operation as prefill_kernel.cu ("vLLM推理引擎架构：PagedAttention机制
+// 与高吞吐推理" §2.3 with a query of several trailing tokens per sequence and
+// the causal rule): rows cu[s] .. cu[s+1]-1 of the query are the last
+// positions p_i of sequence s and see its tokens t <= p_i.
+//
+// One CTA = 128 threads = 128 rows (row = one (query token, head of the
+// kv-head's group)), one row per thread and per tensor-memory lane:
+//  * Q (128 x D) is written once into shared memory, 128-byte swizzled, K-major;
+//  * K and V of 64 tokens per step arrive by TMA into a 2-stage ring (16-row
+//    boxes of one 128-byte segment each, so a stage is [segment][64 rows][128 B]);
+//  * thread 0 issues S = Q K^T (tcgen05.mma kind::f16, M=128, N=64, fp32 in
+//    tensor memory) and commits it to an mbarrier;
+//  * every thread loads its row of S from tensor memory, masks tokens after its
+//    position, and runs the base-2 online softmax with a lazily updated
+//    maximum (the running maximum moves only when a row's maximum grows by more
+//    than 8, i.e. probabilities stay below 2^8, so O rarely needs rescaling);
+//  * P (f16/bf16, bf16 as hi + lo parts) goes to shared memory and thread 0
+//    issues O += P V (M=128, N=D, K=64; V read MN-major), accumulating in
+//    tensor memory, then refills the stage once those MMAs completed;
+//  * the epilogue divides each row of O by its sum and stores it.
+// Every wait is bounded by wall time; a wait that gives up is agreed on by the
+// whole CTA at the next barrier, which then drains its loads and MMAs, frees
+// its tensor memory and reports.
+#include <math_constants.h>
+
+#include <type_traits>
+
+#include "consumer_mma.cuh"
+#include "decode_args.h"
+#include "decode_kernel.cuh"
+#include "device_common.cuh"
+#include "prefill_args.h"
+#include "tc_common.cuh"
+
+namespace paged {
+namespace {
+
+constexpr int kTcRows = 128;       // M: rows per CTA
+constexpr int kTcNT = 64;          // tokens per step
+constexpr int kTcStages = 2;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemO = 128;   // column of O (S at column 0)
+constexpr int kSiteTc = 6;
+
+template <class QF, int D, int G>
+struct TcCfg {
+  static constexpr bool BF = std::is_same<QF, BF16>::value;
+  static constexpr int NSEG = D * 2 / 128;          // 128-byte segments of a row
+  static constexpr int QT = kTcRows / G;            // query tokens per CTA
+  static constexpr int Q_BYTES = NSEG * kTcRows * 128;
+  static constexpr int KV_SEG = kTcNT * 128;        // one segment of K or V in a stage
+  static constexpr int KV_BYTES = NSEG * KV_SEG;    // one stage of K (or V)
+  static constexpr int P_BYTES = kTcRows * kTcNT * 2;
+  static constexpr int OFF_K = Q_BYTES;                         // K ring
+  static constexpr int OFF_V = OFF_K + kTcStages * KV_BYTES;    // V ring
+  static constexpr int P_SET = (BF ? 2 : 1) * P_BYTES;          // P (and for bf16 its residual)
+  static constexpr int OFF_P = OFF_V + kTcStages * KV_BYTES;    // two P sets (steps k, k+1)
+  static constexpr int BYTES = OFF_P + 2 * P_SET;
+  static constexpr uint32_t IDESC_S = tc::idesc_f16<BF, kTcRows, kTcNT, false>();
+  static constexpr uint32_t IDESC_PV = tc::idesc_f16<BF, kTcRows, D, true>();
+  static_assert(kTcNT * 2 == 128, "a row of P is one 128-byte swizzle row");
+};
+
+// 16-byte chunk `c` of row `r` of a 128-byte-swizzled [rows][128 B] tile.
+__device__ __forceinline__ uint32_t sw128(int r, int c) {
+  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t pack_pair(bool bf, float lo, float hi) {
+  return bf ? pack2<true>(lo, hi) : pack2<false>(lo, hi);
+}
+
+
+template <class QF, int D, int G>
+__global__ void __launch_bounds__(kTcRows + 64, 1)
+    paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap kmap,
+                            const __grid_constant__ CUtensorMap vmap) {
+  using C = TcCfg<QF, D, G>;
+  constexpr bool BF = C::BF;
+  constexpr int NSEG = C::NSEG, QT = C::QT, R = kTcStages, NT = kTcNT, TR = kTileRows;
+  constexpr int kMma = kTcRows / 32;        // warp issuing the MMAs (owns the tensor memory)
+  constexpr int kLoader = kMma + 1;         // warp issuing the TMA loads
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sq = smem;
+  auto sp = [&](int k) { return smem + C::OFF_P + (k & 1) * C::P_SET; };
+  auto sk = [&](int k) { return smem + C::OFF_K + (k % R) * C::KV_BYTES; };
+  auto sv = [&](int k) { return smem + C::OFF_V + (k % R) * C::KV_BYTES; };
+  // K / V rings: *full when a stage's boxes landed, *empty when the MMAs that
+  // read it completed. s_bar[b]: S buffer b computed. p_bar[b]: the softmax
+  // warps wrote P set b (and rescaled O). pv_bar[b]: O += P V of P set b done.
+  __shared__ uint64_t kfull[R], kempty[R], vfull[R], vempty[R], s_bar[2], p_bar[2], pv_bar[2],
+      drain_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int aborted;
+
+  const int z = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int r = 0; r < R; ++r) {
+      mbar_init(&kfull[r], 1);
+      mbar_init(&kempty[r], 1);
+      mbar_init(&vfull[r], 1);
+      mbar_init(&vempty[r], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_bar[b], 1);
+      mbar_init(&p_bar[b], kTcRows / 32);
+    }
+    mbar_init(&pv_bar[0], 1);
+    mbar_init(&pv_bar[1], 1);
+    mbar_init(&drain_bar, 1);
+    fence_mbar_init();
+    aborted = 0;
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  const int q0 = a.cu_query_lens[s];
+  const int qlen = a.cu_query_lens[s + 1] - q0;
+  int ctx = a.context_lens[s];
+  if (ctx > a.ctx_limit || ctx < 0) {
+    if (tid == 0 && z == 0 && kvh == 0) report(a.err, kErrContextClipped);
+    ctx = ctx < 0 ? 0 : a.ctx_limit;
+  }
+  const int tok0 = z * QT;
+  if (tok0 >= qlen) return;  // ragged chunk lengths: nothing for this CTA
+  const int ntok = min(QT, qlen - tok0);
+  const int tok = tid / G;   // (softmax threads: row tid)
+  const bool valid = warp < kMma && tok < ntok;
+  const int64_t row_off =
+      (static_cast<int64_t>(q0 + tok0 + tok) * a.num_heads + kvh * G + tid % G) * D;
+  if (qlen > ctx) {  // a query longer than its context: rows become zeros
+    if (tid == 0 && z == 0 && kvh == 0) report(a.err, kErrQueryLonger);
+    if (valid) {
+      uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
+      for (int c = 0; c < D / 8; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    return;
+  }
+  const int pos0 = ctx - qlen + tok0;
+  const int p_max = pos0 + ntok - 1;
+  const int ntiles = p_max / TR + 1;              // 16-token tiles holding tokens 0..p_max
+  const int nsteps = p_max / NT + 1;
+
+  __syncthreads();  // barrier initialisation visible to every thread
+  if (warp == kMma) tc::alloc(&tmem_slot, kTmemCols);
+  if (warp < kMma) {
+    // Q rows -> shared memory (128-byte swizzle, K-major), zeros past the chunk
+    const uint4* q4 = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.query) +
+                                                     row_off * 2);
+#pragma unroll
+    for (int sg = 0; sg < NSEG; ++sg)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = valid ? q4[sg * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sq + sg * (kTcRows * 128) + sw128(tid, c)) = v;
+      }
+    fence_proxy_async_smem();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t t_o = tmem + kTmemO;
+
+  if (warp == kLoader) {
+    // ================= TMA loads (one thread) =================
+    if (lane == 0) {
+      const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
+      const uint64_t policy = l2_policy_evict_last();  // other query tiles read them too
+      auto issue_kv = [&](int k, const int32_t (&bid)[NT / TR], bool is_v) {
+        uint8_t* dst = is_v ? sv(k) : sk(k);
+        uint64_t* bar = is_v ? &vfull[k % R] : &kfull[k % R];
+        const CUtensorMap* map = is_v ? &vmap : &kmap;
+        const int t_begin = k * (NT / TR), t_end = min(ntiles, (k + 1) * (NT / TR));
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(NSEG * (t_end - t_begin) * TR * 128));
+#pragma unroll
+        for (int j = 0; j < NT / TR; ++j) {
+          const int t = t_begin + j;
+          if (t >= t_end) break;
+          int32_t b = bid[j];
+          if (b < 0 || b >= a.num_blocks) {
+            if (!is_v) report(a.err, kErrBadBlockId);
+            b = -1;  // read as a box outside the pool: zero-filled
+          }
+          const int32_t row0 = b >= 0 ? b * a.block_size + (t * TR) % a.block_size : -TR;
+#pragma unroll
+          for (int sg = 0; sg < NSEG; ++sg)
+            tma_load_4d(dst + sg * C::KV_SEG + j * TR * 128, map, bar, 0, row0, kvh, sg, policy);
+        }
+      };
+      // block ids of the next step are fetched while the current one is issued
+      int32_t bid[NT / TR], nbid[NT / TR];
+      auto load_ids = [&](int k, int32_t (&dst)[NT / TR]) {
+#pragma unroll
+        for (int j = 0; j < NT / TR; ++j) {
+          const int t = k * (NT / TR) + j;
+          dst[j] = t < ntiles ? table[(t * TR) / a.block_size] : 0;
+        }
+      };
+      load_ids(0, bid);
+      bool ok = true;
+      int k = 0;
+      for (; ok && k < nsteps; ++k) {
+        if (k + 1 < nsteps) load_ids(k + 1, nbid);
+        if (k >= R) {  // the stage's previous step: S done (K), O += P V done (V)
+          ok = mbar_wait(&kempty[k % R], ((k - R) / R) & 1, &aborted);
+          if (ok) issue_kv(k, bid, false);
+          ok = ok && mbar_wait(&vempty[k % R], ((k - R) / R) & 1, &aborted);
+          if (ok) issue_kv(k, bid, true);
+        } else {
+          issue_kv(k, bid, false);
+          issue_kv(k, bid, true);
+        }
+#pragma unroll
+        for (int j = 0; j < NT / TR; ++j) bid[j] = nbid[j];
+      }
+      if (!ok) {
+        aborted = 1;
+        report(a.err, kErrWaitTimeout);
+      }
+      // before the CTA's shared memory goes away every issued load must have
+      // landed (the last use of each stage; earlier ones completed already)
+      for (int j = max(0, k - R); j < k; ++j) {
+        mbar_wait(&kfull[j % R], (j / R) & 1);
+        mbar_wait(&vfull[j % R], (j / R) & 1);
+      }
+    }
+  } else if (warp == kMma) {
+    // ================= MMA issue (one thread) =================
+    if (lane == 0) {
+      int k_waited = 0, v_waited = 0;
+      auto issue_s = [&](int k) {
+        if (!mbar_wait(&kfull[k % R], (k / R) & 1, &aborted)) return false;
+        k_waited = k + 1;
+        tc::fence_after_sync();
+        uint8_t* ks = sk(k);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int sg = kk / 4, off = (kk % 4) * 32;
+          tc::mma_f16(tmem + (k & 1) * NT,
+                      tc::sw128_desc(sq + sg * (kTcRows * 128) + off, 16, 1024),
+                      tc::sw128_desc(ks + sg * C::KV_SEG + off, 16, 1024), C::IDESC_S, kk > 0);
+        }
+        tc::commit(&s_bar[k & 1]);
+        tc::commit(&kempty[k % R]);
+        return true;
+      };
+      bool ok = issue_s(0);
+      for (int k = 0; ok && k < nsteps; ++k) {
+        // S of the next step, into the S buffer the softmax of step k-1 released
+        if (k + 1 < nsteps)
+          ok = (k < 1 || mbar_wait(&p_bar[(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted)) &&
+               issue_s(k + 1);
+        // O += P V once the softmax warps wrote P of step k
+        if (ok) ok = mbar_wait(&p_bar[k & 1], (k >> 1) & 1, &aborted);
+        if (ok) ok = mbar_wait(&vfull[k % R], (k / R) & 1, &aborted);
+        if (ok) {
+          v_waited = k + 1;
+          tc::fence_after_sync();
+          uint8_t* vs = sv(k);
+          uint8_t* ps = sp(k);
+#pragma unroll
+          for (int kk = 0; kk < NT / 16; ++kk) {
+            const uint64_t bv = tc::sw128_desc(vs + kk * 16 * 128, NT * 128, 1024);
+            tc::mma_f16(t_o, tc::sw128_desc(ps + kk * 32, 16, 1024), bv, C::IDESC_PV,
+                        k > 0 || kk > 0);
+            if constexpr (BF)
+              tc::mma_f16(t_o, tc::sw128_desc(ps + C::P_BYTES + kk * 32, 16, 1024), bv,
+                          C::IDESC_PV, true);
+          }
+          tc::commit(&pv_bar[k & 1]);
+          tc::commit(&vempty[k % R]);
+        }
+      }
+      if (!ok) {
+        // A wait gave up (never expected): let this CTA's MMAs finish (bounded)
+        // before its tensor and shared memory go away.
+        aborted = 1;
+        record_failure(a.diag, kSiteTc, blockIdx.x, blockIdx.y, blockIdx.z, k_waited, v_waited,
+                       nsteps, 0);
+        report(a.err, kErrWaitTimeout);
+        tc::commit(&drain_bar);
+        mbar_wait(&drain_bar, 0);
+      }
+    }
+  } else {
+    // ================= softmax warps: one row per thread =================
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int p_row = valid ? pos0 + tok : -1;
+    const int kv_valid = min(ctx, ntiles * TR);   // tokens with loaded, real rows
+    const float qscale = a.scale_log2;
+    float m_used = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    for (int k = 0; ok && k < nsteps; ++k) {
+      ok = mbar_wait(&s_bar[k & 1], (k >> 1) & 1, &aborted);
+      if (!ok) break;
+      tc::fence_after_sync();
+      float x[NT];
+      const uint32_t t_s = tmem + (k & 1) * NT + lane_base;
+      tc::ld32(t_s, *reinterpret_cast<float(*)[32]>(x));
+      tc::ld32(t_s + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+      const int tk0 = k * NT;
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int i = 0; i < NT; ++i) {
+        x[i] = tk0 + i <= p_row ? x[i] * qscale : -CUDART_INF_F;
+        mx = fmaxf(mx, x[i]);
+      }
+      const bool rescale = mx > m_used + 8.f;   // false while the row sees nothing
+      const float alpha = rescale ? exp2f(m_used - mx) : 1.f;
+      if (rescale) m_used = mx;
+      const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
+      float ps = 0.f;
+#pragma unroll
+      for (int i = 0; i < NT; ++i) {
+        x[i] = exp2f(x[i] - mu);
+        ps += x[i];
+      }
+      l = l * alpha + ps;
+      // P set k&1 is free once O += P V of step k-2 completed; O may be
+      // rescaled only once O += P V of step k-1 completed (rare: the maximum
+      // moves lazily), otherwise that MMA keeps running under this softmax
+      if (k >= 2) {
+        ok = mbar_wait(&pv_bar[k & 1], ((k - 2) >> 1) & 1, &aborted);
+        if (!ok) break;
+      }
+      if (k >= 1 && rescale) {
+        ok = mbar_wait(&pv_bar[(k - 1) & 1], ((k - 1) >> 1) & 1, &aborted);
+        if (!ok) break;
+        tc::fence_after_sync();
+        {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tc::ld32(t_o + lane_base + c * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tc::st32(t_o + lane_base + c * 32, o);
+          }
+        }
+      }
+      // P row (and for bf16 the residual P - bf16(P)) -> shared memory
+#pragma unroll
+      for (int c = 0; c < NT / 8; ++c) {
+        uint32_t w[4], wl[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float p0 = x[c * 8 + 2 * i], p1 = x[c * 8 + 2 * i + 1];
+          w[i] = pack_pair(BF, p0, p1);
+          if constexpr (BF)
+            wl[i] = pack2<true>(p0 - __uint_as_float(w[i] << 16),
+                                p1 - __uint_as_float(w[i] & 0xffff0000u));
+        }
+        uint8_t* ps = sp(k);
+        *reinterpret_cast<uint4*>(ps + sw128(tid, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+        if constexpr (BF)
+          *reinterpret_cast<uint4*>(ps + C::P_BYTES + sw128(tid, c)) =
+              make_uint4(wl[0], wl[1], wl[2], wl[3]);
+      }
+      // V rows without real data in this step (past the context, or tiles not
+      // loaded) may hold anything, even NaN, and 0 * NaN is NaN inside the MMA
+      const int vrows = max(0, min(NT, kv_valid - tk0));
+      if (vrows < NT) {
+        uint8_t* vs = sv(k);
+        ok = mbar_wait(&vfull[k % R], (k / R) & 1, &aborted);  // the TMA writes come first
+        if (!ok) break;
+        for (int i = tid; i < (NT - vrows) * NSEG * 8; i += kTcRows) {
+          const int r = vrows + i / (NSEG * 8), sg = (i / 8) % NSEG, c = i % 8;
+          *reinterpret_cast<uint4*>(vs + sg * C::KV_SEG + r * 128 + c * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_bar[k & 1]);
+    }
+    if (ok) ok = mbar_wait(&pv_bar[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, &aborted);
+    if (!ok) {
+      aborted = 1;
+    } else {
+      // ---- epilogue: out = O / l, rounded to the q dtype
+      tc::fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tc::ld32(t_o + lane_base + c * 32, o);
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            o4[c * 4 + q] = make_uint4(pack_pair(BF, o[8 * q] * inv, o[8 * q + 1] * inv),
+                                       pack_pair(BF, o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                       pack_pair(BF, o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                       pack_pair(BF, o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kMma) {
+    tc::fence_after_sync();
+    tc::dealloc(tmem, kTmemCols);
+  }
+}
+
+template <class QF, int D, int G>
+cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                      int32_t max_query_len, cudaStream_t stream) {
+  using C = TcCfg<QF, D, G>;
+  // at least 80 KB so that at most two CTAs (2 x 256 tensor-memory columns) share an SM
+  const size_t smem = std::max<size_t>(1024 + C::BYTES, 80 * 1024);
+  auto kern = paged_prefill_tc_kernel<QF, D, G>;
+  cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  const unsigned tiles = static_cast<unsigned>((max_query_len + C::QT - 1) / C::QT);
+  return launch_pdl(kern, dim3(tiles, a.num_kv_heads, a.num_seqs), kTcRows + 64, smem, stream,
+                    a, kmap, vmap);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& kmap,
+                              const CUtensorMap& vmap, int q_dtype, int head_dim, int group,
+                              int32_t max_query_len, cudaStream_t stream) {
+#define PAGED_TC(QF, d, g) \
+  if (head_dim == d && group == g) return launch_tc<QF, d, g>(a, kmap, vmap, max_query_len, stream);
+#define PAGED_TC_ALL(QF)                                                  \
+  PAGED_TC(QF, 64, 1) PAGED_TC(QF, 64, 2) PAGED_TC(QF, 64, 4) PAGED_TC(QF, 64, 8) \
+  PAGED_TC(QF, 128, 1) PAGED_TC(QF, 128, 2) PAGED_TC(QF, 128, 4) PAGED_TC(QF, 128, 8)
+  if (q_dtype == kF16) {
+    PAGED_TC_ALL(F16)
+  } else if (q_dtype == kBF16) {
+    PAGED_TC_ALL(BF16)
+  }
+#undef PAGED_TC_ALL
+#undef PAGED_TC
+  return cudaErrorNotSupported;
+}
+
+}  // namespace paged

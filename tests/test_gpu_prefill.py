@@ -59,17 +59,26 @@ def custom(ctxs, qlens, H, Hkv, D, bs, dt, seed):
     return sp, st, hd, q, np.array(qlens, np.int32)
 
 
-# chunk lengths cross CTA tiles (64 / G tokens) and K tiles (16 tokens), with a
-# full prefill (q_len == ctx), single tokens, and a context of one token
-EDGE = ([1, 17, 40, 100, 33, 130], [1, 17, 9, 70, 1, 65])
+# Chunk lengths that cross CTA row tiles and 16-token K tiles, with a full
+# prefill (q_len == ctx), single tokens and a one-token context. The launch
+# picks the kernel by max_query_len x group: >= 128 rows fill a tensor-memory
+# (tcgen05) CTA, fewer run on the 64-row mma.sync kernel; each set below
+# reaches one of them for every group size.
+EDGE = {
+    "tcgen05": ([1, 17, 40, 200, 33, 150, 130], [1, 17, 9, 150, 1, 129, 65]),
+    "mma_sync": ([1, 17, 40, 100, 9], [1, 15, 9, 8, 9]),
+}
 
 
+@pytest.mark.parametrize("kernel", ["tcgen05", "mma_sync"])
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("bs", [16, 32])
-def test_multi_token_edge_sweep(dt, G, D, bs):
-    sp, st, hd, q, qlens = custom(*EDGE, 2 * G, 2, D, bs, dt, seed=G * 100 + D + bs)
+def test_multi_token_edge_sweep(kernel, dt, G, D, bs):
+    ctxs, qlens = EDGE[kernel]
+    assert (max(qlens) * G >= 128) == (kernel == "tcgen05")
+    sp, st, hd, q, qlens = custom(ctxs, qlens, 2 * G, 2, D, bs, dt, seed=G * 100 + D + bs)
     out, ws, cu = run_gpu(sp, st, hd, q, qlens)
     pk.decode_check(ws)
     assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), dt,
