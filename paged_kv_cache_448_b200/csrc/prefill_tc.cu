@@ -37,30 +37,37 @@
 namespace paged {
 namespace {
 
-constexpr int kTcRows = 128;       // M: rows per CTA
+constexpr int kTcRows = 128;       // M: rows of one row group (one MMA)
 constexpr int kTcNT = 64;          // tokens per step
 constexpr int kTcStages = 2;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemO = 128;   // column of O (S at column 0)
+constexpr uint32_t kTmemGroup = 256;  // tensor-memory columns per row group: S x 2, then O
+constexpr uint32_t kTmemO = 128;      // column of O within the group (S buffers at 0 and 64)
 constexpr int kSiteTc = 6;
 
-template <class QF, int D, int G>
+// NG row groups of 128 rows share each K/V step (NG = 2: 256 rows, eight
+// softmax warps, and two independent MMA streams per step).
+template <class QF, int D, int G, int NG>
 struct TcCfg {
   static constexpr bool BF = std::is_same<QF, BF16>::value;
   static constexpr int NSEG = D * 2 / 128;          // 128-byte segments of a row
-  static constexpr int QT = kTcRows / G;            // query tokens per CTA
-  static constexpr int Q_BYTES = NSEG * kTcRows * 128;
+  static constexpr int ROWS = NG * kTcRows;
+  static constexpr int QT = ROWS / G;               // query tokens per CTA
+  static constexpr int QG_BYTES = NSEG * kTcRows * 128;  // Q of one group
   static constexpr int KV_SEG = kTcNT * 128;        // one segment of K or V in a stage
   static constexpr int KV_BYTES = NSEG * KV_SEG;    // one stage of K (or V)
   static constexpr int P_BYTES = kTcRows * kTcNT * 2;
-  static constexpr int OFF_K = Q_BYTES;                         // K ring
+  static constexpr int P_SET = (BF ? 2 : 1) * P_BYTES;  // P (and for bf16 its residual)
+  // P sets per group: two (steps k and k+1) where shared memory allows
+  static constexpr int PB = (BF && NG == 2) ? 1 : 2;
+  static constexpr int OFF_K = NG * QG_BYTES;                   // K ring
   static constexpr int OFF_V = OFF_K + kTcStages * KV_BYTES;    // V ring
-  static constexpr int P_SET = (BF ? 2 : 1) * P_BYTES;          // P (and for bf16 its residual)
-  static constexpr int OFF_P = OFF_V + kTcStages * KV_BYTES;    // two P sets (steps k, k+1)
-  static constexpr int BYTES = OFF_P + 2 * P_SET;
+  static constexpr int OFF_P = OFF_V + kTcStages * KV_BYTES;    // [group][PB] P sets
+  static constexpr int BYTES = OFF_P + NG * PB * P_SET;
+  static constexpr uint32_t TMEM_COLS = NG * kTmemGroup;
   static constexpr uint32_t IDESC_S = tc::idesc_f16<BF, kTcRows, kTcNT, false>();
   static constexpr uint32_t IDESC_PV = tc::idesc_f16<BF, kTcRows, D, true>();
   static_assert(kTcNT * 2 == 128, "a row of P is one 128-byte swizzle row");
+  static_assert(BYTES + 1024 <= 227 * 1024, "shared memory of one CTA");
 };
 
 // 16-byte chunk `c` of row `r` of a 128-byte-swizzled [rows][128 B] tile.
@@ -73,28 +80,30 @@ __device__ __forceinline__ uint32_t pack_pair(bool bf, float lo, float hi) {
 }
 
 
-template <class QF, int D, int G>
-__global__ void __launch_bounds__(kTcRows + 64, 1)
+template <class QF, int D, int G, int NG>
+__global__ void __launch_bounds__(NG * kTcRows + 64, 1)
     paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap kmap,
                             const __grid_constant__ CUtensorMap vmap) {
-  using C = TcCfg<QF, D, G>;
+  using C = TcCfg<QF, D, G, NG>;
   constexpr bool BF = C::BF;
   constexpr int NSEG = C::NSEG, QT = C::QT, R = kTcStages, NT = kTcNT, TR = kTileRows;
-  constexpr int kMma = kTcRows / 32;        // warp issuing the MMAs (owns the tensor memory)
+  constexpr int PB = C::PB;
+  constexpr int kMma = NG * kTcRows / 32;   // warp issuing the MMAs (owns the tensor memory)
   constexpr int kLoader = kMma + 1;         // warp issuing the TMA loads
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sq = smem;
-  auto sp = [&](int k) { return smem + C::OFF_P + (k & 1) * C::P_SET; };
+  auto sq = [&](int g) { return smem + g * C::QG_BYTES; };
   auto sk = [&](int k) { return smem + C::OFF_K + (k % R) * C::KV_BYTES; };
   auto sv = [&](int k) { return smem + C::OFF_V + (k % R) * C::KV_BYTES; };
+  auto sp = [&](int g, int k) { return smem + C::OFF_P + (g * PB + k % PB) * C::P_SET; };
   // K / V rings: *full when a stage's boxes landed, *empty when the MMAs that
-  // read it completed. s_bar[b]: S buffer b computed. p_bar[b]: the softmax
-  // warps wrote P set b (and rescaled O). pv_bar[b]: O += P V of P set b done.
-  __shared__ uint64_t kfull[R], kempty[R], vfull[R], vempty[R], s_bar[2], p_bar[2], pv_bar[2],
-      drain_bar;
+  // read it completed (both groups). Per group g: s_bar[g][b] S buffer b
+  // computed; p_bar[g][b] the group's softmax warps wrote P of a step of parity
+  // b (and rescaled O); pv_bar[g][b] O += P V of such a step done.
+  __shared__ uint64_t kfull[R], kempty[R], vfull[R], vempty[R], s_bar[NG][2], p_bar[NG][2],
+      pv_bar[NG][2], drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int aborted;
 
@@ -107,12 +116,12 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
       mbar_init(&vfull[r], 1);
       mbar_init(&vempty[r], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_bar[b], 1);
-      mbar_init(&p_bar[b], kTcRows / 32);
-    }
-    mbar_init(&pv_bar[0], 1);
-    mbar_init(&pv_bar[1], 1);
+    for (int g = 0; g < NG; ++g)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&s_bar[g][b], 1);
+        mbar_init(&p_bar[g][b], kTcRows / 32);
+        mbar_init(&pv_bar[g][b], 1);
+      }
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
     aborted = 0;
@@ -131,7 +140,8 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
   const int tok0 = z * QT;
   if (tok0 >= qlen) return;  // ragged chunk lengths: nothing for this CTA
   const int ntok = min(QT, qlen - tok0);
-  const int tok = tid / G;   // (softmax threads: row tid)
+  // softmax threads: row tid of the CTA = token tid / G, head tid % G
+  const int tok = tid / G;
   const bool valid = warp < kMma && tok < ntok;
   const int64_t row_off =
       (static_cast<int64_t>(q0 + tok0 + tok) * a.num_heads + kvh * G + tid % G) * D;
@@ -149,9 +159,10 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
   const int nsteps = p_max / NT + 1;
 
   __syncthreads();  // barrier initialisation visible to every thread
-  if (warp == kMma) tc::alloc(&tmem_slot, kTmemCols);
+  if (warp == kMma) tc::alloc(&tmem_slot, C::TMEM_COLS);
   if (warp < kMma) {
-    // Q rows -> shared memory (128-byte swizzle, K-major), zeros past the chunk
+    // Q rows -> shared memory (per group, 128-byte swizzle, K-major), zeros past the chunk
+    const int g = tid / kTcRows, rr = tid % kTcRows;
     const uint4* q4 = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.query) +
                                                      row_off * 2);
 #pragma unroll
@@ -159,7 +170,7 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint4 v = valid ? q4[sg * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(sq + sg * (kTcRows * 128) + sw128(tid, c)) = v;
+        *reinterpret_cast<uint4*>(sq(g) + sg * (kTcRows * 128) + sw128(rr, c)) = v;
       }
     fence_proxy_async_smem();
   }
@@ -167,7 +178,6 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_slot;
-  const uint32_t t_o = tmem + kTmemO;
 
   if (warp == kLoader) {
     // ================= TMA loads (one thread) =================
@@ -236,36 +246,44 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
     // ================= MMA issue (one thread) =================
     if (lane == 0) {
       int k_waited = 0, v_waited = 0;
-      auto issue_s = [&](int k) {
+      auto issue_s = [&](int k) {  // S of step k for every group
         if (!mbar_wait(&kfull[k % R], (k / R) & 1, &aborted)) return false;
         k_waited = k + 1;
         tc::fence_after_sync();
         uint8_t* ks = sk(k);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int sg = kk / 4, off = (kk % 4) * 32;
-          tc::mma_f16(tmem + (k & 1) * NT,
-                      tc::sw128_desc(sq + sg * (kTcRows * 128) + off, 16, 1024),
-                      tc::sw128_desc(ks + sg * C::KV_SEG + off, 16, 1024), C::IDESC_S, kk > 0);
+        for (int g = 0; g < NG; ++g) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int sg = kk / 4, off = (kk % 4) * 32;
+            tc::mma_f16(tmem + g * kTmemGroup + (k & 1) * NT,
+                        tc::sw128_desc(sq(g) + sg * (kTcRows * 128) + off, 16, 1024),
+                        tc::sw128_desc(ks + sg * C::KV_SEG + off, 16, 1024), C::IDESC_S,
+                        kk > 0);
+          }
+          tc::commit(&s_bar[g][k & 1]);
         }
-        tc::commit(&s_bar[k & 1]);
         tc::commit(&kempty[k % R]);
         return true;
       };
       bool ok = issue_s(0);
       for (int k = 0; ok && k < nsteps; ++k) {
-        // S of the next step, into the S buffer the softmax of step k-1 released
-        if (k + 1 < nsteps)
-          ok = (k < 1 || mbar_wait(&p_bar[(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted)) &&
-               issue_s(k + 1);
-        // O += P V once the softmax warps wrote P of step k
-        if (ok) ok = mbar_wait(&p_bar[k & 1], (k >> 1) & 1, &aborted);
+        // S of the next step, into the S buffers the softmax of step k-1 released
+        if (k + 1 < nsteps) {
+          for (int g = 0; ok && g < NG; ++g)
+            ok = k < 1 || mbar_wait(&p_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted);
+          ok = ok && issue_s(k + 1);
+        }
         if (ok) ok = mbar_wait(&vfull[k % R], (k / R) & 1, &aborted);
-        if (ok) {
-          v_waited = k + 1;
+        if (ok) v_waited = k + 1;
+        // O += P V of each group once its softmax warps wrote P of step k
+        for (int g = 0; ok && g < NG; ++g) {
+          ok = mbar_wait(&p_bar[g][k & 1], (k >> 1) & 1, &aborted);
+          if (!ok) break;
           tc::fence_after_sync();
           uint8_t* vs = sv(k);
-          uint8_t* ps = sp(k);
+          uint8_t* ps = sp(g, k);
+          const uint32_t t_o = tmem + g * kTmemGroup + kTmemO;
 #pragma unroll
           for (int kk = 0; kk < NT / 16; ++kk) {
             const uint64_t bv = tc::sw128_desc(vs + kk * 16 * 128, NT * 128, 1024);
@@ -275,16 +293,16 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
               tc::mma_f16(t_o, tc::sw128_desc(ps + C::P_BYTES + kk * 32, 16, 1024), bv,
                           C::IDESC_PV, true);
           }
-          tc::commit(&pv_bar[k & 1]);
-          tc::commit(&vempty[k % R]);
+          tc::commit(&pv_bar[g][k & 1]);
         }
+        if (ok) tc::commit(&vempty[k % R]);
       }
       if (!ok) {
         // A wait gave up (never expected): let this CTA's MMAs finish (bounded)
         // before its tensor and shared memory go away.
         aborted = 1;
         record_failure(a.diag, kSiteTc, blockIdx.x, blockIdx.y, blockIdx.z, k_waited, v_waited,
-                       nsteps, 0);
+                       nsteps, NG);
         report(a.err, kErrWaitTimeout);
         tc::commit(&drain_bar);
         mbar_wait(&drain_bar, 0);
@@ -292,18 +310,22 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
     }
   } else {
     // ================= softmax warps: one row per thread =================
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int g = warp / 4;                      // row group
+    const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
+    const uint32_t t_grp = tmem + g * kTmemGroup;
+    const uint32_t t_o = t_grp + kTmemO + lane_base;
+    const int rr = tid % kTcRows;                // row within the group = tensor-memory lane
     const int p_row = valid ? pos0 + tok : -1;
-    const int kv_valid = min(ctx, ntiles * TR);   // tokens with loaded, real rows
+    const int kv_valid = min(ctx, ntiles * TR);  // tokens with loaded, real rows
     const float qscale = a.scale_log2;
     float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int k = 0; ok && k < nsteps; ++k) {
-      ok = mbar_wait(&s_bar[k & 1], (k >> 1) & 1, &aborted);
+      ok = mbar_wait(&s_bar[g][k & 1], (k >> 1) & 1, &aborted);
       if (!ok) break;
       tc::fence_after_sync();
       float x[NT];
-      const uint32_t t_s = tmem + (k & 1) * NT + lane_base;
+      const uint32_t t_s = t_grp + (k & 1) * NT + lane_base;
       tc::ld32(t_s, *reinterpret_cast<float(*)[32]>(x));
       tc::ld32(t_s + 32, *reinterpret_cast<float(*)[32]>(x + 32));
       const int tk0 = k * NT;
@@ -324,29 +346,28 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
         ps += x[i];
       }
       l = l * alpha + ps;
-      // P set k&1 is free once O += P V of step k-2 completed; O may be
-      // rescaled only once O += P V of step k-1 completed (rare: the maximum
-      // moves lazily), otherwise that MMA keeps running under this softmax
-      if (k >= 2) {
-        ok = mbar_wait(&pv_bar[k & 1], ((k - 2) >> 1) & 1, &aborted);
+      // The P set of step k is free once O += P V of step k-PB completed; O may
+      // be rescaled only once O += P V of step k-1 completed (rare: the
+      // maximum moves lazily), otherwise that MMA keeps running under this softmax
+      if (k >= PB) {
+        ok = mbar_wait(&pv_bar[g][(k - PB) & 1], ((k - PB) >> 1) & 1, &aborted);
         if (!ok) break;
       }
       if (k >= 1 && rescale) {
-        ok = mbar_wait(&pv_bar[(k - 1) & 1], ((k - 1) >> 1) & 1, &aborted);
+        ok = mbar_wait(&pv_bar[g][(k - 1) & 1], ((k - 1) >> 1) & 1, &aborted);
         if (!ok) break;
         tc::fence_after_sync();
-        {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tc::ld32(t_o + lane_base + c * 32, o);
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tc::ld32(t_o + c * 32, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tc::st32(t_o + lane_base + c * 32, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tc::st32(t_o + c * 32, o);
         }
       }
       // P row (and for bf16 the residual P - bf16(P)) -> shared memory
+      uint8_t* psm = sp(g, k);
 #pragma unroll
       for (int c = 0; c < NT / 8; ++c) {
         uint32_t w[4], wl[4];
@@ -358,20 +379,20 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
             wl[i] = pack2<true>(p0 - __uint_as_float(w[i] << 16),
                                 p1 - __uint_as_float(w[i] & 0xffff0000u));
         }
-        uint8_t* ps = sp(k);
-        *reinterpret_cast<uint4*>(ps + sw128(tid, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(psm + sw128(rr, c)) = make_uint4(w[0], w[1], w[2], w[3]);
         if constexpr (BF)
-          *reinterpret_cast<uint4*>(ps + C::P_BYTES + sw128(tid, c)) =
+          *reinterpret_cast<uint4*>(psm + C::P_BYTES + sw128(rr, c)) =
               make_uint4(wl[0], wl[1], wl[2], wl[3]);
       }
       // V rows without real data in this step (past the context, or tiles not
-      // loaded) may hold anything, even NaN, and 0 * NaN is NaN inside the MMA
+      // loaded) may hold anything, even NaN, and 0 * NaN is NaN inside the MMA;
+      // every group's warps clear them (the same zeros) before their P is posted
       const int vrows = max(0, min(NT, kv_valid - tk0));
       if (vrows < NT) {
         uint8_t* vs = sv(k);
         ok = mbar_wait(&vfull[k % R], (k / R) & 1, &aborted);  // the TMA writes come first
         if (!ok) break;
-        for (int i = tid; i < (NT - vrows) * NSEG * 8; i += kTcRows) {
+        for (int i = rr; i < (NT - vrows) * NSEG * 8; i += kTcRows) {
           const int r = vrows + i / (NSEG * 8), sg = (i / 8) % NSEG, c = i % 8;
           *reinterpret_cast<uint4*>(vs + sg * C::KV_SEG + r * 128 + c * 16) =
               make_uint4(0u, 0u, 0u, 0u);
@@ -380,9 +401,10 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
       fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_bar[k & 1]);
+      if (lane == 0) mbar_arrive(&p_bar[g][k & 1]);
     }
-    if (ok) ok = mbar_wait(&pv_bar[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, &aborted);
+    if (ok)
+      ok = mbar_wait(&pv_bar[g][(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, &aborted);
     if (!ok) {
       aborted = 1;
     } else {
@@ -393,7 +415,7 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
-        tc::ld32(t_o + lane_base + c * 32, o);
+        tc::ld32(t_o + c * 32, o);
         if (valid) {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -409,22 +431,23 @@ __global__ void __launch_bounds__(kTcRows + 64, 1)
   __syncthreads();
   if (warp == kMma) {
     tc::fence_after_sync();
-    tc::dealloc(tmem, kTmemCols);
+    tc::dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-template <class QF, int D, int G>
+template <class QF, int D, int G, int NG>
 cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                       int32_t max_query_len, cudaStream_t stream) {
-  using C = TcCfg<QF, D, G>;
-  // at least 80 KB so that at most two CTAs (2 x 256 tensor-memory columns) share an SM
-  const size_t smem = std::max<size_t>(1024 + C::BYTES, 80 * 1024);
-  auto kern = paged_prefill_tc_kernel<QF, D, G>;
+  using C = TcCfg<QF, D, G, NG>;
+  // shared memory keeps the tensor memory of the CTAs on one SM within 512
+  // columns: one CTA of two groups, or at most two CTAs of one (>= 80 KB each)
+  const size_t smem = std::max<size_t>(1024 + C::BYTES, NG == 2 ? 120 * 1024 : 80 * 1024);
+  auto kern = paged_prefill_tc_kernel<QF, D, G, NG>;
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const unsigned tiles = static_cast<unsigned>((max_query_len + C::QT - 1) / C::QT);
-  return launch_pdl(kern, dim3(tiles, a.num_kv_heads, a.num_seqs), kTcRows + 64, smem, stream,
-                    a, kmap, vmap);
+  return launch_pdl(kern, dim3(tiles, a.num_kv_heads, a.num_seqs), NG * kTcRows + 64, smem,
+                    stream, a, kmap, vmap);
 }
 
 }  // namespace
@@ -432,8 +455,12 @@ cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUten
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, int q_dtype, int head_dim, int group,
                               int32_t max_query_len, cudaStream_t stream) {
-#define PAGED_TC(QF, d, g) \
-  if (head_dim == d && group == g) return launch_tc<QF, d, g>(a, kmap, vmap, max_query_len, stream);
+  // two row groups (256 rows) when the chunks fill them
+  const bool two = static_cast<int64_t>(max_query_len) * group >= 2 * kTcRows;
+#define PAGED_TC(QF, d, g)                                                              \
+  if (head_dim == d && group == g)                                                      \
+    return two ? launch_tc<QF, d, g, 2>(a, kmap, vmap, max_query_len, stream)          \
+               : launch_tc<QF, d, g, 1>(a, kmap, vmap, max_query_len, stream);
 #define PAGED_TC_ALL(QF)                                                  \
   PAGED_TC(QF, 64, 1) PAGED_TC(QF, 64, 2) PAGED_TC(QF, 64, 4) PAGED_TC(QF, 64, 8) \
   PAGED_TC(QF, 128, 1) PAGED_TC(QF, 128, 2) PAGED_TC(QF, 128, 4) PAGED_TC(QF, 128, 8)
