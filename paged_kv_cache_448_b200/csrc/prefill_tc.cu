@@ -325,27 +325,33 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       if (!ok) break;
       tc::fence_after_sync();
       float x[NT];
-      const uint32_t t_s = t_grp + (k & 1) * NT + lane_base;
-      tc::ld32(t_s, *reinterpret_cast<float(*)[32]>(x));
-      tc::ld32(t_s + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+      tc::ld64(t_grp + (k & 1) * NT + lane_base, x);
       const int tk0 = k * NT;
-      float mx = -CUDART_INF_F;
+      // causal mask only where the step reaches past this row's position
+      if (tk0 + NT - 1 > p_row) {
 #pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        x[i] = tk0 + i <= p_row ? x[i] * qscale : -CUDART_INF_F;
-        mx = fmaxf(mx, x[i]);
+        for (int i = 0; i < NT; ++i) x[i] = tk0 + i <= p_row ? x[i] : -CUDART_INF_F;
       }
+      // row maximum of the raw logits (the scale is positive): 8 partial chains
+      float m8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m8[j] = x[j];
+#pragma unroll
+      for (int i = 8; i < NT; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * qscale;
       const bool rescale = mx > m_used + 8.f;   // false while the row sees nothing
-      const float alpha = rescale ? exp2f(m_used - mx) : 1.f;
+      const float alpha = rescale ? tc::ex2(m_used - mx) : 1.f;
       if (rescale) m_used = mx;
       const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
-      float ps = 0.f;
+      // p = 2^(s * scale - m), summed in 8 partial chains
+      float s8[8] = {};
 #pragma unroll
       for (int i = 0; i < NT; ++i) {
-        x[i] = exp2f(x[i] - mu);
-        ps += x[i];
+        x[i] = tc::ex2(fmaf(x[i], qscale, -mu));
+        s8[i & 7] += x[i];
       }
-      l = l * alpha + ps;
+      l = l * alpha + (((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7])));
       // The P set of step k is free once O += P V of step k-PB completed; O may
       // be rescaled only once O += P V of step k-1 completed (rare: the
       // maximum moves lazily), otherwise that MMA keeps running under this softmax
