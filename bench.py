@@ -348,7 +348,9 @@ def run_prefill(args):
     bt = torch.from_numpy(st.block_tables).to(dev)
     cl = torch.from_numpy(sp.context_lens).to(dev)
     out = torch.empty_like(q)
-    ws = pk.decode_workspace(1, 1, 1, sp.head_dim, sp.block_size, 0, 0, device=dev)
+    ws = pk.chunked_prefill_workspace(sp.num_seqs, int(qlens.sum()), sp.num_heads,
+                                      sp.num_kv_heads, sp.head_dim, chunk,
+                                      int(sp.context_lens.max()), device=dev)
     mctx = int(sp.context_lens.max())
     fn = lambda: pk.chunked_prefill(out, q, cu, chunk, d["key_cache"], d["value_cache"], bt, cl,
                                     mctx, sp.scale, workspace=ws)

@@ -202,8 +202,10 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* query,
  * key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens,
  * max_context_len, num_blocks: as in pa_decode (context_lens include the
  * query tokens).
- * workspace       >= 256 bytes, 256-byte aligned, zeroed once (pa_workspace_init);
- *                 its error word reports, through pa_decode_check, table
+ * workspace       >= pa_chunked_prefill_workspace_size(...) bytes, 256-byte aligned,
+ *                 zeroed once (pa_workspace_init). Short chunks whose CTAs cannot
+ *                 fill the GPU split each key range into parts combined by a
+ *                 second kernel, with partial results here. Its error word reports, through pa_decode_check, table
  *                 entries outside the pool (read as zeros), clipped context
  *                 lengths, and a query longer than its context (bit 16; those
  *                 rows are written as zeros).
@@ -219,6 +221,15 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
                                     int32_t head_dim, int32_t block_size, int64_t num_blocks,
                                     float scale, pa_dtype dtype, void* workspace,
                                     size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * Bytes of workspace pa_chunked_prefill needs for these sizes on the current
+ * device (256 when the key range is not split). Returns 0 for invalid sizes.
+ */
+PA_API size_t pa_chunked_prefill_workspace_size(int32_t num_seqs, int32_t num_tokens,
+                                                int32_t num_heads, int32_t num_kv_heads,
+                                                int32_t head_dim, int32_t max_query_len,
+                                                int32_t max_context_len);
 
 /*
  * Bytes of workspace pa_decode needs for these sizes on the current device

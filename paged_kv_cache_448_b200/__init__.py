@@ -22,7 +22,8 @@ from ._native import PagedError, check
 
 __all__ = ["reshape_and_cache", "decode", "decode_noalloc", "decode_workspace",
            "decode_workspace_size",
-           "decode_partition_tokens", "decode_check", "chunked_prefill", "copy_blocks", "sha256", "block_hash",
+           "decode_partition_tokens", "decode_check", "chunked_prefill",
+           "chunked_prefill_workspace", "chunked_prefill_workspace_size", "copy_blocks", "sha256", "block_hash",
            "prompt_block_hashes", "BlockAllocator",
            "build_block_table",
            "build_slot_mapping", "PagedError", "dtype_code"]
@@ -133,6 +134,23 @@ def _i32(a) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=np.int32)
 
 
+def chunked_prefill_workspace_size(num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
+                                   max_query_len, max_context_len) -> int:
+    return int(_native.lib().pa_chunked_prefill_workspace_size(
+        num_seqs, num_tokens, num_heads, num_kv_heads, head_dim, max_query_len, max_context_len))
+
+
+def chunked_prefill_workspace(num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
+                              max_query_len, max_context_len, device="cuda", stream=None):
+    """A device workspace for pa_chunked_prefill, error word zeroed."""
+    import torch
+    n = chunked_prefill_workspace_size(num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
+                                       max_query_len, max_context_len)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    check(_native.lib().pa_workspace_init(_ptr(ws), ws.numel(), _stream_handle(stream)))
+    return ws
+
+
 def chunked_prefill(out, query, cu_query_lens, max_query_len: int, key_cache, value_cache,
                     block_tables, context_lens, max_context_len: int, scale: float, *,
                     workspace=None, stream=None):
@@ -143,7 +161,8 @@ def chunked_prefill(out, query, cu_query_lens, max_query_len: int, key_cache, va
     NB, BS, Hkv = key_cache.shape[:3]
     S = context_lens.shape[0]
     if workspace is None:
-        workspace = decode_workspace(1, 1, 1, D, BS, 0, 0, device=query.device, stream=stream)
+        workspace = chunked_prefill_workspace(S, T, H, Hkv, D, max_query_len, max_context_len,
+                                              device=query.device, stream=stream)
     check(_native.lib().pa_chunked_prefill(
         _ptr(out), _ptr(query), _ptr(cu_query_lens), T, int(max_query_len), _ptr(key_cache),
         _ptr(value_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),

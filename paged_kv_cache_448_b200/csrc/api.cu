@@ -414,6 +414,66 @@ PA_API pa_status pa_copy_blocks(const void* src_key_cache, const void* src_value
   return cuda_status(e, "copy_blocks");
 }
 
+}  // extern "C"
+
+namespace paged {
+namespace {
+
+// Split of the key range for the multi-token query (mma.sync kernel only):
+// when its CTAs (query tiles x kv-heads x sequences) cannot fill about four
+// waves of three CTAs per SM, the tiles of each CTA are cut into parts of at
+// least 256 tokens (16 tiles, a multiple of 4) handled by separate CTAs.
+struct PrefillPlan {
+  bool tc;                  // tcgen05 kernel (no split)
+  int32_t q_tiles, partition_tiles, max_parts;
+};
+
+PrefillPlan make_prefill_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t group,
+                              int32_t max_query_len, int32_t max_context_len) {
+  PrefillPlan p{};
+  p.tc = static_cast<int64_t>(max_query_len) * group >= 128;
+  p.q_tiles = (max_query_len + prefill_tokens_per_cta(group) - 1) / prefill_tokens_per_cta(group);
+  const int32_t max_tiles = std::max<int32_t>(1, (max_context_len + 15) / 16);
+  p.partition_tiles = max_tiles;
+  p.max_parts = 1;
+  if (p.tc) return p;
+  const int64_t ctas = static_cast<int64_t>(p.q_tiles) * num_kv_heads * num_seqs;
+  const int64_t want = 4LL * sm_count() * 3;
+  if (ctas >= want || max_tiles < 32) return p;
+  const int64_t by_work = (want + ctas - 1) / ctas;
+  const int32_t parts = static_cast<int32_t>(std::min<int64_t>(by_work, max_tiles / 16));
+  if (parts <= 1) return p;
+  int32_t pt = (max_tiles + parts - 1) / parts;
+  pt = (pt + 3) / 4 * 4;
+  p.partition_tiles = pt;
+  p.max_parts = (max_tiles + pt - 1) / pt;
+  return p;
+}
+
+size_t prefill_workspace_bytes(const PrefillPlan& p, int32_t num_tokens, int32_t num_heads,
+                               int32_t head_dim) {
+  if (p.max_parts <= 1) return kHeaderBytes;
+  const size_t rows = static_cast<size_t>(num_tokens) * num_heads * p.max_parts;
+  return align256(kHeaderBytes + rows * sizeof(float2)) + rows * head_dim * sizeof(float);
+}
+
+}  // namespace
+}  // namespace paged
+
+extern "C" {
+
+PA_API size_t pa_chunked_prefill_workspace_size(int32_t num_seqs, int32_t num_tokens,
+                                                int32_t num_heads, int32_t num_kv_heads,
+                                                int32_t head_dim, int32_t max_query_len,
+                                                int32_t max_context_len) {
+  if (num_seqs < 0 || num_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      max_query_len < 0 || max_context_len < 0 || num_heads % num_kv_heads != 0)
+    return 0;
+  const PrefillPlan p = make_prefill_plan(num_seqs, num_kv_heads, num_heads / num_kv_heads,
+                                          max_query_len, max_context_len);
+  return prefill_workspace_bytes(p, num_tokens, num_heads, head_dim);
+}
+
 PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t* cu_query_lens,
                                     int32_t num_tokens, int32_t max_query_len,
                                     const void* key_cache, const void* value_cache,
@@ -457,7 +517,13 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
   // Chunks that fill the 128 rows of a tensor-memory CTA (query tokens x heads
   // of a kv-head's group) run on tcgen05; shorter ones (a few draft tokens)
   // on the 64-row mma.sync kernel, which wastes fewer rows.
-  const bool tc = static_cast<int64_t>(max_query_len) * group >= 128;
+  const PrefillPlan plan =
+      make_prefill_plan(num_seqs, num_kv_heads, group, max_query_len, max_context_len);
+  const bool tc = plan.tc;
+  const size_t need = prefill_workspace_bytes(plan, num_tokens, num_heads, head_dim);
+  if (workspace_bytes < need)
+    return fail(PA_ERR_INVALID_ARG, "chunked_prefill: workspace %zu bytes < %zu needed",
+                workspace_bytes, need);
   pa_status st = encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads,
                                   head_dim, 2, tc);
   if (st == PA_OK)
@@ -481,6 +547,15 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
   a.num_kv_heads = num_kv_heads;
   a.block_size = block_size;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.q_tiles = plan.q_tiles;
+  a.partition_tiles = plan.partition_tiles;
+  a.max_parts = plan.max_parts;
+  if (plan.max_parts > 1) {
+    const size_t rows = static_cast<size_t>(num_tokens) * num_heads * plan.max_parts;
+    a.ws_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + kHeaderBytes);
+    a.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                      align256(kHeaderBytes + rows * sizeof(float2)));
+  }
   auto launch = tc ? launch_prefill_tc : launch_prefill;
   return cuda_status(launch(a, kmap, vmap, dtype == PA_F16 ? kF16 : kBF16, head_dim, group,
                             max_query_len, reinterpret_cast<cudaStream_t>(stream)),

@@ -23,14 +23,24 @@ struct PrefillArgs {
   int32_t num_kv_heads;
   int32_t block_size;
   float scale_log2;              // softmax scale * log2(e)
+  // split of the key range (mma.sync kernel only; 1 part = no split)
+  int32_t q_tiles;               // query tiles per (sequence, kv-head) in the launch
+  int32_t partition_tiles;       // 16-token tiles per part
+  int32_t max_parts;
+  float* ws_o;                   // [T * H][max_parts][D] partial outputs (normalised)
+  float2* ws_ml;                 // [T * H][max_parts] (max, sum) in base-2 units
 };
 
 // Failure site of a prefill wait that gave up.
 enum : int32_t { kSitePrefill = 5 };
 
-// Launch for one (q dtype == cache dtype) pair; q_tiles = ceil(max_query_len
-// / tokens per CTA) is computed inside. cudaErrorNotSupported for shapes
-// without a kernel.
+// Query tokens per CTA of the mma.sync kernel (64 rows = tokens x group).
+__host__ __device__ constexpr int prefill_tokens_per_cta(int group) { return 64 / group; }
+
+// mma.sync kernel for one (q dtype == cache dtype) pair: grid of
+// a.q_tiles * a.max_parts CTAs per (sequence, kv-head), then, when the key
+// range is split (a.max_parts > 1), the combine kernel. cudaErrorNotSupported
+// for shapes without a kernel.
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                            int q_dtype, int head_dim, int group, int32_t max_query_len,
                            cudaStream_t stream);

@@ -81,7 +81,8 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
   uint64_t* empty = full + R;
   __shared__ int aborted;
 
-  const int z = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+  const int z = blockIdx.x % a.q_tiles, part = blockIdx.x / a.q_tiles;
+  const int kvh = blockIdx.y, s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int r = 0; r < R; ++r) {
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
   const int qlen = a.cu_query_lens[s + 1] - q0;
   int ctx = a.context_lens[s];
   if (ctx > a.ctx_limit || ctx < 0) {
-    if (threadIdx.x == 0 && z == 0 && kvh == 0) report(a.err, kErrContextClipped);
+    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) report(a.err, kErrContextClipped);
     ctx = ctx < 0 ? 0 : a.ctx_limit;
   }
   const int tok0 = z * QT;
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
                           r_hi % G) * D;
 
   if (qlen > ctx) {  // a query longer than its context: rows become zeros
+    if (part > 0) return;
     if (threadIdx.x == 0 && z == 0 && kvh == 0) report(a.err, kErrQueryLonger);
     uint32_t* out32 = static_cast<uint32_t*>(a.out);
     for (int j = 0; j < NO; ++j) {
@@ -128,7 +130,13 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
     return;
   }
   const int pos0 = ctx - qlen + tok0;       // position of the CTA's first query token
-  const int ntiles = (pos0 + ntok - 1) / TR + 1;
+  // 16-token tiles up to the CTA's last position, cut into parts of
+  // partition_tiles; this CTA takes part `part`: tiles tbase .. tbase+ntiles-1
+  const int ntiles_all = (pos0 + ntok - 1) / TR + 1;
+  const int parts = (ntiles_all + a.partition_tiles - 1) / a.partition_tiles;
+  if (part >= parts) return;
+  const int tbase = part * a.partition_tiles;
+  const int ntiles = min(ntiles_all - tbase, a.partition_tiles);
   const int p_lo = v_lo ? pos0 + tk_lo : -1, p_hi = v_hi ? pos0 + tk_hi : -1;
   const int p_min = min(p_lo, p_hi);
 
@@ -141,7 +149,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
       report(a.err, kErrBadBlockId);
       bid = -1;  // read as a box outside the pool: zero-filled
     }
-    const int32_t row0 = bid >= 0 ? bid * a.block_size + (t * TR) % a.block_size : -TR;
+    const int32_t row0 = bid >= 0 ? bid * a.block_size + ((tbase + t) * TR) % a.block_size : -TR;
     uint8_t* kt = smem + stage * STAGE;
     mbar_arrive_expect_tx(&full[stage], STAGE);
     tma_load_4d(kt, &kmap, &full[stage], 0, row0, kvh, 0, policy);
@@ -154,7 +162,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
 #pragma unroll
     for (int j = 0; j < kPrefillTps; ++j) {
       const int tt = k * kPrefillTps + j;
-      bid[j] = tt < ntiles ? table[(tt * TR) / a.block_size] : 0;
+      bid[j] = tt < ntiles ? table[((tbase + tt) * TR) / a.block_size] : 0;
     }
 #pragma unroll
     for (int j = 0; j < kPrefillTps; ++j) {
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
     float mx_lo = -CUDART_INF_F, mx_hi = -CUDART_INF_F;
 #pragma unroll
     for (int j = 0; j < kPrefillTps; ++j) {
-      const int tok_base = (t0 + j) * TR;
+      const int tok_base = (tbase + t0 + j) * TR;
       const bool masked = tok_base + TR - 1 > p_min;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -293,7 +301,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
       const int tt = t0 + j;
       if (tt >= ntiles) break;
       uint8_t* vt = smem + (tt % R) * STAGE + T::BYTES;
-      const int tok_base = tt * TR;
+      const int tok_base = (tbase + tt) * TR;
       // Rows of the tile past the context may hold anything (even NaN) and
       // 0 * NaN is NaN inside the MMA: each warp clears them in its view of
       // the stage before reading V (every warp writes the same zeros; only
@@ -360,12 +368,75 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
   l_hi += __shfl_xor_sync(FULL, l_hi, 1);
   l_hi += __shfl_xor_sync(FULL, l_hi, 2);
   const float i_lo = l_lo > 0.f ? 1.f / l_lo : 0.f, i_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
-  uint32_t* out32 = static_cast<uint32_t*>(a.out);
+  if (parts == 1) {
+    uint32_t* out32 = static_cast<uint32_t*>(a.out);
+#pragma unroll
+    for (int j = 0; j < NO; ++j) {
+      if (v_lo) out32[(row_lo + j * 8 + 2 * c) / 2] = pack2<BF>(o[j][0] * i_lo, o[j][1] * i_lo);
+      if (v_hi) out32[(row_hi + j * 8 + 2 * c) / 2] = pack2<BF>(o[j][2] * i_hi, o[j][3] * i_hi);
+    }
+    return;
+  }
+  // a part of a split key range: (max, sum) and the output normalised by this
+  // part's sum, per row (a row that sees none of this part's tokens leaves
+  // max = -inf, sum = 0); the combine kernel merges the parts
+  const int64_t pl = (row_lo / D) * a.max_parts + part, ph = (row_hi / D) * a.max_parts + part;
+  if (v_lo && c == 0) a.ws_ml[pl] = make_float2(m_lo, l_lo);
+  if (v_hi && c == 0) a.ws_ml[ph] = make_float2(m_hi, l_hi);
 #pragma unroll
   for (int j = 0; j < NO; ++j) {
-    if (v_lo) out32[(row_lo + j * 8 + 2 * c) / 2] = pack2<BF>(o[j][0] * i_lo, o[j][1] * i_lo);
-    if (v_hi) out32[(row_hi + j * 8 + 2 * c) / 2] = pack2<BF>(o[j][2] * i_hi, o[j][3] * i_hi);
+    if (v_lo)
+      *reinterpret_cast<float2*>(a.ws_o + pl * D + j * 8 + 2 * c) =
+          make_float2(o[j][0] * i_lo, o[j][1] * i_lo);
+    if (v_hi)
+      *reinterpret_cast<float2*>(a.ws_o + ph * D + j * 8 + 2 * c) =
+          make_float2(o[j][2] * i_hi, o[j][3] * i_hi);
   }
+}
+
+// Merge the parts of a split key range: part p of row r left (m_p, l_p) and
+// o_p normalised by l_p (base-2 units), so with M = max_p m_p and
+// w_p = l_p 2^(m_p - M): out = sum_p w_p o_p / sum_p w_p. One warp per
+// (query token, head); rows whose range was not split were written directly.
+template <class QF, int D>
+__global__ void __launch_bounds__(128) paged_prefill_combine(const PrefillArgs a, int group) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x * 4 + warp, i = blockIdx.y, s = blockIdx.z;
+  if (h >= a.num_heads) return;
+  const int q0 = a.cu_query_lens[s], qlen = a.cu_query_lens[s + 1] - q0;
+  if (i >= qlen) return;
+  int ctx = a.context_lens[s];
+  ctx = ctx < 0 ? 0 : (ctx > a.ctx_limit ? a.ctx_limit : ctx);
+  if (qlen > ctx) return;  // rows zeroed by the main kernel
+  const int qt = prefill_tokens_per_cta(group);
+  const int tok0 = (i / qt) * qt, ntok = min(qt, qlen - tok0);
+  const int pos0 = ctx - qlen + tok0;
+  const int ntiles_all = (pos0 + ntok - 1) / kTileRows + 1;
+  const int parts = (ntiles_all + a.partition_tiles - 1) / a.partition_tiles;
+  if (parts <= 1) return;
+  const int64_t row = static_cast<int64_t>(q0 + i) * a.num_heads + h;
+  const float2* ml = a.ws_ml + row * a.max_parts;
+  float M = -CUDART_INF_F;
+  for (int p = lane; p < parts; p += 32) M = fmaxf(M, ml[p].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  constexpr int PER = D / 32;
+  float acc[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) acc[j] = 0.f;
+  float L = 0.f;
+  const float* op = a.ws_o + row * a.max_parts * D;
+  for (int p = 0; p < parts; ++p) {
+    const float2 v = ml[p];
+    const float w = v.x == -CUDART_INF_F ? 0.f : v.y * exp2f(v.x - M);
+    L += w;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) acc[j] = fmaf(w, op[p * D + lane + 32 * j], acc[j]);
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) store_out(QF{}, a.out, row * D + lane + 32 * j, acc[j] * inv);
 }
 
 template <class QF, int D, int G>
@@ -377,9 +448,14 @@ cudaError_t launch_one(const PrefillArgs& a, const CUtensorMap& kmap, const CUte
   auto kern = paged_prefill_kernel<QF, D, G>;
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  const unsigned tiles = static_cast<unsigned>((max_query_len + QT - 1) / QT);
-  return launch_pdl(kern, dim3(tiles, a.num_kv_heads, a.num_seqs), kPrefillWarps * 32, smem,
-                    stream, a, kmap, vmap);
+  static_assert(QT == prefill_tokens_per_cta(G), "tokens per CTA");
+  e = launch_pdl(kern, dim3(static_cast<unsigned>(a.q_tiles * a.max_parts), a.num_kv_heads,
+                            a.num_seqs),
+                 kPrefillWarps * 32, smem, stream, a, kmap, vmap);
+  if (e != cudaSuccess || a.max_parts <= 1) return e;
+  return launch_pdl(paged_prefill_combine<QF, D>,
+                    dim3((a.num_heads + 3) / 4, static_cast<unsigned>(max_query_len), a.num_seqs),
+                    128, 0, stream, a, G);
 }
 
 }  // namespace

@@ -265,6 +265,18 @@ def test_prefix_cache_matches_oracle_model_on_random_requests():
                 assert ours.lookup(h) == b
 
 
+def test_chunked_prefill_workspace_plan():
+    # chunks that fill a tensor-memory CTA never split: header only
+    assert pk.chunked_prefill_workspace_size(16, 16 * 512, 32, 32, 128, 512, 4096) == 256
+    # short chunks of many sequences already fill the GPU: no split
+    assert pk.chunked_prefill_workspace_size(4096, 4096 * 8, 64, 8, 128, 8, 4096) == 256
+    # few short-chunk CTAs with long contexts: partial rows for every part
+    n = pk.chunked_prefill_workspace_size(64, 64 * 8, 64, 8, 128, 8, 4096)
+    rows = 64 * 8 * 64
+    assert n > 256 and (n - 256) % (rows * (8 + 128 * 4)) < 256
+    assert pk.chunked_prefill_workspace_size(1, 1, 3, 2, 128, 1, 10) == 0   # H % Hkv != 0
+
+
 def test_copy_blocks_rejects_bad_arguments_before_launch():
     lib = _native.lib()
     P = 1 << 20                                 # any 16-byte aligned address; never touched

@@ -24,7 +24,9 @@ def run_gpu(sp, st, hd, q, qlens, table=None, ctx=None):
     table = st.block_tables if table is None else table
     gq = dev(q, sp.q_dtype)
     out = torch.full_like(gq, float("nan"))
-    ws = pk.decode_workspace(1, 1, 1, sp.head_dim, sp.block_size, 0, 0)
+    ws = pk.chunked_prefill_workspace(sp.num_seqs, int(qlens.sum()), sp.num_heads,
+                                      sp.num_kv_heads, sp.head_dim, int(qlens.max()),
+                                      int(np.max(ctx)))
     pk.chunked_prefill(out, gq, i32(cu), int(qlens.max()), dev(hd.key_cache, sp.cache_dtype),
                        dev(hd.value_cache, sp.cache_dtype), i32(table), i32(ctx),
                        int(np.max(ctx)), sp.scale, workspace=ws)
@@ -85,6 +87,22 @@ def test_multi_token_edge_sweep(kernel, dt, G, D, bs):
                  f"{dt} G{G} D{D} bs{bs}")
 
 
+@pytest.mark.parametrize("dt,G,D,bs", [("bf16", 8, 128, 16), ("f16", 4, 64, 32),
+                                       ("bf16", 2, 128, 32), ("f16", 1, 128, 16)])
+def test_split_key_range_for_short_chunks(dt, G, D, bs):
+    """Few CTAs (short chunks, few sequences and kv-heads) and long contexts:
+    the key range is cut into parts combined by a second kernel; ragged last
+    parts, rows whose causal range ends inside an earlier part."""
+    ctxs, qlens = [2100, 700, 3333], [8, 5, 8]
+    assert max(qlens) * G < 128
+    assert pk.chunked_prefill_workspace_size(3, sum(qlens), 2 * G, 2, D, 8, 3333) > 256
+    sp, st, hd, q, qlens = custom(ctxs, qlens, 2 * G, 2, D, bs, dt, seed=900 + G)
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), dt,
+                 f"split {dt} G{G} D{D} bs{bs}")
+
+
 def test_one_token_per_sequence_matches_decode_and_oracle():
     sp, st, hd, q, qlens = custom([5, 64, 300, 1], [1, 1, 1, 1], 16, 2, 128, 16, "bf16", seed=5)
     out, ws, cu = run_gpu(sp, st, hd, q, qlens)
@@ -141,7 +159,9 @@ def test_multi_token_full_size_sampled(name):
     q = wl.prefill_queries_device(sp, qlens)
     cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
     out = torch.empty_like(q)
-    ws = pk.decode_workspace(1, 1, 1, sp.head_dim, sp.block_size, 0, 0)
+    ws = pk.chunked_prefill_workspace(sp.num_seqs, int(qlens.sum()), sp.num_heads,
+                                      sp.num_kv_heads, sp.head_dim, int(qlens.max()),
+                                      int(sp.context_lens.max()))
     pk.chunked_prefill(out, q, i32(cu), int(qlens.max()), d["key_cache"], d["value_cache"],
                        i32(st.block_tables), i32(sp.context_lens), int(sp.context_lens.max()),
                        sp.scale, workspace=ws)
