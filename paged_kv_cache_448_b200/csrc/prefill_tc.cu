@@ -59,9 +59,11 @@ struct TcCfg {
   static constexpr int P_SET = (BF ? 2 : 1) * P_BYTES;  // P (and for bf16 its residual)
   // P sets per group: two (steps k and k+1) where shared memory allows
   static constexpr int PB = (BF && NG == 2) ? 1 : 2;
+  // ring depths: K (needed first, by S) three steps deep where shared memory allows
+  static constexpr int KR = kTcStages, VR = kTcStages;
   static constexpr int OFF_K = NG * QG_BYTES;                   // K ring
-  static constexpr int OFF_V = OFF_K + kTcStages * KV_BYTES;    // V ring
-  static constexpr int OFF_P = OFF_V + kTcStages * KV_BYTES;    // [group][PB] P sets
+  static constexpr int OFF_V = OFF_K + KR * KV_BYTES;           // V ring
+  static constexpr int OFF_P = OFF_V + VR * KV_BYTES;           // [group][PB] P sets
   static constexpr int BYTES = OFF_P + NG * PB * P_SET;
   static constexpr uint32_t TMEM_COLS = NG * kTmemGroup;
   static constexpr uint32_t IDESC_S = tc::idesc_f16<BF, kTcRows, kTcNT, false>();
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
                             const __grid_constant__ CUtensorMap vmap) {
   using C = TcCfg<QF, D, G, NG>;
   constexpr bool BF = C::BF;
-  constexpr int NSEG = C::NSEG, QT = C::QT, R = kTcStages, NT = kTcNT, TR = kTileRows;
+  constexpr int NSEG = C::NSEG, QT = C::QT, KR = C::KR, VR = C::VR, NT = kTcNT, TR = kTileRows;
   constexpr int PB = C::PB;
   constexpr int kMma = NG * kTcRows / 32;   // warp issuing the MMAs (owns the tensor memory)
   constexpr int kLoader = kMma + 1;         // warp issuing the TMA loads
@@ -95,14 +97,14 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   auto sq = [&](int g) { return smem + g * C::QG_BYTES; };
-  auto sk = [&](int k) { return smem + C::OFF_K + (k % R) * C::KV_BYTES; };
-  auto sv = [&](int k) { return smem + C::OFF_V + (k % R) * C::KV_BYTES; };
+  auto sk = [&](int k) { return smem + C::OFF_K + (k % KR) * C::KV_BYTES; };
+  auto sv = [&](int k) { return smem + C::OFF_V + (k % VR) * C::KV_BYTES; };
   auto sp = [&](int g, int k) { return smem + C::OFF_P + (g * PB + k % PB) * C::P_SET; };
   // K / V rings: *full when a stage's boxes landed, *empty when the MMAs that
   // read it completed (both groups). Per group g: s_bar[g][b] S buffer b
   // computed; p_bar[g][b] the group's softmax warps wrote P of a step of parity
   // b (and rescaled O); pv_bar[g][b] O += P V of such a step done.
-  __shared__ uint64_t kfull[R], kempty[R], vfull[R], vempty[R], s_bar[NG][2], p_bar[NG][2],
+  __shared__ uint64_t kfull[KR], kempty[KR], vfull[VR], vempty[VR], s_bar[NG][2], p_bar[NG][2],
       pv_bar[NG][2], drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int aborted;
@@ -110,9 +112,11 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   const int z = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int r = 0; r < R; ++r) {
+    for (int r = 0; r < KR; ++r) {
       mbar_init(&kfull[r], 1);
       mbar_init(&kempty[r], 1);
+    }
+    for (int r = 0; r < VR; ++r) {
       mbar_init(&vfull[r], 1);
       mbar_init(&vempty[r], 1);
     }
@@ -181,12 +185,14 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
 
   if (warp == kLoader) {
     // ================= TMA loads (one thread) =================
+    // K of step k is issued before V of step k-1: K (needed first, by S) never
+    // waits behind the release of a V stage.
     if (lane == 0) {
       const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
       const uint64_t policy = l2_policy_evict_last();  // other query tiles read them too
-      auto issue_kv = [&](int k, const int32_t (&bid)[NT / TR], bool is_v) {
+      auto issue = [&](int k, const int32_t (&bid)[NT / TR], bool is_v) {
         uint8_t* dst = is_v ? sv(k) : sk(k);
-        uint64_t* bar = is_v ? &vfull[k % R] : &kfull[k % R];
+        uint64_t* bar = is_v ? &vfull[k % VR] : &kfull[k % KR];
         const CUtensorMap* map = is_v ? &vmap : &kmap;
         const int t_begin = k * (NT / TR), t_end = min(ntiles, (k + 1) * (NT / TR));
         mbar_arrive_expect_tx(bar, static_cast<uint32_t>(NSEG * (t_end - t_begin) * TR * 128));
@@ -205,8 +211,8 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
             tma_load_4d(dst + sg * C::KV_SEG + j * TR * 128, map, bar, 0, row0, kvh, sg, policy);
         }
       };
-      // block ids of the next step are fetched while the current one is issued
-      int32_t bid[NT / TR], nbid[NT / TR];
+      // block ids: of step k (for K) and of step k-1 (kept for V)
+      int32_t bid[NT / TR], pbid[NT / TR];
       auto load_ids = [&](int k, int32_t (&dst)[NT / TR]) {
 #pragma unroll
         for (int j = 0; j < NT / TR; ++j) {
@@ -214,22 +220,26 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
           dst[j] = t < ntiles ? table[(t * TR) / a.block_size] : 0;
         }
       };
-      load_ids(0, bid);
       bool ok = true;
-      int k = 0;
-      for (; ok && k < nsteps; ++k) {
-        if (k + 1 < nsteps) load_ids(k + 1, nbid);
-        if (k >= R) {  // the stage's previous step: S done (K), O += P V done (V)
-          ok = mbar_wait(&kempty[k % R], ((k - R) / R) & 1, &aborted);
-          if (ok) issue_kv(k, bid, false);
-          ok = ok && mbar_wait(&vempty[k % R], ((k - R) / R) & 1, &aborted);
-          if (ok) issue_kv(k, bid, true);
-        } else {
-          issue_kv(k, bid, false);
-          issue_kv(k, bid, true);
+      int kk_issued = 0, vv_issued = 0;
+      for (int k = 0; ok && k <= nsteps; ++k) {
+        if (k < nsteps) {
+          load_ids(k, bid);
+          if (k >= KR) ok = mbar_wait(&kempty[k % KR], ((k - KR) / KR) & 1, &aborted);
+          if (ok) {
+            issue(k, bid, false);
+            kk_issued = k + 1;
+          }
+        }
+        if (ok && k >= 1) {
+          if (k - 1 >= VR) ok = mbar_wait(&vempty[(k - 1) % VR], ((k - 1 - VR) / VR) & 1, &aborted);
+          if (ok) {
+            issue(k - 1, pbid, true);
+            vv_issued = k;
+          }
         }
 #pragma unroll
-        for (int j = 0; j < NT / TR; ++j) bid[j] = nbid[j];
+        for (int j = 0; j < NT / TR; ++j) pbid[j] = bid[j];
       }
       if (!ok) {
         aborted = 1;
@@ -237,33 +247,40 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       }
       // before the CTA's shared memory goes away every issued load must have
       // landed (the last use of each stage; earlier ones completed already)
-      for (int j = max(0, k - R); j < k; ++j) {
-        mbar_wait(&kfull[j % R], (j / R) & 1);
-        mbar_wait(&vfull[j % R], (j / R) & 1);
-      }
+      for (int j = max(0, kk_issued - KR); j < kk_issued; ++j)
+        mbar_wait(&kfull[j % KR], (j / KR) & 1);
+      for (int j = max(0, vv_issued - VR); j < vv_issued; ++j)
+        mbar_wait(&vfull[j % VR], (j / VR) & 1);
     }
   } else if (warp == kMma) {
     // ================= MMA issue (one thread) =================
     if (lane == 0) {
       int k_waited = 0, v_waited = 0;
+      // descriptors computed once; a k-step or stage offset is added to the
+      // start-address field (bits 0-13, in 16-byte units)
+      uint64_t qd[NG];
+      for (int g = 0; g < NG; ++g) qd[g] = tc::sw128_desc(sq(g), 16, 1024);
+      const uint64_t kd0 = tc::sw128_desc(sk(0), 16, 1024);
+      const uint64_t vd0 = tc::sw128_desc(sv(0), NT * 128, 1024);
+      const uint64_t pd0 = tc::sw128_desc(sp(0, 0), 16, 1024);
       auto issue_s = [&](int k) {  // S of step k for every group
-        if (!mbar_wait(&kfull[k % R], (k / R) & 1, &aborted)) return false;
+        if (!mbar_wait(&kfull[k % KR], (k / KR) & 1, &aborted)) return false;
         k_waited = k + 1;
         tc::fence_after_sync();
-        uint8_t* ks = sk(k);
+        const uint64_t kd = kd0 + static_cast<uint64_t>(((k % KR) * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const int sg = kk / 4, off = (kk % 4) * 32;
             tc::mma_f16(tmem + g * kTmemGroup + (k & 1) * NT,
-                        tc::sw128_desc(sq(g) + sg * (kTcRows * 128) + off, 16, 1024),
-                        tc::sw128_desc(ks + sg * C::KV_SEG + off, 16, 1024), C::IDESC_S,
+                        qd[g] + static_cast<uint64_t>((sg * (kTcRows * 128) + off) >> 4),
+                        kd + static_cast<uint64_t>((sg * C::KV_SEG + off) >> 4), C::IDESC_S,
                         kk > 0);
           }
           tc::commit(&s_bar[g][k & 1]);
         }
-        tc::commit(&kempty[k % R]);
+        tc::commit(&kempty[k % KR]);
         return true;
       };
       bool ok = issue_s(0);
@@ -274,28 +291,29 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
             ok = k < 1 || mbar_wait(&p_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted);
           ok = ok && issue_s(k + 1);
         }
-        if (ok) ok = mbar_wait(&vfull[k % R], (k / R) & 1, &aborted);
+        if (ok) ok = mbar_wait(&vfull[k % VR], (k / VR) & 1, &aborted);
         if (ok) v_waited = k + 1;
         // O += P V of each group once its softmax warps wrote P of step k
+        const uint64_t vd = vd0 + static_cast<uint64_t>(((k % VR) * C::KV_BYTES) >> 4);
         for (int g = 0; ok && g < NG; ++g) {
           ok = mbar_wait(&p_bar[g][k & 1], (k >> 1) & 1, &aborted);
           if (!ok) break;
           tc::fence_after_sync();
-          uint8_t* vs = sv(k);
-          uint8_t* ps = sp(g, k);
+          const uint64_t pd =
+              pd0 + static_cast<uint64_t>(((g * PB + k % PB) * C::P_SET) >> 4);
           const uint32_t t_o = tmem + g * kTmemGroup + kTmemO;
 #pragma unroll
           for (int kk = 0; kk < NT / 16; ++kk) {
-            const uint64_t bv = tc::sw128_desc(vs + kk * 16 * 128, NT * 128, 1024);
-            tc::mma_f16(t_o, tc::sw128_desc(ps + kk * 32, 16, 1024), bv, C::IDESC_PV,
+            const uint64_t bv = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
+            tc::mma_f16(t_o, pd + static_cast<uint64_t>((kk * 32) >> 4), bv, C::IDESC_PV,
                         k > 0 || kk > 0);
             if constexpr (BF)
-              tc::mma_f16(t_o, tc::sw128_desc(ps + C::P_BYTES + kk * 32, 16, 1024), bv,
+              tc::mma_f16(t_o, pd + static_cast<uint64_t>((C::P_BYTES + kk * 32) >> 4), bv,
                           C::IDESC_PV, true);
           }
           tc::commit(&pv_bar[g][k & 1]);
         }
-        if (ok) tc::commit(&vempty[k % R]);
+        if (ok) tc::commit(&vempty[k % VR]);
       }
       if (!ok) {
         // A wait gave up (never expected): let this CTA's MMAs finish (bounded)
@@ -396,7 +414,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       const int vrows = max(0, min(NT, kv_valid - tk0));
       if (vrows < NT) {
         uint8_t* vs = sv(k);
-        ok = mbar_wait(&vfull[k % R], (k / R) & 1, &aborted);  // the TMA writes come first
+        ok = mbar_wait(&vfull[k % VR], (k / VR) & 1, &aborted);  // the TMA writes come first
         if (!ok) break;
         for (int i = rr; i < (NT - vrows) * NSEG * 8; i += kTcRows) {
           const int r = vrows + i / (NSEG * 8), sg = (i / 8) % NSEG, c = i % 8;
