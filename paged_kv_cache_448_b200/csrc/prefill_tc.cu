@@ -55,20 +55,15 @@ struct TcCfg {
   static constexpr int QG_BYTES = NSEG * kTcRows * 128;  // Q of one group
   static constexpr int KV_SEG = kTcNT * 128;        // one segment of K or V in a stage
   static constexpr int KV_BYTES = NSEG * KV_SEG;    // one stage of K (or V)
-  static constexpr int P_BYTES = kTcRows * kTcNT * 2;
-  static constexpr int P_SET = (BF ? 2 : 1) * P_BYTES;  // P (and for bf16 its residual)
-  // P sets per group: two (steps k and k+1) where shared memory allows
-  static constexpr int PB = (BF && NG == 2) ? 1 : 2;
-  // ring depths: K (needed first, by S) three steps deep where shared memory allows
+  // ring depths (K, needed first by S, and V)
   static constexpr int KR = kTcStages, VR = kTcStages;
   static constexpr int OFF_K = NG * QG_BYTES;                   // K ring
   static constexpr int OFF_V = OFF_K + KR * KV_BYTES;           // V ring
-  static constexpr int OFF_P = OFF_V + VR * KV_BYTES;           // [group][PB] P sets
-  static constexpr int BYTES = OFF_P + NG * PB * P_SET;
+  static constexpr int BYTES = OFF_V + VR * KV_BYTES;
   static constexpr uint32_t TMEM_COLS = NG * kTmemGroup;
   static constexpr uint32_t IDESC_S = tc::idesc_f16<BF, kTcRows, kTcNT, false>();
   static constexpr uint32_t IDESC_PV = tc::idesc_f16<BF, kTcRows, D, true>();
-  static_assert(kTcNT * 2 == 128, "a row of P is one 128-byte swizzle row");
+  static_assert(kTcNT == 64, "P (64 16-bit values) fills half of its S buffer's columns");
   static_assert(BYTES + 1024 <= 227 * 1024, "shared memory of one CTA");
 };
 
@@ -89,7 +84,6 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   using C = TcCfg<QF, D, G, NG>;
   constexpr bool BF = C::BF;
   constexpr int NSEG = C::NSEG, QT = C::QT, KR = C::KR, VR = C::VR, NT = kTcNT, TR = kTileRows;
-  constexpr int PB = C::PB;
   constexpr int kMma = NG * kTcRows / 32;   // warp issuing the MMAs (owns the tensor memory)
   constexpr int kLoader = kMma + 1;         // warp issuing the TMA loads
 
@@ -99,7 +93,6 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   auto sq = [&](int g) { return smem + g * C::QG_BYTES; };
   auto sk = [&](int k) { return smem + C::OFF_K + (k % KR) * C::KV_BYTES; };
   auto sv = [&](int k) { return smem + C::OFF_V + (k % VR) * C::KV_BYTES; };
-  auto sp = [&](int g, int k) { return smem + C::OFF_P + (g * PB + k % PB) * C::P_SET; };
   // K / V rings: *full when a stage's boxes landed, *empty when the MMAs that
   // read it completed (both groups). Per group g: s_bar[g][b] S buffer b
   // computed; p_bar[g][b] the group's softmax warps wrote P of a step of parity
@@ -262,7 +255,6 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       for (int g = 0; g < NG; ++g) qd[g] = tc::sw128_desc(sq(g), 16, 1024);
       const uint64_t kd0 = tc::sw128_desc(sk(0), 16, 1024);
       const uint64_t vd0 = tc::sw128_desc(sv(0), NT * 128, 1024);
-      const uint64_t pd0 = tc::sw128_desc(sp(0, 0), 16, 1024);
       auto issue_s = [&](int k) {  // S of step k for every group
         if (!mbar_wait(&kfull[k % KR], (k / KR) & 1, &aborted)) return false;
         k_waited = k + 1;
@@ -285,10 +277,12 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       };
       bool ok = issue_s(0);
       for (int k = 0; ok && k < nsteps; ++k) {
-        // S of the next step, into the S buffers the softmax of step k-1 released
+        // S of the next step, into the S buffers of step k-1: their softmax read
+        // S and wrote P there, and O += P V of step k-1 read P
         if (k + 1 < nsteps) {
-          for (int g = 0; ok && g < NG; ++g)
-            ok = k < 1 || mbar_wait(&p_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted);
+          for (int g = 0; ok && g < NG && k >= 1; ++g)
+            ok = mbar_wait(&p_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted) &&
+                 mbar_wait(&pv_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted);
           ok = ok && issue_s(k + 1);
         }
         if (ok) ok = mbar_wait(&vfull[k % VR], (k / VR) & 1, &aborted);
@@ -299,17 +293,15 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
           ok = mbar_wait(&p_bar[g][k & 1], (k >> 1) & 1, &aborted);
           if (!ok) break;
           tc::fence_after_sync();
-          const uint64_t pd =
-              pd0 + static_cast<uint64_t>(((g * PB + k % PB) * C::P_SET) >> 4);
+          // P of step k in tensor memory: the S buffer's columns 0-31 (and the
+          // bf16 residual in columns 32-63), 8 columns per 16-token k-step
+          const uint32_t t_p = tmem + g * kTmemGroup + (k & 1) * NT;
           const uint32_t t_o = tmem + g * kTmemGroup + kTmemO;
 #pragma unroll
           for (int kk = 0; kk < NT / 16; ++kk) {
             const uint64_t bv = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
-            tc::mma_f16(t_o, pd + static_cast<uint64_t>((kk * 32) >> 4), bv, C::IDESC_PV,
-                        k > 0 || kk > 0);
-            if constexpr (BF)
-              tc::mma_f16(t_o, pd + static_cast<uint64_t>((C::P_BYTES + kk * 32) >> 4), bv,
-                          C::IDESC_PV, true);
+            tc::mma_f16_ts(t_o, t_p + kk * 8, bv, C::IDESC_PV, k > 0 || kk > 0);
+            if constexpr (BF) tc::mma_f16_ts(t_o, t_p + 32 + kk * 8, bv, C::IDESC_PV, true);
           }
           tc::commit(&pv_bar[g][k & 1]);
         }
@@ -370,13 +362,8 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
         s8[i & 7] += x[i];
       }
       l = l * alpha + (((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7])));
-      // The P set of step k is free once O += P V of step k-PB completed; O may
-      // be rescaled only once O += P V of step k-1 completed (rare: the
+      // O may be rescaled only once O += P V of step k-1 completed (rare: the
       // maximum moves lazily), otherwise that MMA keeps running under this softmax
-      if (k >= PB) {
-        ok = mbar_wait(&pv_bar[g][(k - PB) & 1], ((k - PB) >> 1) & 1, &aborted);
-        if (!ok) break;
-      }
       if (k >= 1 && rescale) {
         ok = mbar_wait(&pv_bar[g][(k - 1) & 1], ((k - 1) >> 1) & 1, &aborted);
         if (!ok) break;
@@ -390,23 +377,22 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
           tc::st32(t_o + c * 32, o);
         }
       }
-      // P row (and for bf16 the residual P - bf16(P)) -> shared memory
-      uint8_t* psm = sp(g, k);
+      // P row (and for bf16 the residual P - bf16(P)) -> tensor memory, over the
+      // S it came from: columns 0-31 (pairs of 16-bit values), residual 32-63
+      {
+        uint32_t w[NT / 2], wl[NT / 2];
 #pragma unroll
-      for (int c = 0; c < NT / 8; ++c) {
-        uint32_t w[4], wl[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float p0 = x[c * 8 + 2 * i], p1 = x[c * 8 + 2 * i + 1];
+        for (int i = 0; i < NT / 2; ++i) {
+          const float p0 = x[2 * i], p1 = x[2 * i + 1];
           w[i] = pack_pair(BF, p0, p1);
           if constexpr (BF)
             wl[i] = pack2<true>(p0 - __uint_as_float(w[i] << 16),
                                 p1 - __uint_as_float(w[i] & 0xffff0000u));
         }
-        *reinterpret_cast<uint4*>(psm + sw128(rr, c)) = make_uint4(w[0], w[1], w[2], w[3]);
-        if constexpr (BF)
-          *reinterpret_cast<uint4*>(psm + C::P_BYTES + sw128(rr, c)) =
-              make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        const uint32_t t_p = t_grp + (k & 1) * NT + lane_base;
+        tc::st32u(t_p, w);
+        if constexpr (BF) tc::st32u(t_p + 32, wl);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
       // V rows without real data in this step (past the context, or tiles not
       // loaded) may hold anything, even NaN, and 0 * NaN is NaN inside the MMA;
