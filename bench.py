@@ -306,7 +306,8 @@ def prefill_oracle_sample(sp, qlens, budget_s):
         t0 = time.perf_counter()
         oracle.chunked_prefill(q, hd.key_cache, hd.value_cache, st.block_tables, sub.context_lens,
                                np.array([0, ql[0]], np.int32), scale=np.float32(sp.scale),
-                               q_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype)
+                               q_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype,
+                               k_scale=hd.k_scale, v_scale=hd.v_scale)
         t_total += time.perf_counter() - t0
         flops += wl.prefill_flops(sub, ql)
         done += 1
@@ -326,7 +327,8 @@ def run_prefill(args):
     config = {"workload": f"{sp.name}: {sp.num_seqs} seqs x {chunk} query tokens, ctx "
                           f"{int(sp.context_lens.min())}-{int(sp.context_lens.max())}, "
                           f"{sp.num_heads} q / {sp.num_kv_heads} kv heads, head_dim {sp.head_dim}, "
-                          f"block_size {sp.block_size}, {sp.q_dtype}"}
+                          f"block_size {sp.block_size}, {sp.q_dtype} query, "
+                          f"{sp.cache_dtype} cache"}
     # tensor-bound when the work per K/V byte is above the machine balance
     peak_t, kind_t = measured_tensor_peak()
     peak_b, kind_b = measured_peaks()
@@ -350,10 +352,12 @@ def run_prefill(args):
     out = torch.empty_like(q)
     ws = pk.chunked_prefill_workspace(sp.num_seqs, int(qlens.sum()), sp.num_heads,
                                       sp.num_kv_heads, sp.head_dim, chunk,
-                                      int(sp.context_lens.max()), device=dev)
+                                      int(sp.context_lens.max()),
+                                      pk.dtype_code(d["key_cache"]), device=dev)
     mctx = int(sp.context_lens.max())
     fn = lambda: pk.chunked_prefill(out, q, cu, chunk, d["key_cache"], d["value_cache"], bt, cl,
-                                    mctx, sp.scale, workspace=ws)
+                                    mctx, sp.scale, k_scale=d["k_scale"], v_scale=d["v_scale"],
+                                    workspace=ws)
     sampler = ClockSampler(0)
     sampler.start()
     ms = _time_device(fn, args.steps, max(3, args.warmup))

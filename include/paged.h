@@ -195,8 +195,11 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* query,
  * the cache (pa_reshape_and_cache). Row i attends to the tokens t <= p_i of
  * its sequence (the causal rule of autoregressive attention), query head h
  * to kv-head h / (num_heads / num_kv_heads), with softmax scale `scale`.
- * out, query      device [num_tokens, num_heads, head_dim] of `dtype`
- *                 (f16 or bf16; the cache has the same dtype).
+ * out, query      device [num_tokens, num_heads, head_dim] of q_dtype (f16 or bf16).
+ * cache_dtype     q_dtype, or PA_FP8_E4M3 with k_scale / v_scale (device float
+ *                 [num_kv_heads], as written by pa_reshape_and_cache; null otherwise):
+ *                 logits use scale * k_scale[kv-head], outputs are multiplied by
+ *                 v_scale[kv-head].
  * cu_query_lens   device int32 [num_seqs + 1], cu[0] = 0, cu[num_seqs] = num_tokens.
  * max_query_len   host int >= every q_len_s; sizes the launch.
  * key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens,
@@ -219,17 +222,20 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
                                     const int32_t* context_lens, int32_t max_context_len,
                                     int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                     int32_t head_dim, int32_t block_size, int64_t num_blocks,
-                                    float scale, pa_dtype dtype, void* workspace,
-                                    size_t workspace_bytes, pa_stream_t stream);
+                                    float scale, pa_dtype q_dtype, pa_dtype cache_dtype,
+                                    const float* k_scale, const float* v_scale,
+                                    void* workspace, size_t workspace_bytes,
+                                    pa_stream_t stream);
 
 /*
- * Bytes of workspace pa_chunked_prefill needs for these sizes on the current
- * device (256 when the key range is not split). Returns 0 for invalid sizes.
+ * Bytes of workspace pa_chunked_prefill needs for these sizes and cache dtype
+ * on the current device (256 when the key range is not split). Returns 0 for
+ * invalid sizes.
  */
 PA_API size_t pa_chunked_prefill_workspace_size(int32_t num_seqs, int32_t num_tokens,
                                                 int32_t num_heads, int32_t num_kv_heads,
                                                 int32_t head_dim, int32_t max_query_len,
-                                                int32_t max_context_len);
+                                                int32_t max_context_len, pa_dtype cache_dtype);
 
 /*
  * Bytes of workspace pa_decode needs for these sizes on the current device

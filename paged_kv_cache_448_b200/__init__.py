@@ -135,17 +135,22 @@ def _i32(a) -> np.ndarray:
 
 
 def chunked_prefill_workspace_size(num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
-                                   max_query_len, max_context_len) -> int:
+                                   max_query_len, max_context_len,
+                                   cache_dtype: int = _native.PA_F16) -> int:
+    """Bytes pa_chunked_prefill needs; cache_dtype is a pa_dtype code (an
+    E4M3 cache always takes the mma.sync kernel, which may split)."""
     return int(_native.lib().pa_chunked_prefill_workspace_size(
-        num_seqs, num_tokens, num_heads, num_kv_heads, head_dim, max_query_len, max_context_len))
+        num_seqs, num_tokens, num_heads, num_kv_heads, head_dim, max_query_len, max_context_len,
+        int(cache_dtype)))
 
 
 def chunked_prefill_workspace(num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
-                              max_query_len, max_context_len, device="cuda", stream=None):
+                              max_query_len, max_context_len, cache_dtype: int = _native.PA_F16,
+                              device="cuda", stream=None):
     """A device workspace for pa_chunked_prefill, error word zeroed."""
     import torch
     n = chunked_prefill_workspace_size(num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
-                                       max_query_len, max_context_len)
+                                       max_query_len, max_context_len, cache_dtype)
     ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
     check(_native.lib().pa_workspace_init(_ptr(ws), ws.numel(), _stream_handle(stream)))
     return ws
@@ -153,21 +158,24 @@ def chunked_prefill_workspace(num_seqs, num_tokens, num_heads, num_kv_heads, hea
 
 def chunked_prefill(out, query, cu_query_lens, max_query_len: int, key_cache, value_cache,
                     block_tables, context_lens, max_context_len: int, scale: float, *,
-                    workspace=None, stream=None):
+                    k_scale=None, v_scale=None, workspace=None, stream=None):
     """Several query tokens per sequence (its last positions), causal
-    (pa_chunked_prefill). out/query [T, H, D] f16|bf16 (cache of the same
-    dtype); cu_query_lens int32 [S+1]; context_lens include the query tokens."""
+    (pa_chunked_prefill). out/query [T, H, D] f16|bf16; caches of the query's
+    dtype, or E4M3 (uint8 / float8_e4m3fn) with k_scale / v_scale float32
+    [Hkv]; cu_query_lens int32 [S+1]; context_lens include the query tokens."""
     T, H, D = query.shape
     NB, BS, Hkv = key_cache.shape[:3]
     S = context_lens.shape[0]
     if workspace is None:
         workspace = chunked_prefill_workspace(S, T, H, Hkv, D, max_query_len, max_context_len,
-                                              device=query.device, stream=stream)
+                                              dtype_code(key_cache), device=query.device,
+                                              stream=stream)
     check(_native.lib().pa_chunked_prefill(
         _ptr(out), _ptr(query), _ptr(cu_query_lens), T, int(max_query_len), _ptr(key_cache),
         _ptr(value_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
         int(max_context_len), S, H, Hkv, D, BS, NB, float(scale), dtype_code(query),
-        _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+        dtype_code(key_cache), _ptr(k_scale), _ptr(v_scale), _ptr(workspace), workspace.numel(),
+        _stream_handle(stream)))
     return out
 
 

@@ -419,8 +419,11 @@ PA_API pa_status pa_copy_blocks(const void* src_key_cache, const void* src_value
 namespace paged {
 namespace {
 
-// Split of the key range for the multi-token query (mma.sync kernel only):
-// when its CTAs (query tiles x kv-heads x sequences) cannot fill about four
+// Kernel choice and split of the key range for the multi-token query.
+// Chunks that fill the 128 rows of a tensor-memory CTA (query tokens x heads
+// of a kv-head's group) run on tcgen05 (an E4M3 cache: head_dim 128 only);
+// shorter ones (a few draft tokens) on the 64-row mma.sync kernel. There,
+// when the CTAs (query tiles x kv-heads x sequences) cannot fill about four
 // waves of three CTAs per SM, the tiles of each CTA are cut into parts of at
 // least 256 tokens (16 tiles, a multiple of 4) handled by separate CTAs.
 struct PrefillPlan {
@@ -429,9 +432,10 @@ struct PrefillPlan {
 };
 
 PrefillPlan make_prefill_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t group,
-                              int32_t max_query_len, int32_t max_context_len) {
+                              int32_t head_dim, int32_t max_query_len, int32_t max_context_len,
+                              bool fp8) {
   PrefillPlan p{};
-  p.tc = static_cast<int64_t>(max_query_len) * group >= 128;
+  p.tc = (!fp8 || head_dim == 128) && static_cast<int64_t>(max_query_len) * group >= 128;
   p.q_tiles = (max_query_len + prefill_tokens_per_cta(group) - 1) / prefill_tokens_per_cta(group);
   const int32_t max_tiles = std::max<int32_t>(1, (max_context_len + 15) / 16);
   p.partition_tiles = max_tiles;
@@ -465,12 +469,14 @@ extern "C" {
 PA_API size_t pa_chunked_prefill_workspace_size(int32_t num_seqs, int32_t num_tokens,
                                                 int32_t num_heads, int32_t num_kv_heads,
                                                 int32_t head_dim, int32_t max_query_len,
-                                                int32_t max_context_len) {
+                                                int32_t max_context_len, pa_dtype cache_dtype) {
   if (num_seqs < 0 || num_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
-      max_query_len < 0 || max_context_len < 0 || num_heads % num_kv_heads != 0)
+      max_query_len < 0 || max_context_len < 0 || num_heads % num_kv_heads != 0 ||
+      (cache_dtype != PA_F16 && cache_dtype != PA_BF16 && cache_dtype != PA_FP8_E4M3))
     return 0;
   const PrefillPlan p = make_prefill_plan(num_seqs, num_kv_heads, num_heads / num_kv_heads,
-                                          max_query_len, max_context_len);
+                                          head_dim, max_query_len, max_context_len,
+                                          cache_dtype == PA_FP8_E4M3);
   return prefill_workspace_bytes(p, num_tokens, num_heads, head_dim);
 }
 
@@ -481,8 +487,10 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
                                     const int32_t* context_lens, int32_t max_context_len,
                                     int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                     int32_t head_dim, int32_t block_size, int64_t num_blocks,
-                                    float scale, pa_dtype dtype, void* workspace,
-                                    size_t workspace_bytes, pa_stream_t stream) {
+                                    float scale, pa_dtype q_dtype, pa_dtype cache_dtype,
+                                    const float* k_scale, const float* v_scale,
+                                    void* workspace, size_t workspace_bytes,
+                                    pa_stream_t stream) {
   clear_error();
   if (num_tokens < 0 || max_query_len < 0 || num_seqs < 0 || num_heads <= 0 ||
       num_kv_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || num_blocks <= 0)
@@ -495,8 +503,14 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
   if (!shape_supported(head_dim, block_size))
     return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: head_dim %d / block_size %d unsupported",
                 head_dim, block_size);
-  if (dtype != PA_F16 && dtype != PA_BF16)
-    return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: query and cache must be f16 or bf16");
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: query must be f16 or bf16");
+  if (cache_dtype != q_dtype && cache_dtype != PA_FP8_E4M3)
+    return fail(PA_ERR_UNSUPPORTED,
+                "chunked_prefill: cache dtype must equal query dtype or be e4m3");
+  const bool fp8 = cache_dtype == PA_FP8_E4M3;
+  if (fp8 != (k_scale != nullptr) || fp8 != (v_scale != nullptr))
+    return fail(PA_ERR_INVALID_ARG, "chunked_prefill: k_scale/v_scale required exactly for e4m3");
   if (num_blocks * block_size > INT32_MAX)
     return fail(PA_ERR_UNSUPPORTED, "chunked_prefill: pool rows exceed 2^31");
   if (num_seqs > 65535 || num_kv_heads > 65535)
@@ -510,25 +524,25 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
     return fail(PA_ERR_INVALID_ARG, "chunked_prefill: null pointer");
   if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) ||
       !aligned(value_cache, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4) ||
-      !aligned(cu_query_lens, 4))
+      !aligned(cu_query_lens, 4) || (k_scale && !aligned(k_scale, 4)) ||
+      (v_scale && !aligned(v_scale, 4)))
     return fail(PA_ERR_INVALID_ARG, "chunked_prefill: misaligned pointer");
 
   CUtensorMap kmap, vmap;
-  // Chunks that fill the 128 rows of a tensor-memory CTA (query tokens x heads
-  // of a kv-head's group) run on tcgen05; shorter ones (a few draft tokens)
-  // on the 64-row mma.sync kernel, which wastes fewer rows.
   const PrefillPlan plan =
-      make_prefill_plan(num_seqs, num_kv_heads, group, max_query_len, max_context_len);
+      make_prefill_plan(num_seqs, num_kv_heads, group, head_dim, max_query_len,
+                        max_context_len, fp8);
   const bool tc = plan.tc;
   const size_t need = prefill_workspace_bytes(plan, num_tokens, num_heads, head_dim);
   if (workspace_bytes < need)
     return fail(PA_ERR_INVALID_ARG, "chunked_prefill: workspace %zu bytes < %zu needed",
                 workspace_bytes, need);
+  const int elem = elem_bytes(cache_dtype);
   pa_status st = encode_cache_map(&kmap, key_cache, num_blocks, block_size, num_kv_heads,
-                                  head_dim, 2, tc);
+                                  head_dim, elem, tc);
   if (st == PA_OK)
-    st = encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim, 2,
-                          tc);
+    st = encode_cache_map(&vmap, value_cache, num_blocks, block_size, num_kv_heads, head_dim,
+                          elem, tc);
   if (st != PA_OK) return st;
   PrefillArgs a{};
   a.out = out;
@@ -536,6 +550,8 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
   a.cu_query_lens = cu_query_lens;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   a.err = reinterpret_cast<int32_t*>(workspace) + kWordError;
   a.diag = reinterpret_cast<int32_t*>(workspace) + kWordDiag;
   a.num_blocks = num_blocks;
@@ -556,10 +572,13 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
     a.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                       align256(kHeaderBytes + rows * sizeof(float2)));
   }
-  auto launch = tc ? launch_prefill_tc : launch_prefill;
-  return cuda_status(launch(a, kmap, vmap, dtype == PA_F16 ? kF16 : kBF16, head_dim, group,
-                            max_query_len, reinterpret_cast<cudaStream_t>(stream)),
-                     "chunked_prefill");
+  const int qd = q_dtype == PA_F16 ? kF16 : kBF16;
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int cd = fp8 ? kE4M3 : qd;
+  const cudaError_t e =
+      tc ? launch_prefill_tc(a, kmap, vmap, qd, cd, head_dim, group, max_query_len, cs)
+         : launch_prefill(a, kmap, vmap, qd, cd, head_dim, group, max_query_len, cs);
+  return cuda_status(e, "chunked_prefill");
 }
 
 }  // extern "C"

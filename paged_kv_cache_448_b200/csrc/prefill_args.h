@@ -13,6 +13,8 @@ struct PrefillArgs {
   const int32_t* cu_query_lens;  // [S + 1]: rows of sequence s are cu[s] .. cu[s+1]-1
   const int32_t* block_tables;   // [S, max_blocks_per_seq]
   const int32_t* context_lens;   // [S], including the query tokens
+  const float* k_scale;          // [Hkv] (E4M3 cache) or null
+  const float* v_scale;
   int32_t* err;                  // error word
   int32_t* diag;                 // failure record
   int64_t num_blocks;
@@ -37,18 +39,20 @@ enum : int32_t { kSitePrefill = 5 };
 // Query tokens per CTA of the mma.sync kernel (64 rows = tokens x group).
 __host__ __device__ constexpr int prefill_tokens_per_cta(int group) { return 64 / group; }
 
-// mma.sync kernel for one (q dtype == cache dtype) pair: grid of
+// mma.sync kernel for one (q dtype, cache dtype) pair: grid of
 // a.q_tiles * a.max_parts CTAs per (sequence, kv-head), then, when the key
 // range is split (a.max_parts > 1), the combine kernel. cudaErrorNotSupported
 // for shapes without a kernel.
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                           int q_dtype, int head_dim, int group, int32_t max_query_len,
-                           cudaStream_t stream);
+                           int q_dtype, int cache_dtype, int head_dim, int group,
+                           int32_t max_query_len, cudaStream_t stream);
 
 // The same on the 5th-generation tensor cores (tcgen05, tensor memory); the
 // tensor maps are the one-segment boxes of encode_cache_map(..., 1 segment).
+// An E4M3 cache needs head_dim 128.
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& kmap,
-                              const CUtensorMap& vmap, int q_dtype, int head_dim, int group,
-                              int32_t max_query_len, cudaStream_t stream);
+                              const CUtensorMap& vmap, int q_dtype, int cache_dtype,
+                              int head_dim, int group, int32_t max_query_len,
+                              cudaStream_t stream);
 
 }  // namespace paged

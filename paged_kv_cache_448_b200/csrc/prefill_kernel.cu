@@ -62,12 +62,21 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
   }
 }
 
-template <class QF, int D, int G>
+// QF: query / output type; CF: cache type (QF, or E4M3). An E4M3 cache is
+// widened exactly to f16 in registers (every E4M3 value is an f16 value) as
+// in the decode kernel's tensor-core consumer: K with the k order inside each
+// 16-wide MMA step permuted to match 4-byte ldmatrix rows (the query uses the
+// same permutation), V split into even / odd dimensions by byte permutes; the
+// query goes to f16 scaled by a power of two (undone in the logit scale with
+// the kv-head's K scale), the V scale applies to the output.
+template <class QF, class CF, int D, int G>
 __global__ void __launch_bounds__(kPrefillWarps * 32)
     paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap) {
-  using T = Tile<QF, D>;
-  constexpr bool BF = std::is_same<QF, BF16>::value;
+  using T = Tile<CF, D>;
+  constexpr bool FP8 = CF::kBytes == 1;
+  constexpr bool QBF = std::is_same<QF, BF16>::value;
+  constexpr bool BF = QBF && !FP8;   // MMA operand type: bf16 (16-bit bf16 cache) or f16
   constexpr int R = kPrefillStages, NW = kPrefillWarps, TR = kTileRows;
   constexpr int QT = kPrefillRows / G;  // query tokens per CTA
   constexpr int KS = D / 16, NO = D / 8;
@@ -176,7 +185,8 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
 
   // Q fragments (A operand, rows r_lo / r_hi, k-steps of 16 dims)
   uint32_t qa[KS][4];
-  {
+  float qscale = a.scale_log2;
+  if constexpr (!FP8) {
     const uint32_t* q32 = static_cast<const uint32_t*>(a.query);
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
@@ -185,12 +195,39 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
       qa[kk][2] = v_lo ? q32[(row_lo + kk * 16 + 8 + 2 * c) / 2] : 0u;
       qa[kk][3] = v_hi ? q32[(row_hi + kk * 16 + 8 + 2 * c) / 2] : 0u;
     }
+  } else {
+    // permuted k order: k 2c, 2c+1 <-> dims 4c, 4c+1; k 2c+8, 2c+9 <-> dims 4c+2, 4c+3
+    float qv[KS][2][4];
+    float mq = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        qv[kk][0][j] = v_lo ? load_in(QF{}, a.query, row_lo + 16 * kk + 4 * c + j) : 0.f;
+        qv[kk][1][j] = v_hi ? load_in(QF{}, a.query, row_hi + 16 * kk + 4 * c + j) : 0.f;
+        mq = fmaxf(mq, fmaxf(fabsf(qv[kk][0][j]), fabsf(qv[kk][1][j])));
+      }
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) mq = fmaxf(mq, __shfl_xor_sync(FULL, mq, o2));
+    int e = 0;
+    if (mq > 0.f && isfinite(mq)) {
+      int k2;
+      frexpf(mq, &k2);                      // mq < 2^k2
+      e = min(max(15 - k2, -100), 100);     // mq * 2^e < 2^15
+    }
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      qa[kk][0] = pack2<false>(ldexpf(qv[kk][0][0], e), ldexpf(qv[kk][0][1], e));
+      qa[kk][1] = pack2<false>(ldexpf(qv[kk][1][0], e), ldexpf(qv[kk][1][1], e));
+      qa[kk][2] = pack2<false>(ldexpf(qv[kk][0][2], e), ldexpf(qv[kk][0][3], e));
+      qa[kk][3] = pack2<false>(ldexpf(qv[kk][1][2], e), ldexpf(qv[kk][1][3], e));
+    }
+    qscale *= a.k_scale[kvh] * ldexpf(1.f, -e);
   }
   float o[NO][4];
 #pragma unroll
   for (int j = 0; j < NO; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   float m_lo = -CUDART_INF_F, m_hi = -CUDART_INF_F, l_lo = 0.f, l_hi = 0.f;
-  const float qscale = a.scale_log2;
 
   int k = 0, t = 0;  // step, and the first tile not yet received
   bool failed = false;
@@ -232,12 +269,25 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const int row = nt * 8 + (lane & 7);
+        if constexpr (!FP8) {
 #pragma unroll
-        for (int kk = 0; kk < KS; kk += 2) {
-          uint32_t b[4];
-          ldsm_x4(kt + T::off(row, (2 * kk + (lane >> 3)) * 16), b);
-          mma_16816<BF>(sacc[j][nt], qa[kk], b[0], b[1]);
-          mma_16816<BF>(s2[nt], qa[kk + 1], b[2], b[3]);
+          for (int kk = 0; kk < KS; kk += 2) {
+            uint32_t b[4];
+            ldsm_x4(kt + T::off(row, (2 * kk + (lane >> 3)) * 16), b);
+            mma_16816<BF>(sacc[j][nt], qa[kk], b[0], b[1]);
+            mma_16816<BF>(s2[nt], qa[kk + 1], b[2], b[3]);
+          }
+        } else {
+          // 16 E4M3 dims per 16-byte chunk: one ldmatrix x4 covers 4 k-steps
+#pragma unroll
+          for (int kk = 0; kk < KS; kk += 4) {
+            uint32_t b[4];
+            ldsm_x4(kt + T::off(row, (kk + (lane >> 3)) * 16), b);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              mma_16816<false>((q & 1) ? s2[nt] : sacc[j][nt], qa[kk + q],
+                               e4m3x2_to_f16x2(b[q]), e4m3x2_to_f16x2(b[q] >> 16));
+          }
         }
       }
 #pragma unroll
@@ -330,15 +380,34 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
         }
       }
       const int vrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+      if constexpr (!FP8) {
 #pragma unroll
-      for (int dn = 0; dn < NO; dn += 2) {
-        uint32_t b[4];
-        ldsm_x4_trans(vt + T::off(vrow, (dn + (lane >> 4)) * 16), b);
-        mma_16816<BF>(o[dn], pa, b[0], b[1]);
-        mma_16816<BF>(o[dn + 1], pa, b[2], b[3]);
-        if constexpr (BF) {
-          mma_16816<BF>(o[dn], pl, b[0], b[1]);
-          mma_16816<BF>(o[dn + 1], pl, b[2], b[3]);
+        for (int dn = 0; dn < NO; dn += 2) {
+          uint32_t b[4];
+          ldsm_x4_trans(vt + T::off(vrow, (dn + (lane >> 4)) * 16), b);
+          mma_16816<BF>(o[dn], pa, b[0], b[1]);
+          mma_16816<BF>(o[dn + 1], pa, b[2], b[3]);
+          if constexpr (BF) {
+            mma_16816<BF>(o[dn], pl, b[0], b[1]);
+            mma_16816<BF>(o[dn + 1], pl, b[2], b[3]);
+          }
+        }
+      } else {
+        // ldmatrix.trans gives byte pairs of two tokens x two dims: a byte
+        // permute splits them into an even-dim and an odd-dim n-tile
+#pragma unroll
+        for (int q = 0; q < D / 16; q += 2) {
+          uint32_t b[4];
+          ldsm_x4_trans(vt + T::off(vrow, (q + (lane >> 4)) * 16), b);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t lo = b[2 * h], hi = b[2 * h + 1];
+            mma_16816<false>(o[2 * (q + h)], pa, e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0020)),
+                             e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0020)));
+            mma_16816<false>(o[2 * (q + h) + 1], pa,
+                             e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0031)),
+                             e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0031)));
+          }
         }
       }
       __syncwarp();
@@ -367,13 +436,34 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
   l_lo += __shfl_xor_sync(FULL, l_lo, 2);
   l_hi += __shfl_xor_sync(FULL, l_hi, 1);
   l_hi += __shfl_xor_sync(FULL, l_hi, 2);
-  const float i_lo = l_lo > 0.f ? 1.f / l_lo : 0.f, i_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
+  float i_lo = l_lo > 0.f ? 1.f / l_lo : 0.f, i_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
+  if constexpr (FP8) {
+    const float vs = a.v_scale[kvh];
+    i_lo *= vs;
+    i_hi *= vs;
+  }
+  // pairs of adjacent output dims d, d+1 and their accumulators: 16-bit cache
+  // columns 8j + 2c (+1) of n-tile j; E4M3 dims 16m + 4c + 2i (+1) of the
+  // even / odd n-tiles 2m, 2m+1
+  auto pair_dim = [&](int pi) { return FP8 ? 16 * (pi / 2) + 4 * c + 2 * (pi % 2) : 8 * pi + 2 * c; };
+  auto pair_val = [&](int pi, int hi, float& x, float& y) {
+    if constexpr (FP8) {
+      x = o[2 * (pi / 2)][2 * hi + pi % 2];
+      y = o[2 * (pi / 2) + 1][2 * hi + pi % 2];
+    } else {
+      x = o[pi][2 * hi];
+      y = o[pi][2 * hi + 1];
+    }
+  };
   if (parts == 1) {
     uint32_t* out32 = static_cast<uint32_t*>(a.out);
 #pragma unroll
-    for (int j = 0; j < NO; ++j) {
-      if (v_lo) out32[(row_lo + j * 8 + 2 * c) / 2] = pack2<BF>(o[j][0] * i_lo, o[j][1] * i_lo);
-      if (v_hi) out32[(row_hi + j * 8 + 2 * c) / 2] = pack2<BF>(o[j][2] * i_hi, o[j][3] * i_hi);
+    for (int pi = 0; pi < NO; ++pi) {
+      float x, y;
+      pair_val(pi, 0, x, y);
+      if (v_lo) out32[(row_lo + pair_dim(pi)) / 2] = pack2<QBF>(x * i_lo, y * i_lo);
+      pair_val(pi, 1, x, y);
+      if (v_hi) out32[(row_hi + pair_dim(pi)) / 2] = pack2<QBF>(x * i_hi, y * i_hi);
     }
     return;
   }
@@ -384,13 +474,14 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
   if (v_lo && c == 0) a.ws_ml[pl] = make_float2(m_lo, l_lo);
   if (v_hi && c == 0) a.ws_ml[ph] = make_float2(m_hi, l_hi);
 #pragma unroll
-  for (int j = 0; j < NO; ++j) {
+  for (int pi = 0; pi < NO; ++pi) {
+    float x, y;
+    pair_val(pi, 0, x, y);
     if (v_lo)
-      *reinterpret_cast<float2*>(a.ws_o + pl * D + j * 8 + 2 * c) =
-          make_float2(o[j][0] * i_lo, o[j][1] * i_lo);
+      *reinterpret_cast<float2*>(a.ws_o + pl * D + pair_dim(pi)) = make_float2(x * i_lo, y * i_lo);
+    pair_val(pi, 1, x, y);
     if (v_hi)
-      *reinterpret_cast<float2*>(a.ws_o + ph * D + j * 8 + 2 * c) =
-          make_float2(o[j][2] * i_hi, o[j][3] * i_hi);
+      *reinterpret_cast<float2*>(a.ws_o + ph * D + pair_dim(pi)) = make_float2(x * i_hi, y * i_hi);
   }
 }
 
@@ -439,13 +530,13 @@ __global__ void __launch_bounds__(128) paged_prefill_combine(const PrefillArgs a
   for (int j = 0; j < PER; ++j) store_out(QF{}, a.out, row * D + lane + 32 * j, acc[j] * inv);
 }
 
-template <class QF, int D, int G>
+template <class QF, class CF, int D, int G>
 cudaError_t launch_one(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                        int32_t max_query_len, cudaStream_t stream) {
   constexpr int QT = kPrefillRows / G;
-  constexpr int STAGE = 2 * Tile<QF, D>::BYTES;
+  constexpr int STAGE = 2 * Tile<CF, D>::BYTES;
   const size_t smem = 1024 + kPrefillStages * STAGE + 16 * kPrefillStages;
-  auto kern = paged_prefill_kernel<QF, D, G>;
+  auto kern = paged_prefill_kernel<QF, CF, D, G>;
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   static_assert(QT == prefill_tokens_per_cta(G), "tokens per CTA");
@@ -461,18 +552,28 @@ cudaError_t launch_one(const PrefillArgs& a, const CUtensorMap& kmap, const CUte
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                           int q_dtype, int head_dim, int group, int32_t max_query_len,
-                           cudaStream_t stream) {
-#define PAGED_PREFILL(QF, d, g) \
-  if (head_dim == d && group == g) return launch_one<QF, d, g>(a, kmap, vmap, max_query_len, stream);
-#define PAGED_PREFILL_ALL(QF)                                                   \
-  PAGED_PREFILL(QF, 64, 1) PAGED_PREFILL(QF, 64, 2) PAGED_PREFILL(QF, 64, 4)     \
-  PAGED_PREFILL(QF, 64, 8) PAGED_PREFILL(QF, 128, 1) PAGED_PREFILL(QF, 128, 2)   \
-  PAGED_PREFILL(QF, 128, 4) PAGED_PREFILL(QF, 128, 8)
+                           int q_dtype, int cache_dtype, int head_dim, int group,
+                           int32_t max_query_len, cudaStream_t stream) {
+#define PAGED_PREFILL(QF, CF, d, g) \
+  if (head_dim == d && group == g)  \
+    return launch_one<QF, CF, d, g>(a, kmap, vmap, max_query_len, stream);
+#define PAGED_PREFILL_ALL(QF, CF)                                                           \
+  PAGED_PREFILL(QF, CF, 64, 1) PAGED_PREFILL(QF, CF, 64, 2) PAGED_PREFILL(QF, CF, 64, 4)     \
+  PAGED_PREFILL(QF, CF, 64, 8) PAGED_PREFILL(QF, CF, 128, 1) PAGED_PREFILL(QF, CF, 128, 2)   \
+  PAGED_PREFILL(QF, CF, 128, 4) PAGED_PREFILL(QF, CF, 128, 8)
+  const bool fp8 = cache_dtype == kE4M3;
   if (q_dtype == kF16) {
-    PAGED_PREFILL_ALL(F16)
+    if (fp8) {
+      PAGED_PREFILL_ALL(F16, E4M3)
+    } else {
+      PAGED_PREFILL_ALL(F16, F16)
+    }
   } else if (q_dtype == kBF16) {
-    PAGED_PREFILL_ALL(BF16)
+    if (fp8) {
+      PAGED_PREFILL_ALL(BF16, E4M3)
+    } else {
+      PAGED_PREFILL_ALL(BF16, BF16)
+    }
   }
 #undef PAGED_PREFILL_ALL
 #undef PAGED_PREFILL

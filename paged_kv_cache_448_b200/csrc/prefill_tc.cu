@@ -20,6 +20,13 @@
 //    issues O += P V (M=128, N=D, K=64; V read MN-major), accumulating in
 //    tensor memory, then refills the stage once those MMAs completed;
 //  * the epilogue divides each row of O by its sum and stores it.
+// An E4M3 cache (head_dim 128: a 128-byte row) runs on kind::f8f6f4 with the
+// cache tiles as they arrive: Q goes to shared memory as E4M3 hi + lo parts
+// (q * 2^e = hi + lo, e a power of two per row that puts max |q| below 2^8,
+// undone in the row's logit scale with the kv-head's K scale), so S takes two
+// 8-bit MMAs per K step; P (<= 2^8 under the lazy maximum) goes to tensor
+// memory as an E4M3 hi part and an E5M2 residual, so O += P V takes two
+// 8-bit MMAs with V read MN-major; the V scale applies in the epilogue.
 // Every wait is bounded by wall time; a wait that gives up is agreed on by the
 // whole CTA at the next barrier, which then drains its loads and MMAs, frees
 // its tensor memory and reports.
@@ -46,13 +53,17 @@ constexpr int kSiteTc = 6;
 
 // NG row groups of 128 rows share each K/V step (NG = 2: 256 rows, eight
 // softmax warps, and two independent MMA streams per step).
-template <class QF, int D, int G, int NG>
+template <class QF, class CF, int D, int G, int NG>
 struct TcCfg {
+  static constexpr bool FP8 = CF::kBytes == 1;
   static constexpr bool BF = std::is_same<QF, BF16>::value;
-  static constexpr int NSEG = D * 2 / 128;          // 128-byte segments of a row
+  static constexpr int NSEG = D * CF::kBytes / 128;  // 128-byte segments of a cache row
+  static_assert(NSEG >= 1, "rows of at least 128 bytes");
   static constexpr int ROWS = NG * kTcRows;
   static constexpr int QT = ROWS / G;               // query tokens per CTA
-  static constexpr int QG_BYTES = NSEG * kTcRows * 128;  // Q of one group
+  // Q of one group: NSEG segments (16-bit), or the E4M3 hi and lo parts
+  static constexpr int QPART = kTcRows * 128;
+  static constexpr int QG_BYTES = (FP8 ? 2 : NSEG) * QPART;
   static constexpr int KV_SEG = kTcNT * 128;        // one segment of K or V in a stage
   static constexpr int KV_BYTES = NSEG * KV_SEG;    // one stage of K (or V)
   // ring depths (K, needed first by S, and V)
@@ -61,8 +72,11 @@ struct TcCfg {
   static constexpr int OFF_V = OFF_K + KR * KV_BYTES;           // V ring
   static constexpr int BYTES = OFF_V + VR * KV_BYTES;
   static constexpr uint32_t TMEM_COLS = NG * kTmemGroup;
-  static constexpr uint32_t IDESC_S = tc::idesc_f16<BF, kTcRows, kTcNT, false>();
-  static constexpr uint32_t IDESC_PV = tc::idesc_f16<BF, kTcRows, D, true>();
+  static constexpr uint32_t IDESC_S = FP8 ? tc::idesc_f8<0, 0, kTcRows, kTcNT, false>()
+                                           : tc::idesc_f16<BF, kTcRows, kTcNT, false>();
+  static constexpr uint32_t IDESC_PV = FP8 ? tc::idesc_f8<0, 0, kTcRows, D, true>()
+                                            : tc::idesc_f16<BF, kTcRows, D, true>();
+  static constexpr uint32_t IDESC_PV_LO = tc::idesc_f8<1, 0, kTcRows, D, true>();  // E5M2 P
   static_assert(kTcNT == 64, "P (64 16-bit values) fills half of its S buffer's columns");
   static_assert(BYTES + 1024 <= 227 * 1024, "shared memory of one CTA");
 };
@@ -76,13 +90,47 @@ __device__ __forceinline__ uint32_t pack_pair(bool bf, float lo, float hi) {
   return bf ? pack2<true>(lo, hi) : pack2<false>(lo, hi);
 }
 
+// Two 16-bit query values (low half first) as floats.
+template <class QF>
+__device__ __forceinline__ float2 unpack_q(uint32_t w) {
+  if constexpr (std::is_same<QF, BF16>::value)
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  const __half2 h = *reinterpret_cast<const __half2*>(&w);
+  return __half22float2(h);
+}
 
-template <class QF, int D, int G, int NG>
+// Four values -> E4M3 hi parts and 8-bit residuals (E4M3 or E5M2), four bytes
+// each in order. The values go through f16 (exact for the inputs here: bf16 /
+// f16 queries times a power of two, probabilities of at most 2^8); the
+// residual h - hi is exact in f16.
+template <bool LO_E5M2>
+__device__ __forceinline__ void split_fp8x4(float a, float b, float c, float d, uint32_t& hi,
+                                            uint32_t& lo) {
+  const __half2 h01 = __floats2half2_rn(a, b), h23 = __floats2half2_rn(c, d);
+  const __nv_fp8x2_storage_t hi01 = __nv_cvt_halfraw2_to_fp8x2(
+      *reinterpret_cast<const __half2_raw*>(&h01), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi23 = __nv_cvt_halfraw2_to_fp8x2(
+      *reinterpret_cast<const __half2_raw*>(&h23), __NV_SATFINITE, __NV_E4M3);
+  const __half2_raw b01 = __nv_cvt_fp8x2_to_halfraw2(hi01, __NV_E4M3);
+  const __half2_raw b23 = __nv_cvt_fp8x2_to_halfraw2(hi23, __NV_E4M3);
+  const __half2 r01 = __hsub2(h01, *reinterpret_cast<const __half2*>(&b01));
+  const __half2 r23 = __hsub2(h23, *reinterpret_cast<const __half2*>(&b23));
+  constexpr __nv_fp8_interpretation_t LO = LO_E5M2 ? __NV_E5M2 : __NV_E4M3;
+  const __nv_fp8x2_storage_t lo01 =
+      __nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r01), __NV_SATFINITE, LO);
+  const __nv_fp8x2_storage_t lo23 =
+      __nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r23), __NV_SATFINITE, LO);
+  hi = static_cast<uint32_t>(hi01) | (static_cast<uint32_t>(hi23) << 16);
+  lo = static_cast<uint32_t>(lo01) | (static_cast<uint32_t>(lo23) << 16);
+}
+
+
+template <class QF, class CF, int D, int G, int NG>
 __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
     paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap kmap,
                             const __grid_constant__ CUtensorMap vmap) {
-  using C = TcCfg<QF, D, G, NG>;
-  constexpr bool BF = C::BF;
+  using C = TcCfg<QF, CF, D, G, NG>;
+  constexpr bool BF = C::BF, FP8 = C::FP8;
   constexpr int NSEG = C::NSEG, QT = C::QT, KR = C::KR, VR = C::VR, NT = kTcNT, TR = kTileRows;
   constexpr int kMma = NG * kTcRows / 32;   // warp issuing the MMAs (owns the tensor memory)
   constexpr int kLoader = kMma + 1;         // warp issuing the TMA loads
@@ -157,18 +205,60 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
 
   __syncthreads();  // barrier initialisation visible to every thread
   if (warp == kMma) tc::alloc(&tmem_slot, C::TMEM_COLS);
+  float qscale = a.scale_log2;  // logit scale of this thread's row (base 2)
   if (warp < kMma) {
     // Q rows -> shared memory (per group, 128-byte swizzle, K-major), zeros past the chunk
     const int g = tid / kTcRows, rr = tid % kTcRows;
     const uint4* q4 = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.query) +
                                                      row_off * 2);
+    if constexpr (!FP8) {
 #pragma unroll
-    for (int sg = 0; sg < NSEG; ++sg)
+      for (int sg = 0; sg < NSEG; ++sg)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = valid ? q4[sg * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(sq(g) + sg * (kTcRows * 128) + sw128(rr, c)) = v;
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = valid ? q4[sg * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(sq(g) + sg * C::QPART + sw128(rr, c)) = v;
+        }
+    } else {
+      // row maximum, then q * 2^e = hi + lo (E4M3 each), 16 dims per 16-byte chunk
+      float mq = 0.f;
+      if (valid) {
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 v = q4[c];
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = unpack_q<QF>(w[j]);
+            mq = fmaxf(mq, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        }
       }
+      int e = 0;
+      if (mq > 0.f && isfinite(mq)) {
+        int k2;
+        frexpf(mq, &k2);                  // mq < 2^k2
+        e = min(max(8 - k2, -100), 100);  // mq * 2^e < 2^8
+      }
+      qscale *= a.k_scale[kvh] * ldexpf(1.f, -e);
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
+        if (valid) {
+          const uint4 v0 = q4[2 * c], v1 = q4[2 * c + 1];
+          const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f0 = unpack_q<QF>(w[2 * j]), f1 = unpack_q<QF>(w[2 * j + 1]);
+            split_fp8x4<false>(ldexpf(f0.x, e), ldexpf(f0.y, e), ldexpf(f1.x, e),
+                               ldexpf(f1.y, e), hw[j], lw[j]);
+          }
+        }
+        *reinterpret_cast<uint4*>(sq(g) + sw128(rr, c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(sq(g) + C::QPART + sw128(rr, c)) =
+            make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    }
     fence_proxy_async_smem();
   }
   tc::fence_before_sync();
@@ -262,13 +352,24 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
         const uint64_t kd = kd0 + static_cast<uint64_t>(((k % KR) * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
+          if constexpr (!FP8) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int sg = kk / 4, off = (kk % 4) * 32;
-            tc::mma_f16(tmem + g * kTmemGroup + (k & 1) * NT,
-                        qd[g] + static_cast<uint64_t>((sg * (kTcRows * 128) + off) >> 4),
-                        kd + static_cast<uint64_t>((sg * C::KV_SEG + off) >> 4), C::IDESC_S,
-                        kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int sg = kk / 4, off = (kk % 4) * 32;
+              tc::mma_f16(tmem + g * kTmemGroup + (k & 1) * NT,
+                          qd[g] + static_cast<uint64_t>((sg * C::QPART + off) >> 4),
+                          kd + static_cast<uint64_t>((sg * C::KV_SEG + off) >> 4), C::IDESC_S,
+                          kk > 0);
+            }
+          } else {
+            // Q hi, then Q lo, each 4 K steps of 32 dims (32 bytes) along the row
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const int part = kk / 4, off = (kk % 4) * 32;
+              tc::mma_f8(tmem + g * kTmemGroup + (k & 1) * NT,
+                         qd[g] + static_cast<uint64_t>((part * C::QPART + off) >> 4),
+                         kd + static_cast<uint64_t>(off >> 4), C::IDESC_S, kk > 0);
+            }
           }
           tc::commit(&s_bar[g][k & 1]);
         }
@@ -297,11 +398,21 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
           // bf16 residual in columns 32-63), 8 columns per 16-token k-step
           const uint32_t t_p = tmem + g * kTmemGroup + (k & 1) * NT;
           const uint32_t t_o = tmem + g * kTmemGroup + kTmemO;
+          if constexpr (!FP8) {
 #pragma unroll
-          for (int kk = 0; kk < NT / 16; ++kk) {
-            const uint64_t bv = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
-            tc::mma_f16_ts(t_o, t_p + kk * 8, bv, C::IDESC_PV, k > 0 || kk > 0);
-            if constexpr (BF) tc::mma_f16_ts(t_o, t_p + 32 + kk * 8, bv, C::IDESC_PV, true);
+            for (int kk = 0; kk < NT / 16; ++kk) {
+              const uint64_t bv = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
+              tc::mma_f16_ts(t_o, t_p + kk * 8, bv, C::IDESC_PV, k > 0 || kk > 0);
+              if constexpr (BF) tc::mma_f16_ts(t_o, t_p + 32 + kk * 8, bv, C::IDESC_PV, true);
+            }
+          } else {
+            // E4M3 P in columns 0-15, its E5M2 residual in 16-31; 32 tokens per K step
+#pragma unroll
+            for (int kk = 0; kk < NT / 32; ++kk) {
+              const uint64_t bv = vd + static_cast<uint64_t>((kk * 32 * 128) >> 4);
+              tc::mma_f8_ts(t_o, t_p + kk * 8, bv, C::IDESC_PV, k > 0 || kk > 0);
+              tc::mma_f8_ts(t_o, t_p + 16 + kk * 8, bv, C::IDESC_PV_LO, true);
+            }
           }
           tc::commit(&pv_bar[g][k & 1]);
         }
@@ -327,7 +438,6 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
     const int rr = tid % kTcRows;                // row within the group = tensor-memory lane
     const int p_row = valid ? pos0 + tok : -1;
     const int kv_valid = min(ctx, ntiles * TR);  // tokens with loaded, real rows
-    const float qscale = a.scale_log2;
     float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int k = 0; ok && k < nsteps; ++k) {
@@ -379,7 +489,16 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       }
       // P row (and for bf16 the residual P - bf16(P)) -> tensor memory, over the
       // S it came from: columns 0-31 (pairs of 16-bit values), residual 32-63
-      {
+      if constexpr (FP8) {
+        uint32_t w[NT / 4], wl[NT / 4];
+#pragma unroll
+        for (int i = 0; i < NT / 4; ++i)
+          split_fp8x4<true>(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3], w[i], wl[i]);
+        const uint32_t t_p = t_grp + (k & 1) * NT + lane_base;
+        tc::st16u(t_p, w);
+        tc::st16u(t_p + 16, wl);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      } else {
         uint32_t w[NT / 2], wl[NT / 2];
 #pragma unroll
         for (int i = 0; i < NT / 2; ++i) {
@@ -420,7 +539,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
     } else {
       // ---- epilogue: out = O / l, rounded to the q dtype
       tc::fence_after_sync();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = (l > 0.f ? 1.f / l : 0.f) * (FP8 ? a.v_scale[kvh] : 1.f);
       uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -445,14 +564,14 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   }
 }
 
-template <class QF, int D, int G, int NG>
+template <class QF, class CF, int D, int G, int NG>
 cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                       int32_t max_query_len, cudaStream_t stream) {
-  using C = TcCfg<QF, D, G, NG>;
+  using C = TcCfg<QF, CF, D, G, NG>;
   // shared memory keeps the tensor memory of the CTAs on one SM within 512
   // columns: one CTA of two groups, or at most two CTAs of one (>= 80 KB each)
   const size_t smem = std::max<size_t>(1024 + C::BYTES, NG == 2 ? 120 * 1024 : 80 * 1024);
-  auto kern = paged_prefill_tc_kernel<QF, D, G, NG>;
+  auto kern = paged_prefill_tc_kernel<QF, CF, D, G, NG>;
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const unsigned tiles = static_cast<unsigned>((max_query_len + C::QT - 1) / C::QT);
@@ -463,22 +582,37 @@ cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUten
 }  // namespace
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& kmap,
-                              const CUtensorMap& vmap, int q_dtype, int head_dim, int group,
-                              int32_t max_query_len, cudaStream_t stream) {
+                              const CUtensorMap& vmap, int q_dtype, int cache_dtype,
+                              int head_dim, int group, int32_t max_query_len,
+                              cudaStream_t stream) {
   // two row groups (256 rows) when the chunks fill them
   const bool two = static_cast<int64_t>(max_query_len) * group >= 2 * kTcRows;
-#define PAGED_TC(QF, d, g)                                                              \
+#define PAGED_TC(QF, CF, d, g)                                                          \
   if (head_dim == d && group == g)                                                      \
-    return two ? launch_tc<QF, d, g, 2>(a, kmap, vmap, max_query_len, stream)          \
-               : launch_tc<QF, d, g, 1>(a, kmap, vmap, max_query_len, stream);
-#define PAGED_TC_ALL(QF)                                                  \
-  PAGED_TC(QF, 64, 1) PAGED_TC(QF, 64, 2) PAGED_TC(QF, 64, 4) PAGED_TC(QF, 64, 8) \
-  PAGED_TC(QF, 128, 1) PAGED_TC(QF, 128, 2) PAGED_TC(QF, 128, 4) PAGED_TC(QF, 128, 8)
+    return two ? launch_tc<QF, CF, d, g, 2>(a, kmap, vmap, max_query_len, stream)      \
+               : launch_tc<QF, CF, d, g, 1>(a, kmap, vmap, max_query_len, stream);
+#define PAGED_TC_ALL(QF)                                                              \
+  PAGED_TC(QF, QF, 64, 1) PAGED_TC(QF, QF, 64, 2) PAGED_TC(QF, QF, 64, 4)             \
+  PAGED_TC(QF, QF, 64, 8) PAGED_TC(QF, QF, 128, 1) PAGED_TC(QF, QF, 128, 2)           \
+  PAGED_TC(QF, QF, 128, 4) PAGED_TC(QF, QF, 128, 8)
+#define PAGED_TC_FP8(QF)                                                              \
+  PAGED_TC(QF, E4M3, 128, 1) PAGED_TC(QF, E4M3, 128, 2) PAGED_TC(QF, E4M3, 128, 4)    \
+  PAGED_TC(QF, E4M3, 128, 8)
+  const bool fp8 = cache_dtype == kE4M3;
   if (q_dtype == kF16) {
-    PAGED_TC_ALL(F16)
+    if (fp8) {
+      PAGED_TC_FP8(F16)
+    } else {
+      PAGED_TC_ALL(F16)
+    }
   } else if (q_dtype == kBF16) {
-    PAGED_TC_ALL(BF16)
+    if (fp8) {
+      PAGED_TC_FP8(BF16)
+    } else {
+      PAGED_TC_ALL(BF16)
+    }
   }
+#undef PAGED_TC_FP8
 #undef PAGED_TC_ALL
 #undef PAGED_TC
   return cudaErrorNotSupported;

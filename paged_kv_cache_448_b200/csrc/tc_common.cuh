@@ -1,6 +1,6 @@
 // tc_common.cuh — 5th-generation tensor core (tcgen05) building blocks:
 // tensor-memory allocation, shared-memory matrix descriptors, the f16/bf16
-// instruction descriptor, MMA issue and commit, tensor-memory loads/stores.
+// and 8-bit (E4M3 / E5M2) instruction descriptors, MMA issue and commit, tensor-memory loads/stores.
 // Bit layouts follow the PTX ISA's tcgen05 description (the same encoding
 // CUTLASS's sm100 UMMA descriptors use).
 #pragma once
@@ -18,8 +18,8 @@ namespace tc {
 //   bits 61-63: layout (2 = 128-byte swizzle)
 // K-major (rows of K elements, 128 bytes per row, 8-row groups 1024 bytes
 // apart): lbo = 16 (unused), sbo = 1024. MN-major (rows of the K index, each
-// 64 MN elements, 8-row groups `sbo` apart, the next 64 MN elements `lbo`
-// apart).
+// 128 bytes of MN elements (64 16-bit or 128 8-bit ones), 8-row groups `sbo`
+// apart, the next 128 bytes of MN elements `lbo` apart).
 __device__ __forceinline__ uint64_t sw128_desc(const void* smem, uint32_t lbo_bytes,
                                                uint32_t sbo_bytes) {
   const uint64_t a = (smem_addr(smem) >> 4) & 0x3FFFu;
@@ -37,6 +37,44 @@ __device__ __forceinline__ constexpr uint32_t idesc_f16() {
   return (1u << 4) | ((BF ? 1u : 0u) << 7) | ((BF ? 1u : 0u) << 10) |
          ((B_MN_MAJOR ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::f8f6f4 with fp32 accumulators; operand
+// formats 0 = E4M3, 1 = E5M2 (bits 7-9 for A, 10-12 for B), the other fields
+// as in idesc_f16.
+template <int A_FMT, int B_FMT, int M, int N, bool B_MN_MAJOR>
+__device__ __forceinline__ constexpr uint32_t idesc_f8() {
+  static_assert(M == 128 && N % 16 == 0 && N >= 16 && N <= 256, "UMMA shape");
+  static_assert((A_FMT == 0 || A_FMT == 1) && (B_FMT == 0 || B_FMT == 1), "E4M3 / E5M2");
+  return (1u << 4) | (static_cast<uint32_t>(A_FMT) << 7) | (static_cast<uint32_t>(B_FMT) << 10) |
+         ((B_MN_MAJOR ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D (tensor memory) (+)= A . B, 8-bit operands (K = 32 per instruction), both
+// from shared memory.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      :
+      : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+
+// The same with A in tensor memory (lane = row, four 8-bit K elements per
+// 32-bit column, K order; 8 columns per instruction).
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      :
+      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
 }
 
 // D[tmem] (+)= A[smem] . B[smem]; issued by one thread.
@@ -158,6 +196,16 @@ __device__ __forceinline__ void st32u(uint32_t taddr, const uint32_t (&v)[32]) {
       "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
       "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
       "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
       : "memory");
 }
 

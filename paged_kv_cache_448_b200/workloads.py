@@ -114,7 +114,7 @@ def spec(config: int, seed: int | None = None, *, small: bool = False) -> Spec:
 
 # ---------------------------------------------------- multi-token queries
 
-PREFILL_NAMES = ("chunk_llama7b", "chunk_gqa70b", "verify_gqa70b")
+PREFILL_NAMES = ("chunk_llama7b", "chunk_gqa70b", "verify_gqa70b", "chunk_gqa70b_fp8")
 
 
 def prefill_spec(name: str, seed: int | None = None, *, small: bool = False):
@@ -129,6 +129,8 @@ def prefill_spec(name: str, seed: int | None = None, *, small: bool = False):
       64 query / 8 kv heads, block_size 32, bf16.
     * ``verify_gqa70b``  verification of 8 draft tokens for 64 sequences with
       prior contexts uniform in [1024, 4096]; 64 / 8 heads, block_size 16, bf16.
+    * ``chunk_gqa70b_fp8``  ``chunk_gqa70b`` over an FP8 E4M3 cache with
+      per-kv-head scales (bf16 queries), as in the prefix_fp8 decode workload.
     """
     if seed is None:
         seed = 2000 + PREFILL_NAMES.index(name)
@@ -137,7 +139,7 @@ def prefill_spec(name: str, seed: int | None = None, *, small: bool = False):
         S, chunk, lo, hi, H, Hkv, bs, dt = (3, 40, 0, 100, 4, 4, 16, "f16") if small else \
             (16, 512, 0, 3584, 32, 32, 16, "f16")
         prior = _uniform_ints(rng, lo, hi, S)
-    elif name == "chunk_gqa70b":
+    elif name in ("chunk_gqa70b", "chunk_gqa70b_fp8"):
         S, chunk, lo, hi, H, Hkv, bs, dt = (3, 33, 10, 150, 16, 2, 32, "bf16") if small else \
             (16, 256, 1024, 8192, 64, 8, 32, "bf16")
         prior = np.round(np.exp(rng.uniform(math.log(lo), math.log(hi), size=S))).astype(np.int32)
@@ -148,8 +150,8 @@ def prefill_spec(name: str, seed: int | None = None, *, small: bool = False):
     else:
         raise ValueError(f"unknown multi-token workload {name}")
     qlens = np.full(S, chunk, np.int32)
-    sp = Spec(name, S, H, Hkv, 128, bs, dt, dt, 1.0 / math.sqrt(128),
-              (prior + qlens).astype(np.int32), seed=seed)
+    sp = Spec(name, S, H, Hkv, 128, bs, dt, "e4m3" if name.endswith("_fp8") else dt,
+              1.0 / math.sqrt(128), (prior + qlens).astype(np.int32), seed=seed)
     return sp, qlens
 
 

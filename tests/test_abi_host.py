@@ -275,6 +275,13 @@ def test_chunked_prefill_workspace_plan():
     rows = 64 * 8 * 64
     assert n > 256 and (n - 256) % (rows * (8 + 128 * 4)) < 256
     assert pk.chunked_prefill_workspace_size(1, 1, 3, 2, 128, 1, 10) == 0   # H % Hkv != 0
+    # an E4M3 cache takes tcgen05 only with head_dim 128: a long chunk of one
+    # sequence with head_dim 64 runs on the mma.sync kernel, split
+    fp8 = _native.PA_FP8_E4M3
+    assert pk.chunked_prefill_workspace_size(1, 512, 32, 32, 128, 512, 4096, fp8) == 256
+    assert pk.chunked_prefill_workspace_size(1, 512, 32, 32, 64, 512, 4096) == 256
+    assert pk.chunked_prefill_workspace_size(1, 512, 32, 32, 64, 512, 4096, fp8) > 256
+    assert pk.chunked_prefill_workspace_size(1, 512, 32, 32, 128, 512, 4096, 7) == 0
 
 
 def test_copy_blocks_rejects_bad_arguments_before_launch():

@@ -13,7 +13,7 @@ import torch
 import oracle
 import paged_kv_cache_448_b200 as pk
 from paged_kv_cache_448_b200 import workloads as wl
-from gpu_helpers import assert_close, dev, host_codes, i32
+from gpu_helpers import assert_close, dev, f32, host_codes, i32
 
 pytestmark = pytest.mark.gpu
 
@@ -24,12 +24,13 @@ def run_gpu(sp, st, hd, q, qlens, table=None, ctx=None):
     table = st.block_tables if table is None else table
     gq = dev(q, sp.q_dtype)
     out = torch.full_like(gq, float("nan"))
+    kc, vc = dev(hd.key_cache, sp.cache_dtype), dev(hd.value_cache, sp.cache_dtype)
     ws = pk.chunked_prefill_workspace(sp.num_seqs, int(qlens.sum()), sp.num_heads,
                                       sp.num_kv_heads, sp.head_dim, int(qlens.max()),
-                                      int(np.max(ctx)))
-    pk.chunked_prefill(out, gq, i32(cu), int(qlens.max()), dev(hd.key_cache, sp.cache_dtype),
-                       dev(hd.value_cache, sp.cache_dtype), i32(table), i32(ctx),
-                       int(np.max(ctx)), sp.scale, workspace=ws)
+                                      int(np.max(ctx)), pk.dtype_code(kc))
+    pk.chunked_prefill(out, gq, i32(cu), int(qlens.max()), kc, vc, i32(table), i32(ctx),
+                       int(np.max(ctx)), sp.scale, k_scale=f32(hd.k_scale),
+                       v_scale=f32(hd.v_scale), workspace=ws)
     return out, ws, cu
 
 
@@ -38,7 +39,8 @@ def run_oracle(sp, st, hd, q, cu, table=None, ctx=None):
                                   st.block_tables if table is None else table,
                                   sp.context_lens if ctx is None else ctx, cu,
                                   scale=np.float32(sp.scale), q_dtype=sp.q_dtype,
-                                  cache_dtype=sp.cache_dtype)
+                                  cache_dtype=sp.cache_dtype, k_scale=hd.k_scale,
+                                  v_scale=hd.v_scale)
 
 
 @pytest.mark.parametrize("name", wl.PREFILL_NAMES)
@@ -52,8 +54,8 @@ def test_multi_token_workloads_small(name):
     assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), sp.cache_dtype, name)
 
 
-def custom(ctxs, qlens, H, Hkv, D, bs, dt, seed):
-    sp = wl.Spec("custom", len(ctxs), H, Hkv, D, bs, dt, dt, 1.0 / math.sqrt(D),
+def custom(ctxs, qlens, H, Hkv, D, bs, dt, seed, cache_dt=None):
+    sp = wl.Spec("custom", len(ctxs), H, Hkv, D, bs, dt, cache_dt or dt, 1.0 / math.sqrt(D),
                  np.array(ctxs, np.int32), spare_blocks=3, seed=seed)
     st = wl.structure(sp)
     hd = wl.host_data(sp, st)
@@ -85,6 +87,37 @@ def test_multi_token_edge_sweep(kernel, dt, G, D, bs):
     pk.decode_check(ws)
     assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), dt,
                  f"{dt} G{G} D{D} bs{bs}")
+
+
+@pytest.mark.parametrize("chunks", ["tcgen05", "mma_sync"])
+@pytest.mark.parametrize("qdt", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_multi_token_e4m3_cache(chunks, qdt, G, D, bs):
+    """An E4M3 cache with per-kv-head scales, both chunk sets of the edge
+    sweep: long chunks with head_dim 128 on tcgen05 (kind::f8f6f4), the rest
+    on the mma.sync kernel."""
+    ctxs, qlens = EDGE[chunks]
+    sp, st, hd, q, qlens = custom(ctxs, qlens, 2 * G, 2, D, bs, qdt, seed=G * 10 + D + bs + 7,
+                                  cache_dt="e4m3")
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), "e4m3",
+                 f"e4m3 {qdt} G{G} D{D} bs{bs}")
+
+
+@pytest.mark.parametrize("qdt,G,D,bs", [("bf16", 8, 128, 16), ("f16", 2, 64, 32)])
+def test_split_key_range_e4m3(qdt, G, D, bs):
+    ctxs, qlens = [2100, 700, 3333], [8, 5, 8]
+    sp, st, hd, q, qlens = custom(ctxs, qlens, 2 * G, 2, D, bs, qdt, seed=950 + G,
+                                  cache_dt="e4m3")
+    assert pk.chunked_prefill_workspace_size(3, sum(qlens), 2 * G, 2, D, 8, 3333,
+                                             pk._native.PA_FP8_E4M3) > 256
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), "e4m3",
+                 f"split e4m3 {qdt} G{G}")
 
 
 @pytest.mark.parametrize("dt,G,D,bs", [("bf16", 8, 128, 16), ("f16", 4, 64, 32),
@@ -161,10 +194,10 @@ def test_multi_token_full_size_sampled(name):
     out = torch.empty_like(q)
     ws = pk.chunked_prefill_workspace(sp.num_seqs, int(qlens.sum()), sp.num_heads,
                                       sp.num_kv_heads, sp.head_dim, int(qlens.max()),
-                                      int(sp.context_lens.max()))
+                                      int(sp.context_lens.max()), pk.dtype_code(d["key_cache"]))
     pk.chunked_prefill(out, q, i32(cu), int(qlens.max()), d["key_cache"], d["value_cache"],
                        i32(st.block_tables), i32(sp.context_lens), int(sp.context_lens.max()),
-                       sp.scale, workspace=ws)
+                       sp.scale, k_scale=d["k_scale"], v_scale=d["v_scale"], workspace=ws)
     pk.decode_check(ws)
     assert torch.isfinite(out.float()).all()
     picks = [int(np.argmin(sp.context_lens))]
@@ -177,8 +210,11 @@ def test_multi_token_full_size_sampled(name):
         vc = host_codes(d["value_cache"].index_select(0, sel))
         table = np.arange(len(ids), dtype=np.int32)[None, :]
         qs = host_codes(q[cu[s]:cu[s + 1]])
+        ks, vs = (None, None) if d["k_scale"] is None else \
+            (d["k_scale"].cpu().numpy(), d["v_scale"].cpu().numpy())
         ref = oracle.chunked_prefill(qs, kc, vc, table, sp.context_lens[[s]],
                                      np.array([0, qlens[s]], np.int32), scale=np.float32(sp.scale),
-                                     q_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype)
+                                     q_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype,
+                                     k_scale=ks, v_scale=vs)
         assert_close(out[cu[s]:cu[s + 1]].double().cpu().numpy(), ref, sp.cache_dtype,
                      f"{name} seq {s}")
