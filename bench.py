@@ -331,6 +331,11 @@ def run_prefill(args):
                           f"{sp.cache_dtype} cache"}
     # tensor-bound when the work per K/V byte is above the machine balance
     peak_t, kind_t = measured_tensor_peak()
+    kind_t = f"{kind_t} dense bf16 (cuBLAS)"
+    G = sp.num_heads // sp.num_kv_heads
+    if sp.cache_dtype == "e4m3" and sp.head_dim == 128 and chunk * G >= 128:
+        # the tcgen05 kernel runs 8-bit MMAs (kind::f8f6f4): nominal fp8 = 2 x bf16
+        peak_t, kind_t = round(2 * peak_t, 1), f"{kind_t} x 2 (nominal fp8 / bf16 ratio)"
     peak_b, kind_b = measured_peaks()
     tensor_bound = flops / nbytes > peak_t * 1e12 / (peak_b * 1e9)
     if args.impl == "reference":
@@ -366,7 +371,7 @@ def run_prefill(args):
     tflops = flops / (ms * 1e-3) / 1e12
     gbs = nbytes / (ms * 1e-3) / 1e9
     roof = ({"bound": "tensor", "achieved": round(tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
-             "frac": round(tflops / peak_t, 4), "peak_kind": f"{kind_t} dense bf16 (cuBLAS)"}
+             "frac": round(tflops / peak_t, 4), "peak_kind": kind_t}
             if tensor_bound else
             {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak_b, "unit": "GB/s",
              "frac": round(gbs / peak_b, 4), "peak_kind": f"{kind_b} HBM copy GB/s"})
