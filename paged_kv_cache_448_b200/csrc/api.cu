@@ -421,8 +421,13 @@ namespace {
 
 // Kernel choice and split of the key range for the multi-token query.
 // Chunks that fill the 128 rows of a tensor-memory CTA (query tokens x heads
-// of a kv-head's group) run on tcgen05 (an E4M3 cache: head_dim 128 only);
-// shorter ones (a few draft tokens) on the 64-row mma.sync kernel. There,
+// of a kv-head's group) run on tcgen05 (an E4M3 cache: head_dim 128 only).
+// Shorter ones (a few draft tokens) leave most of those rows empty, yet the
+// tcgen05 kernel still wins while its CTAs fill a wave (two per SM) and each
+// kv-head has at least 8 rows (measured on B200: 8 draft tokens x 8 heads for
+// 64 sequences, 313 -> 275 us with a bf16 cache and 404 -> 259 us with E4M3,
+// where the mma.sync kernel widens every code in each of its four warps);
+// with fewer CTAs or rows they run on the 64-row mma.sync kernel. There,
 // when the CTAs (query tiles x kv-heads x sequences) cannot fill about four
 // waves of three CTAs per SM, the tiles of each CTA are cut into parts of at
 // least 256 tokens (16 tiles, a multiple of 4) handled by separate CTAs.
@@ -435,7 +440,11 @@ PrefillPlan make_prefill_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t gr
                               int32_t head_dim, int32_t max_query_len, int32_t max_context_len,
                               bool fp8) {
   PrefillPlan p{};
-  p.tc = (!fp8 || head_dim == 128) && static_cast<int64_t>(max_query_len) * group >= 128;
+  const int64_t rows = static_cast<int64_t>(max_query_len) * group;
+  const int64_t tc_ctas = static_cast<int64_t>(num_seqs) * num_kv_heads *
+                          ((max_query_len + 128 / group - 1) / (128 / group));
+  p.tc = (!fp8 || head_dim == 128) &&
+         (rows >= 128 || (rows >= 8 && tc_ctas >= 2LL * sm_count()));
   p.q_tiles = (max_query_len + prefill_tokens_per_cta(group) - 1) / prefill_tokens_per_cta(group);
   const int32_t max_tiles = std::max<int32_t>(1, (max_context_len + 15) / 16);
   p.partition_tiles = max_tiles;

@@ -271,9 +271,13 @@ def test_chunked_prefill_workspace_plan():
     # short chunks of many sequences already fill the GPU: no split
     assert pk.chunked_prefill_workspace_size(4096, 4096 * 8, 64, 8, 128, 8, 4096) == 256
     # few short-chunk CTAs with long contexts: partial rows for every part
-    n = pk.chunked_prefill_workspace_size(64, 64 * 8, 64, 8, 128, 8, 4096)
-    rows = 64 * 8 * 64
+    n = pk.chunked_prefill_workspace_size(16, 16 * 8, 64, 8, 128, 8, 4096)
+    rows = 16 * 8 * 64
     assert n > 256 and (n - 256) % (rows * (8 + 128 * 4)) < 256
+    # short chunks whose tcgen05 CTAs fill a wave (64 x 8 >= 2 per SM) run
+    # there, unsplit; with 2 rows per kv-head they stay on mma.sync, split
+    assert pk.chunked_prefill_workspace_size(64, 64 * 8, 64, 8, 128, 8, 4096) == 256
+    assert pk.chunked_prefill_workspace_size(16, 16 * 2, 32, 32, 128, 2, 4096) > 256
     assert pk.chunked_prefill_workspace_size(1, 1, 3, 2, 128, 1, 10) == 0   # H % Hkv != 0
     # an E4M3 cache takes tcgen05 only with head_dim 128: a long chunk of one
     # sequence with head_dim 64 runs on the mma.sync kernel, split

@@ -107,6 +107,29 @@ def test_multi_token_e4m3_cache(chunks, qdt, G, D, bs):
                  f"e4m3 {qdt} G{G} D{D} bs{bs}")
 
 
+@pytest.mark.parametrize("cache", ["bf16", "e4m3"])
+@pytest.mark.parametrize("G,q", [(4, 8), (8, 1), (8, 5)])
+def test_short_chunks_of_many_sequences_on_tcgen05(cache, G, q):
+    """Short chunks (fewer than 128 rows per kv-head) whose tcgen05 CTAs fill
+    a wave run there, unsplit: 150 sequences x 2 kv-heads, ragged chunks of at
+    most q tokens, contexts long enough that the mma.sync kernel would split."""
+    rng = np.random.default_rng(40 + G + q)
+    n = 150
+    ctxs = rng.integers(1, 700, size=n)
+    ctxs[:3] = [1, 699, 520]
+    qlens = np.minimum(rng.integers(1, q + 1, size=n), ctxs)
+    qlens[1] = q
+    sp, st, hd, qv, qlens = custom(list(ctxs), list(qlens), 2 * G, 2, 128, 16, "bf16",
+                                   seed=70 + G + q, cache_dt=cache)
+    code = pk._native.PA_FP8_E4M3 if cache == "e4m3" else pk._native.PA_BF16
+    assert pk.chunked_prefill_workspace_size(n, int(qlens.sum()), 2 * G, 2, 128, q, 699,
+                                             code) == 256
+    out, ws, cu = run_gpu(sp, st, hd, qv, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, qv, cu), cache,
+                 f"short chunks {cache} G{G} q{q}")
+
+
 @pytest.mark.parametrize("qdt,G,D,bs", [("bf16", 8, 128, 16), ("f16", 2, 64, 32)])
 def test_split_key_range_e4m3(qdt, G, D, bs):
     ctxs, qlens = [2100, 700, 3333], [8, 5, 8]
