@@ -206,9 +206,9 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* query,
  * max_context_len, num_blocks: as in pa_decode (context_lens include the
  * query tokens).
  * workspace       >= pa_chunked_prefill_workspace_size(...) bytes, 256-byte aligned,
- *                 zeroed once (pa_workspace_init). Short chunks whose CTAs cannot
- *                 fill the GPU split each key range into parts combined by a
- *                 second kernel, with partial results here. Its error word reports, through pa_decode_check, table
+ *                 zeroed once (pa_workspace_init). Launches whose CTAs cannot
+ *                 fill the GPU (few sequences or kv-heads) split each key range
+ *                 into parts combined by a second kernel, with partial results here. Its error word reports, through pa_decode_check, table
  *                 entries outside the pool (read as zeros), clipped context
  *                 lengths, and a query longer than its context (bit 16; those
  *                 rows are written as zeros).

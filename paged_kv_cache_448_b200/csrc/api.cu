@@ -427,12 +427,13 @@ namespace {
 // kv-head has at least 8 rows (measured on B200: 8 draft tokens x 8 heads for
 // 64 sequences, 313 -> 275 us with a bf16 cache and 404 -> 259 us with E4M3,
 // where the mma.sync kernel widens every code in each of its four warps);
-// with fewer CTAs or rows they run on the 64-row mma.sync kernel. There,
-// when the CTAs (query tiles x kv-heads x sequences) cannot fill about four
-// waves of three CTAs per SM, the tiles of each CTA are cut into parts of at
-// least 256 tokens (16 tiles, a multiple of 4) handled by separate CTAs.
+// with fewer CTAs or rows they run on the 64-row mma.sync kernel. When the
+// CTAs (query tiles x kv-heads x sequences) cannot fill a wave of the
+// tcgen05 kernel, or about four waves of three mma.sync CTAs per SM, the
+// tiles of each CTA are cut into parts of at least 256 tokens (16 tiles, a
+// multiple of 4) handled by separate CTAs and merged by a combine kernel.
 struct PrefillPlan {
-  bool tc;                  // tcgen05 kernel (no split)
+  bool tc;                  // tcgen05 kernel, else mma.sync
   int32_t q_tiles, partition_tiles, max_parts;
 };
 
@@ -441,18 +442,26 @@ PrefillPlan make_prefill_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t gr
                               bool fp8) {
   PrefillPlan p{};
   const int64_t rows = static_cast<int64_t>(max_query_len) * group;
+  // query tokens per CTA: tcgen05 128 rows per group, two groups once the
+  // chunks fill 256 rows; mma.sync 64 rows
+  const int32_t qt_tc = (rows >= 256 ? 256 : 128) / group;
   const int64_t tc_ctas = static_cast<int64_t>(num_seqs) * num_kv_heads *
-                          ((max_query_len + 128 / group - 1) / (128 / group));
+                          ((max_query_len + qt_tc - 1) / qt_tc);
   p.tc = (!fp8 || head_dim == 128) &&
          (rows >= 128 || (rows >= 8 && tc_ctas >= 2LL * sm_count()));
-  p.q_tiles = (max_query_len + prefill_tokens_per_cta(group) - 1) / prefill_tokens_per_cta(group);
+  const int32_t qt = p.tc ? qt_tc : prefill_tokens_per_cta(group);
+  p.q_tiles = (max_query_len + qt - 1) / qt;
   const int32_t max_tiles = std::max<int32_t>(1, (max_context_len + 15) / 16);
   p.partition_tiles = max_tiles;
   p.max_parts = 1;
-  if (p.tc) return p;
   const int64_t ctas = static_cast<int64_t>(p.q_tiles) * num_kv_heads * num_seqs;
-  const int64_t want = 4LL * sm_count() * 3;
-  if (ctas >= want || max_tiles < 32) return p;
+  // CTAs wanted: tcgen05 splits below half a wave (one CTA of two groups, or
+  // two of one group, per SM) up to a wave - measured on B200, 64 CTAs of
+  // 4 x 128-token chunks 325 -> 247 us, while 128 CTAs of one 512-token
+  // chunk lost (326 -> 354 us); mma.sync about four waves of three per SM
+  const int64_t wave = (rows >= 256 ? 1LL : 2LL) * sm_count();
+  const int64_t want = p.tc ? wave : 4LL * sm_count() * 3;
+  if (ctas >= (p.tc ? (wave + 1) / 2 : want) || max_tiles < 32) return p;
   const int64_t by_work = (want + ctas - 1) / ctas;
   const int32_t parts = static_cast<int32_t>(std::min<int64_t>(by_work, max_tiles / 16));
   if (parts <= 1) return p;

@@ -25,9 +25,9 @@ struct PrefillArgs {
   int32_t num_kv_heads;
   int32_t block_size;
   float scale_log2;              // softmax scale * log2(e)
-  // split of the key range (mma.sync kernel only; 1 part = no split)
+  // split of the key range (1 part = no split)
   int32_t q_tiles;               // query tiles per (sequence, kv-head) in the launch
-  int32_t partition_tiles;       // 16-token tiles per part
+  int32_t partition_tiles;       // 16-token tiles per part (a multiple of 4)
   int32_t max_parts;
   float* ws_o;                   // [T * H][max_parts][D] partial outputs (normalised)
   float2* ws_ml;                 // [T * H][max_parts] (max, sum) in base-2 units
@@ -46,6 +46,11 @@ __host__ __device__ constexpr int prefill_tokens_per_cta(int group) { return 64 
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                            int q_dtype, int cache_dtype, int head_dim, int group,
                            int32_t max_query_len, cudaStream_t stream);
+
+// Merge of the key-range parts of a split launch (a.max_parts > 1) whose
+// CTAs took qt query tokens each: one warp per (query token, head).
+cudaError_t launch_prefill_combine(const PrefillArgs& a, int q_dtype, int head_dim, int qt,
+                                   int32_t max_query_len, cudaStream_t stream);
 
 // The same on the 5th-generation tensor cores (tcgen05, tensor memory); the
 // tensor maps are the one-segment boxes of encode_cache_map(..., 1 segment).

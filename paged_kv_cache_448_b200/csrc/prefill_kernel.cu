@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
 // w_p = l_p 2^(m_p - M): out = sum_p w_p o_p / sum_p w_p. One warp per
 // (query token, head); rows whose range was not split were written directly.
 template <class QF, int D>
-__global__ void __launch_bounds__(128) paged_prefill_combine(const PrefillArgs a, int group) {
+__global__ void __launch_bounds__(128) paged_prefill_combine(const PrefillArgs a, int qt) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x * 4 + warp, i = blockIdx.y, s = blockIdx.z;
@@ -500,7 +500,6 @@ __global__ void __launch_bounds__(128) paged_prefill_combine(const PrefillArgs a
   int ctx = a.context_lens[s];
   ctx = ctx < 0 ? 0 : (ctx > a.ctx_limit ? a.ctx_limit : ctx);
   if (qlen > ctx) return;  // rows zeroed by the main kernel
-  const int qt = prefill_tokens_per_cta(group);
   const int tok0 = (i / qt) * qt, ntok = min(qt, qlen - tok0);
   const int pos0 = ctx - qlen + tok0;
   const int ntiles_all = (pos0 + ntok - 1) / kTileRows + 1;
@@ -546,10 +545,24 @@ cudaError_t launch_one(const PrefillArgs& a, const CUtensorMap& kmap, const CUte
   if (e != cudaSuccess || a.max_parts <= 1) return e;
   return launch_pdl(paged_prefill_combine<QF, D>,
                     dim3((a.num_heads + 3) / 4, static_cast<unsigned>(max_query_len), a.num_seqs),
-                    128, 0, stream, a, G);
+                    128, 0, stream, a, QT);
 }
 
 }  // namespace
+
+cudaError_t launch_prefill_combine(const PrefillArgs& a, int q_dtype, int head_dim, int qt,
+                                   int32_t max_query_len, cudaStream_t stream) {
+  const dim3 grid((a.num_heads + 3) / 4, static_cast<unsigned>(max_query_len), a.num_seqs);
+  if (q_dtype == kF16 && head_dim == 64)
+    return launch_pdl(paged_prefill_combine<F16, 64>, grid, 128, 0, stream, a, qt);
+  if (q_dtype == kF16 && head_dim == 128)
+    return launch_pdl(paged_prefill_combine<F16, 128>, grid, 128, 0, stream, a, qt);
+  if (q_dtype == kBF16 && head_dim == 64)
+    return launch_pdl(paged_prefill_combine<BF16, 64>, grid, 128, 0, stream, a, qt);
+  if (q_dtype == kBF16 && head_dim == 128)
+    return launch_pdl(paged_prefill_combine<BF16, 128>, grid, 128, 0, stream, a, qt);
+  return cudaErrorNotSupported;
+}
 
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                            int q_dtype, int cache_dtype, int head_dim, int group,

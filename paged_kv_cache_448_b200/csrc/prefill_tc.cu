@@ -19,7 +19,10 @@
 //  * P (f16/bf16, bf16 as hi + lo parts) goes to shared memory and thread 0
 //    issues O += P V (M=128, N=D, K=64; V read MN-major), accumulating in
 //    tensor memory, then refills the stage once those MMAs completed;
-//  * the epilogue divides each row of O by its sum and stores it.
+//  * the epilogue divides each row of O by its sum and stores it. When the
+//    key range is split (few CTAs), a CTA takes one part of its 16-token
+//    tiles and writes (max, sum) and its normalised O per row for the
+//    combine kernel, as the mma.sync kernel does.
 // An E4M3 cache (head_dim 128: a 128-byte row) runs on kind::f8f6f4 with the
 // cache tiles as they arrive: Q goes to shared memory as E4M3 hi + lo parts
 // (q * 2^e = hi + lo, e a power of two per row that puts max |q| below 2^8,
@@ -150,7 +153,8 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   __shared__ uint32_t tmem_slot;
   __shared__ int aborted;
 
-  const int z = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+  const int z = blockIdx.x % a.q_tiles, part = blockIdx.x / a.q_tiles;
+  const int kvh = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int r = 0; r < KR; ++r) {
@@ -191,6 +195,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   const int64_t row_off =
       (static_cast<int64_t>(q0 + tok0 + tok) * a.num_heads + kvh * G + tid % G) * D;
   if (qlen > ctx) {  // a query longer than its context: rows become zeros
+    if (part > 0) return;
     if (tid == 0 && z == 0 && kvh == 0) report(a.err, kErrQueryLonger);
     if (valid) {
       uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
@@ -200,8 +205,16 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   }
   const int pos0 = ctx - qlen + tok0;
   const int p_max = pos0 + ntok - 1;
-  const int ntiles = p_max / TR + 1;              // 16-token tiles holding tokens 0..p_max
-  const int nsteps = p_max / NT + 1;
+  // 16-token tiles holding tokens 0..p_max, cut into parts of partition_tiles
+  // (a multiple of the 4 tiles of a step); this CTA takes part `part`: tiles
+  // tbase .. tend-1, steps kbase .. kbase+nsteps-1
+  const int ntiles_all = p_max / TR + 1;
+  const int parts = (ntiles_all + a.partition_tiles - 1) / a.partition_tiles;
+  if (part >= parts) return;
+  const int tbase = part * a.partition_tiles;
+  const int tend = min(ntiles_all, tbase + a.partition_tiles);
+  const int kbase = tbase / (NT / TR);
+  const int nsteps = (tend - tbase + NT / TR - 1) / (NT / TR);
 
   __syncthreads();  // barrier initialisation visible to every thread
   if (warp == kMma) tc::alloc(&tmem_slot, C::TMEM_COLS);
@@ -277,7 +290,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
         uint8_t* dst = is_v ? sv(k) : sk(k);
         uint64_t* bar = is_v ? &vfull[k % VR] : &kfull[k % KR];
         const CUtensorMap* map = is_v ? &vmap : &kmap;
-        const int t_begin = k * (NT / TR), t_end = min(ntiles, (k + 1) * (NT / TR));
+        const int t_begin = (kbase + k) * (NT / TR), t_end = min(tend, t_begin + NT / TR);
         mbar_arrive_expect_tx(bar, static_cast<uint32_t>(NSEG * (t_end - t_begin) * TR * 128));
 #pragma unroll
         for (int j = 0; j < NT / TR; ++j) {
@@ -299,8 +312,8 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       auto load_ids = [&](int k, int32_t (&dst)[NT / TR]) {
 #pragma unroll
         for (int j = 0; j < NT / TR; ++j) {
-          const int t = k * (NT / TR) + j;
-          dst[j] = t < ntiles ? table[(t * TR) / a.block_size] : 0;
+          const int t = (kbase + k) * (NT / TR) + j;
+          dst[j] = t < tend ? table[(t * TR) / a.block_size] : 0;
         }
       };
       bool ok = true;
@@ -437,7 +450,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
     const uint32_t t_o = t_grp + kTmemO + lane_base;
     const int rr = tid % kTcRows;                // row within the group = tensor-memory lane
     const int p_row = valid ? pos0 + tok : -1;
-    const int kv_valid = min(ctx, ntiles * TR);  // tokens with loaded, real rows
+    const int kv_valid = min(ctx, tend * TR);    // tokens with loaded, real rows
     float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int k = 0; ok && k < nsteps; ++k) {
@@ -446,7 +459,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       tc::fence_after_sync();
       float x[NT];
       tc::ld64(t_grp + (k & 1) * NT + lane_base, x);
-      const int tk0 = k * NT;
+      const int tk0 = (kbase + k) * NT;
       // causal mask only where the step reaches past this row's position
       if (tk0 + NT - 1 > p_row) {
 #pragma unroll
@@ -537,21 +550,40 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
     if (!ok) {
       aborted = 1;
     } else {
-      // ---- epilogue: out = O / l, rounded to the q dtype
+      // ---- epilogue: out = O / l, rounded to the q dtype; or, for a part of
+      // a split key range, (max, sum) and O / l in fp32 for the combine
+      // kernel (a row that sees none of the part's tokens leaves -inf, 0, 0)
       tc::fence_after_sync();
       const float inv = (l > 0.f ? 1.f / l : 0.f) * (FP8 ? a.v_scale[kvh] : 1.f);
-      uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
+      if (parts == 1) {
+        uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tc::ld32(t_o + c * 32, o);
-        if (valid) {
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tc::ld32(t_o + c * 32, o);
+          if (valid) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            o4[c * 4 + q] = make_uint4(pack_pair(BF, o[8 * q] * inv, o[8 * q + 1] * inv),
-                                       pack_pair(BF, o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                       pack_pair(BF, o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                       pack_pair(BF, o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+            for (int q = 0; q < 4; ++q)
+              o4[c * 4 + q] = make_uint4(pack_pair(BF, o[8 * q] * inv, o[8 * q + 1] * inv),
+                                         pack_pair(BF, o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                         pack_pair(BF, o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                         pack_pair(BF, o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+          }
+        }
+      } else {
+        const int64_t prow = (row_off / D) * a.max_parts + part;
+        if (valid) a.ws_ml[prow] = make_float2(m_used, l);
+        float4* w4 = reinterpret_cast<float4*>(a.ws_o + prow * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tc::ld32(t_o + c * 32, o);
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              w4[c * 8 + q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv,
+                                          o[4 * q + 3] * inv);
+          }
         }
       }
     }
@@ -574,9 +606,13 @@ cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUten
   auto kern = paged_prefill_tc_kernel<QF, CF, D, G, NG>;
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  const unsigned tiles = static_cast<unsigned>((max_query_len + C::QT - 1) / C::QT);
-  return launch_pdl(kern, dim3(tiles, a.num_kv_heads, a.num_seqs), NG * kTcRows + 64, smem,
-                    stream, a, kmap, vmap);
+  if (a.q_tiles != (max_query_len + C::QT - 1) / C::QT) return cudaErrorInvalidValue;
+  e = launch_pdl(kern, dim3(static_cast<unsigned>(a.q_tiles * a.max_parts), a.num_kv_heads,
+                            a.num_seqs),
+                 NG * kTcRows + 64, smem, stream, a, kmap, vmap);
+  if (e != cudaSuccess || a.max_parts <= 1) return e;
+  return launch_prefill_combine(a, std::is_same<QF, BF16>::value ? kBF16 : kF16, D, C::QT,
+                                max_query_len, stream);
 }
 
 }  // namespace

@@ -266,8 +266,14 @@ def test_prefix_cache_matches_oracle_model_on_random_requests():
 
 
 def test_chunked_prefill_workspace_plan():
-    # chunks that fill a tensor-memory CTA never split: header only
+    # chunks that fill tensor-memory CTAs, enough of them for a wave: header only
     assert pk.chunked_prefill_workspace_size(16, 16 * 512, 32, 32, 128, 512, 4096) == 256
+    # one sequence's 128-token chunk (8 x 2 tcgen05 CTAs, below half a wave
+    # of 148): the key range splits, partial rows for every part; its
+    # 512-token chunk (8 x 16 CTAs) does not
+    n = pk.chunked_prefill_workspace_size(1, 128, 32, 8, 128, 128, 8192)
+    assert n > 256 and (n - 256) % (128 * 32 * (8 + 128 * 4)) < 256
+    assert pk.chunked_prefill_workspace_size(1, 512, 64, 8, 128, 512, 8192) == 256
     # short chunks of many sequences already fill the GPU: no split
     assert pk.chunked_prefill_workspace_size(4096, 4096 * 8, 64, 8, 128, 8, 4096) == 256
     # few short-chunk CTAs with long contexts: partial rows for every part
@@ -279,13 +285,14 @@ def test_chunked_prefill_workspace_plan():
     assert pk.chunked_prefill_workspace_size(64, 64 * 8, 64, 8, 128, 8, 4096) == 256
     assert pk.chunked_prefill_workspace_size(16, 16 * 2, 32, 32, 128, 2, 4096) > 256
     assert pk.chunked_prefill_workspace_size(1, 1, 3, 2, 128, 1, 10) == 0   # H % Hkv != 0
-    # an E4M3 cache takes tcgen05 only with head_dim 128: a long chunk of one
-    # sequence with head_dim 64 runs on the mma.sync kernel, split
+    # an E4M3 cache takes tcgen05 only with head_dim 128: 4 sequences' long
+    # chunks fill a tcgen05 wave (256 CTAs), unsplit, but with head_dim 64
+    # they run on the mma.sync kernel, whose 1024 CTAs are split
     fp8 = _native.PA_FP8_E4M3
-    assert pk.chunked_prefill_workspace_size(1, 512, 32, 32, 128, 512, 4096, fp8) == 256
-    assert pk.chunked_prefill_workspace_size(1, 512, 32, 32, 64, 512, 4096) == 256
-    assert pk.chunked_prefill_workspace_size(1, 512, 32, 32, 64, 512, 4096, fp8) > 256
-    assert pk.chunked_prefill_workspace_size(1, 512, 32, 32, 128, 512, 4096, 7) == 0
+    assert pk.chunked_prefill_workspace_size(4, 2048, 32, 32, 128, 512, 4096, fp8) == 256
+    assert pk.chunked_prefill_workspace_size(4, 2048, 32, 32, 64, 512, 4096) == 256
+    assert pk.chunked_prefill_workspace_size(4, 2048, 32, 32, 64, 512, 4096, fp8) > 256
+    assert pk.chunked_prefill_workspace_size(4, 2048, 32, 32, 128, 512, 4096, 7) == 0
 
 
 def test_copy_blocks_rejects_bad_arguments_before_launch():

@@ -130,6 +130,29 @@ def test_short_chunks_of_many_sequences_on_tcgen05(cache, G, q):
                  f"short chunks {cache} G{G} q{q}")
 
 
+@pytest.mark.parametrize("qdt,cache,G,D,bs,qlens", [
+    ("bf16", "bf16", 8, 128, 16, [150, 129, 140]),   # two row groups (>= 256 rows)
+    ("f16", "f16", 1, 128, 32, [200, 129, 160]),     # one row group
+    ("bf16", "e4m3", 4, 128, 16, [64, 40, 33]),
+    ("f16", "f16", 2, 64, 32, [100, 70, 65]),
+])
+def test_split_key_range_tcgen05(qdt, cache, G, D, bs, qlens):
+    """Long chunks of three sequences: too few tcgen05 CTAs for a wave, so
+    each key range is cut into parts merged by the combine kernel; rows
+    whose causal range ends inside an earlier part, ragged last parts."""
+    ctxs = [2100, 700, 3333]
+    sp, st, hd, q, qlens = custom(ctxs, qlens, 2 * G, 2, D, bs, qdt, seed=990 + G + D,
+                                  cache_dt=cache)
+    code = {"f16": 0, "bf16": 1, "e4m3": 2}[cache]
+    assert max(qlens) * G >= 128
+    assert pk.chunked_prefill_workspace_size(3, int(qlens.sum()), 2 * G, 2, D, int(qlens.max()),
+                                             3333, code) > 256
+    out, ws, cu = run_gpu(sp, st, hd, q, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, q, cu), cache,
+                 f"tcgen05 split {cache} G{G} D{D}")
+
+
 @pytest.mark.parametrize("qdt,G,D,bs", [("bf16", 8, 128, 16), ("f16", 2, 64, 32)])
 def test_split_key_range_e4m3(qdt, G, D, bs):
     ctxs, qlens = [2100, 700, 3333], [8, 5, 8]
