@@ -313,6 +313,41 @@ def test_copy_blocks_rejects_bad_arguments_before_launch():
     assert call(n=0) == _native.PA_OK           # nothing to do, no device call
 
 
+def test_chunked_prefill_rejects_bad_arguments_before_launch():
+    lib = _native.lib()
+    P = 1 << 20                                 # any 256-byte aligned address; never touched
+    F16, BF16, E4M3 = _native.PA_F16, _native.PA_BF16, _native.PA_FP8_E4M3
+    def call(T=8, mql=8, S=1, H=8, Hkv=2, D=128, bs=16, qd=BF16, cd=BF16, ks=None, vs=None,
+             ws=P, wsb=256, scale=0.088, q=P, out=P, mctx=64):
+        return lib.pa_chunked_prefill(out, q, P, T, mql, P, P, P, 64, P, mctx, S, H, Hkv, D, bs,
+                                      64, scale, qd, cd, ks, vs, ws, wsb, None)
+    bad, unsup = _native.PA_ERR_INVALID_ARG, _native.PA_ERR_UNSUPPORTED
+    assert call(cd=F16) == unsup                # 16-bit cache of another dtype than the query
+    assert call(qd=E4M3, cd=E4M3, ks=P, vs=P) == unsup   # the query is f16 or bf16
+    assert call(cd=E4M3) == bad                 # E4M3 without its scales
+    assert call(cd=E4M3, ks=P) == bad
+    assert call(ks=P, vs=P) == bad              # scales with a 16-bit cache
+    assert call(cd=E4M3, ks=P + 2, vs=P) == bad  # misaligned scale
+    assert call(H=12) == unsup                  # group 6
+    assert call(H=7) == bad                     # H % Hkv != 0
+    assert call(D=96) == unsup
+    assert call(bs=8) == unsup
+    assert call(scale=float("nan")) == bad
+    assert call(ws=None) == bad
+    assert call(ws=P + 16) == bad               # not 256-byte aligned
+    assert call(wsb=128) == bad                 # smaller than the header
+    assert call(q=None) == bad
+    assert call(out=P + 4) == bad
+    assert call(T=-1) == bad
+    assert call(T=0) == _native.PA_OK           # nothing to do, no device call
+    # a split launch (8 tokens of one sequence over 1024 keys) needs its
+    # partial rows: a workspace one vector short is refused
+    need = pk.chunked_prefill_workspace_size(1, 8, 8, 2, 128, 8, 1024, BF16)
+    assert need > 256
+    assert call(mctx=1024, wsb=need - 16) == bad
+    assert b"workspace" in lib.pa_last_error()
+
+
 def test_workspace_sizes_and_partition_plan():
     # single pass: only the 256-byte header (error word and failure record)
     assert pk.decode_workspace_size(4, 4, 4, 64, 16, 100, 0) == 256
