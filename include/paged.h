@@ -208,12 +208,20 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* query,
  * workspace       >= pa_chunked_prefill_workspace_size(...) bytes, 256-byte aligned,
  *                 zeroed once (pa_workspace_init). Launches whose CTAs cannot
  *                 fill the GPU (few sequences or kv-heads) split each key range
- *                 into parts combined by a second kernel, with partial results here. Its error word reports, through pa_decode_check, table
+ *                 into parts combined by a second kernel, with partial results
+ *                 here. Its error word reports, through pa_decode_check, table
  *                 entries outside the pool (read as zeros), clipped context
  *                 lengths, and a query longer than its context (bit 16; those
  *                 rows are written as zeros).
  * Supported: head_dim in {64, 128}; block_size in {16, 32}; group in {1, 2, 4, 8};
  *            at most 65535 sequences and kv-heads.
+ * Errors (returned before any launch, nothing written): PA_ERR_INVALID_ARG for
+ * negative sizes, num_heads % num_kv_heads != 0, a non-finite scale, null or
+ * misaligned pointers (16 bytes for tensors, 4 for tables and scales), scales
+ * given for a 16-bit cache or missing for E4M3, and a workspace that is
+ * missing, misaligned or smaller than needed; PA_ERR_UNSUPPORTED for other
+ * dtypes, head_dim, block_size or group; PA_ERR_CUDA for a failed launch.
+ * Nothing to do (no sequences, tokens or query rows) returns PA_OK at once.
  */
 PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t* cu_query_lens,
                                     int32_t num_tokens, int32_t max_query_len,
