@@ -67,3 +67,58 @@ def test_slots_and_sizes_from_c(c_output):
         16, 16 * 512, 32, 32, 128, 512, 4096)
     status, msg = c_output["bad_decode"].split()
     assert int(status) == _native.PA_ERR_INVALID_ARG and msg == "message"
+
+
+@pytest.mark.gpu
+def test_decode_step_from_c(tmp_path):
+    """tests/abi_c_decode.c runs reshape_and_cache and decode through the C
+    ABI with only the CUDA runtime (no PyTorch): its tables equal the oracle
+    allocator's, its scattered caches equal the oracle's bit for bit, and its
+    output is within the bf16 tolerance of the oracle's decode."""
+    import numpy as np
+
+    import oracle
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler on this machine")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    lib_dir = os.path.dirname(_native.LIB_PATH)
+    _native.lib()
+    exe = str(tmp_path / "abi_c_decode")
+    subprocess.run([gcc, "-std=c11", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), "-I", os.path.join(cuda, "include"),
+                    os.path.join(ROOT, "tests", "abi_c_decode.c"),
+                    "-L", lib_dir, "-lpaged", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                    f"-Wl,-rpath,{lib_dir}", f"-Wl,-rpath,{os.path.join(cuda, 'lib64')}",
+                    "-o", exe], check=True, capture_output=True, text=True)
+    run = subprocess.run([exe, str(tmp_path)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stderr
+    S, H, HKV, D, BS, NB, MAXB = 3, 8, 2, 128, 16, 32, 19
+
+    def load(name, dtype, shape):
+        return np.fromfile(tmp_path / name, dtype=dtype).reshape(shape)
+
+    ctx = load("context_lens.bin", np.int32, (S,))
+    table = load("block_tables.bin", np.int32, (S, MAXB))
+    slots = load("slots.bin", np.int32, (S,))
+    bm = BlockManager(NB, [(i * 7 + 3) % NB for i in range(NB)])
+    ref_table = np.full((S, MAXB), -1, np.int32)
+    for s in range(S):
+        ids = bm.allocate(-(-int(ctx[s]) // BS))
+        ref_table[s, :len(ids)] = ids
+    assert np.array_equal(table, ref_table)
+    assert np.array_equal(slots, oracle.slot_mapping(ref_table, ctx - 1, BS))
+    kc = load("key_cache_in.bin", np.uint16, (NB, BS, HKV, D)).copy()
+    vc = load("value_cache_in.bin", np.uint16, (NB, BS, HKV, D)).copy()
+    oracle.reshape_and_cache(load("new_key.bin", np.uint16, (S, HKV, D)),
+                             load("new_value.bin", np.uint16, (S, HKV, D)), kc, vc, slots,
+                             block_size=BS, kv_dtype="bf16", cache_dtype="bf16")
+    assert np.array_equal(load("key_cache_out.bin", np.uint16, (NB, BS, HKV, D)), kc)
+    assert np.array_equal(load("value_cache_out.bin", np.uint16, (NB, BS, HKV, D)), vc)
+    ref = oracle.decode(load("query.bin", np.uint16, (S, H, D)), kc, vc, ref_table, ctx,
+                        scale=np.float32(0.08838834764831845), q_dtype="bf16",
+                        cache_dtype="bf16")
+    # bf16 output codes -> values: the code is the upper half of an fp32
+    got = (load("out.bin", np.uint16, (S, H, D)).astype(np.uint32) << 16).view(np.float32)
+    err = np.abs(got.astype(np.float64) - ref)
+    assert np.all(err <= 2e-3 + 1e-2 * np.abs(ref)), float(err.max())
