@@ -18,6 +18,13 @@ algorithmic bytes (K/V rows read once per kv-head + query + output + block
 table entries + context lengths) per step over the device time of the step.
 `--impl reference` times the CPU oracle (plain fp64 C) on the host cores
 instead, on a sample of the same workload sized so the run ends in minutes.
+
+The other rows of the path, one JSON line each:
+    --op prefill --workload chunk_llama7b|chunk_gqa70b|verify_gqa70b|chunk_gqa70b_fp8
+        multi-token query (TFLOP/s; against the tensor or HBM roofline,
+        whichever the work per byte makes binding)
+    --op copy_blocks    copy-on-write copies of 2048 blocks (GB/s read + write)
+    --op swap           512 blocks to a pinned host pool and back (GB/s)
 """
 from __future__ import annotations
 
