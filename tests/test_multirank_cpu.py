@@ -56,3 +56,17 @@ def test_job_throughput_counts_every_rank():
     one = bench.job_throughput_gbs(1, 1_000_000_000, 100.0)
     assert one == pytest.approx(10.0)
     assert bench.job_throughput_gbs(4, 1_000_000_000, 100.0) == pytest.approx(4 * one)
+
+
+def test_cpu_baseline_runs_on_one_core_and_on_all_cores():
+    """bench.py's cpu_baseline: the oracle single-threaded and on every host
+    core (spawned processes behind a barrier), here on the tiny workload and
+    on the shared-prefix one (whose samples become private copies)."""
+    import bench
+    from paged_kv_cache_448_b200 import workloads as wl
+    for cfg in (1, 5):
+        cb = bench.cpu_baseline(wl.spec(cfg, small=True), 0.5)
+        assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0
+        allc = cb["all_cores"]
+        assert "unavailable" not in allc, allc
+        assert allc["cores"] >= 1 and allc["value"] > 0
