@@ -98,9 +98,29 @@ def measured_tensor_peak():
     return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def decode_sources() -> list:
+    """The files the decode kernels are built from: the decode_*.cu units,
+    everything they include (transitively), and api.cu, which launches them."""
+    import re
+    csrc = os.path.join(ROOT, "paged_kv_cache_448_b200", "csrc")
+    todo = sorted(glob.glob(os.path.join(csrc, "decode_*.cu"))) + [os.path.join(csrc, "api.cu")]
+    seen = set()
+    while todo:
+        f = todo.pop()
+        if f in seen or not os.path.exists(f):
+            continue
+        seen.add(f)
+        with open(f, encoding="utf-8") as fh:
+            for inc in re.findall(r'^#include "([^"]+)"', fh.read(), re.M):
+                todo.append(os.path.join(csrc, inc))
+    return sorted(seen)
+
+
 def sources_digest() -> str:
+    """Digest of the decode kernels' sources: a recorded DRAM traffic figure
+    stands only for the exact sources it was taken on."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_448_b200", "csrc", "*"))):
+    for f in decode_sources():
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())

@@ -20,6 +20,11 @@
 // row's position, runs the online softmax in base 2 and accumulates
 // O += P V with P re-packed from the S accumulators as the A operand and V
 // transposed by ldmatrix.trans. Every wait is bounded by wall time.
+//
+// This kernel serves the shapes the tensor-memory kernel (prefill_tc.cu)
+// does not take: short chunks of few sequences (with the key range split
+// across CTAs and merged by paged_prefill_combine), fewer than 8 rows per
+// kv-head, and E4M3 caches with head_dim 64.
 #include <math_constants.h>
 
 #include "consumer_mma.cuh"

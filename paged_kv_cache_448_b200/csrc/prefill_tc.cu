@@ -5,24 +5,29 @@
 // the causal rule): rows cu[s] .. cu[s+1]-1 of the query are the last
 // positions p_i of sequence s and see its tokens t <= p_i.
 //
-// One CTA = 128 threads = 128 rows (row = one (query token, head of the
-// kv-head's group)), one row per thread and per tensor-memory lane:
-//  * Q (128 x D) is written once into shared memory, 128-byte swizzled, K-major;
-//  * K and V of 64 tokens per step arrive by TMA into a 2-stage ring (16-row
-//    boxes of one 128-byte segment each, so a stage is [segment][64 rows][128 B]);
-//  * thread 0 issues S = Q K^T (tcgen05.mma kind::f16, M=128, N=64, fp32 in
-//    tensor memory) and commits it to an mbarrier;
-//  * every thread loads its row of S from tensor memory, masks tokens after its
-//    position, and runs the base-2 online softmax with a lazily updated
-//    maximum (the running maximum moves only when a row's maximum grows by more
-//    than 8, i.e. probabilities stay below 2^8, so O rarely needs rescaling);
-//  * P (f16/bf16, bf16 as hi + lo parts) goes to shared memory and thread 0
-//    issues O += P V (M=128, N=D, K=64; V read MN-major), accumulating in
-//    tensor memory, then refills the stage once those MMAs completed;
-//  * the epilogue divides each row of O by its sum and stores it. When the
-//    key range is split (few CTAs), a CTA takes one part of its 16-token
-//    tiles and writes (max, sum) and its normalised O per row for the
-//    combine kernel, as the mma.sync kernel does.
+// A CTA holds NG row groups of 128 rows (row = one (query token, head of the
+// kv-head's group); NG = 2 once the chunks fill 256 rows) and 4 NG + 2 warps:
+//  * softmax warps, 4 per group: one row per thread and per tensor-memory
+//    lane. They write Q once into shared memory (128-byte swizzled, K-major),
+//    then per 64-token step load their row of S from tensor memory, mask
+//    tokens after the row's position, and run the base-2 online softmax with
+//    a lazily updated maximum (it moves only when a row's maximum grows by
+//    more than 8, so probabilities stay below 2^8 and O in tensor memory is
+//    rarely rescaled). They store P back into tensor memory over the S it
+//    came from (f16/bf16 pairs, bf16 as hi + lo parts) and post it;
+//  * the MMA warp (one thread) owns the tensor memory: per group two 64-column
+//    S buffers and D columns of O. It issues S = Q K^T of step k+1 into the
+//    buffer that step k-1 released, so S is computed under the softmax of
+//    step k, and O += P V of step k (A = P from tensor memory, V read
+//    MN-major) once the group posted P;
+//  * the TMA warp (one thread) loads K and V of 64 tokens per step into
+//    2-stage rings (16-row boxes of one 128-byte segment each, so a stage is
+//    [segment][64 rows][128 B]), K of step k ahead of V of step k-1, and
+//    refills a stage when the MMAs that read it completed.
+// The epilogue divides each row of O by its sum and stores it. When the key
+// range is split (few CTAs), a CTA takes one part of its 16-token tiles and
+// writes (max, sum) and its normalised O per row for the combine kernel, as
+// the mma.sync kernel does.
 // An E4M3 cache (head_dim 128: a 128-byte row) runs on kind::f8f6f4 with the
 // cache tiles as they arrive: Q goes to shared memory as E4M3 hi + lo parts
 // (q * 2^e = hi + lo, e a power of two per row that puts max |q| below 2^8,
@@ -30,9 +35,10 @@
 // 8-bit MMAs per K step; P (<= 2^8 under the lazy maximum) goes to tensor
 // memory as an E4M3 hi part and an E5M2 residual, so O += P V takes two
 // 8-bit MMAs with V read MN-major; the V scale applies in the epilogue.
-// Every wait is bounded by wall time; a wait that gives up is agreed on by the
-// whole CTA at the next barrier, which then drains its loads and MMAs, frees
-// its tensor memory and reports.
+// Every wait is bounded by wall time. A wait that gives up sets a shared
+// abort flag that ends the other roles' waits; the MMA warp lets its issued
+// MMAs and the TMA warp its issued loads complete (bounded) before the
+// tensor memory is freed, and the failure is recorded in the error word.
 #include <math_constants.h>
 
 #include <type_traits>
