@@ -70,3 +70,23 @@ def test_cpu_baseline_runs_on_one_core_and_on_all_cores():
         allc = cb["all_cores"]
         assert "unavailable" not in allc, allc
         assert allc["cores"] >= 1 and allc["value"] > 0
+
+
+def test_recorded_traffic_is_tied_to_the_decode_sources():
+    """roofline.traffic comes from profiles/traffic.json only for the workload
+    it was captured on and while the decode kernels' sources (decode_*.cu,
+    their headers, api.cu) still hash to the recorded digest."""
+    import json
+
+    import bench
+    names = {os.path.basename(f) for f in bench.decode_sources()}
+    assert {"decode_kernel.cuh", "api.cu", "decode_f16_f16.cu", "decode_reduce.cu"} <= names
+    assert "prefill_tc.cu" not in names and "copy_blocks.cu" not in names
+    assert bench.recorded_traffic("gqa70b_long") is None
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)["decode"]
+    got = bench.recorded_traffic(rec["workload"])
+    if rec["sources_sha256"] == bench.sources_digest():
+        assert got == rec["dram_read_bytes"] + rec["dram_write_bytes"]
+    else:
+        assert got is None
