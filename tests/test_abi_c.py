@@ -59,6 +59,23 @@ def test_allocator_from_c(c_output):
     assert int(c_output["oom"]) == _native.PA_ERR_OOM
 
 
+def test_header_links_from_cpp(tmp_path):
+    """The same client compiled as C++17: the header's extern "C" block gives
+    C linkage, so the library's symbols resolve from C++ too."""
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("no C++ compiler on this machine")
+    lib_dir = os.path.dirname(_native.LIB_PATH)
+    _native.lib()
+    exe = str(tmp_path / "abi_cpp_check")
+    subprocess.run([gxx, "-x", "c++", "-std=c++17", "-Wall", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "abi_c_check.c"),
+                    "-L", lib_dir, "-lpaged", f"-Wl,-rpath,{lib_dir}", "-o", exe],
+                   check=True, capture_output=True, text=True)
+    run = subprocess.run([exe], check=True, capture_output=True, text=True, timeout=60)
+    assert f"sha256_abc {hashlib.sha256(b'abc').hexdigest()}" in run.stdout
+
+
 def test_slots_and_sizes_from_c(c_output):
     # table rows {4, 9, -1} and {3, 8, 11}, block size 16
     assert c_output["slots"].split() == [str(4 * 16 + 0), str(9 * 16 + 1), str(11 * 16 + 8),
