@@ -359,3 +359,36 @@ def test_workspace_sizes_and_partition_plan():
     assert pk.decode_partition_tokens(32, 32, 32, 128, 16, 2048, 512) == 512
     # partitions are whole blocks
     assert pk.decode_partition_tokens(2, 8, 8, 128, 32, 4096, 300) == 320
+
+
+def test_slot_mapping_agrees_with_oracle_on_random_tables():
+    """Property check over random tables (including -1 padding and ids near
+    the int32 slot limit), positions (padding, past the table) and sequence
+    ids: the library succeeds exactly when the oracle does, with equal slots."""
+    from hypothesis import given, settings, strategies as st_
+
+    @settings(max_examples=300, deadline=None, derandomize=True)
+    @given(st_.data())
+    def check(data):
+        S = data.draw(st_.integers(1, 6))
+        MB = data.draw(st_.integers(1, 6))
+        bs = data.draw(st_.sampled_from([16, 32]))
+        ids = st_.one_of(st_.integers(-1, 50), st_.integers(2**31 // bs - 3, 2**31 // bs + 3))
+        table = np.array(data.draw(st_.lists(ids, min_size=S * MB, max_size=S * MB)),
+                         np.int32).reshape(S, MB)
+        n = data.draw(st_.integers(1, 12))
+        pos = np.array(data.draw(st_.lists(st_.integers(-2, MB * bs + 3), min_size=n,
+                                           max_size=n)), np.int32)
+        sid = np.array(data.draw(st_.lists(st_.integers(0, S - 1), min_size=n, max_size=n)),
+                       np.int32)
+        try:
+            ref = oracle.slot_mapping(table, pos, bs, sid)
+        except ValueError:
+            ref = None
+        if ref is None:
+            with pytest.raises(pk.PagedError):
+                pk.build_slot_mapping(table, pos, bs, sid)
+        else:
+            assert np.array_equal(pk.build_slot_mapping(table, pos, bs, sid), ref)
+
+    check()
