@@ -7,11 +7,13 @@ context tokens, 32 heads, head_dim 128, block_size 16, fp16 K/V, pool of
 into their slots, then paged decode attention over the whole context.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-    torchrun --nproc-per-node N bench.py --gpus N ...     (one process per GPU)
 
-Multi-GPU: every rank runs its own batch on its own GPU (sequences are
-independent; no collective on the data path): weak scaling, value = bytes of
-all ranks / max-over-ranks device time.
+Multi-GPU: one process per GPU. Under a launcher (torch.distributed.run sets
+WORLD_SIZE) each process is one rank; `--gpus N` started as a plain process
+starts the N ranks itself through torch.distributed.run. Every rank runs its
+own batch on its own GPU (sequences are independent; no collective on the
+data path, NCCL only for the barrier and the maximum of the times): weak
+scaling, value = bytes of all ranks / max-over-ranks device time.
 
 Rank 0 prints one JSON line. `value` is KV-read GB/s: the decode's
 algorithmic bytes (K/V rows read once per kv-head + query + output + block
@@ -307,7 +309,7 @@ def run_reference(args, sp, st):
         return
     import oracle
     oracle.build()
-    budget = 150.0
+    budget = 12.5 * args.cpu_seconds    # 150 s of oracle work at the default 12
     per_step = budget / max(1, args.steps + args.warmup)
     one_head = oracle_sample(sp, 1, 1)
     t_pair = time_oracle(*one_head)
@@ -541,6 +543,153 @@ def run_copy(args):
                       "clocks": clocks}), flush=True)
 
 
+def relaunch_command(gpus: int, port: int, argv: list) -> list:
+    """One process per GPU through torch.distributed.run on this node (the
+    form the multi-GPU contract uses), bounded by `timeout` as the last
+    resort; the process group itself has a short timeout."""
+    return ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run",
+            "--nnodes=1", f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1",
+            f"--master-port={port}", os.path.abspath(__file__)] + list(argv)
+
+
+def relaunch(args) -> int:
+    """`--gpus N` (N > 1) started as a plain process: start N ranks and pass
+    rank 0's line through."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    return subprocess.call(relaunch_command(args.gpus, port, sys.argv[1:]))
+
+
+def world_of(args) -> tuple:
+    """(world, rank, local rank) from the launcher's environment; the world
+    must be the --gpus the run was asked for."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but {world} rank(s) were started")
+    return world, rank, local
+
+
+def decode_line(args, sp: wl.Spec, st: wl.Structure, world: int, step_ms: float,
+                dec_ms: float, eff_part: int, launches_per_step: int, clocks: dict,
+                e2e=None) -> dict:
+    """The JSON line of a decode run from the max-over-ranks times: `value`
+    is every rank's bytes over the slowest rank's step time."""
+    dbytes = wl.decode_bytes(sp, st)
+    max_ctx = int(sp.context_lens.max())
+    split = eff_part < max_ctx
+    peak, peak_kind = measured_peaks()
+    value = job_throughput_gbs(world, dbytes, step_ms)
+    achieved = dbytes / (dec_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": sp.cache_dtype, "data": "synthetic",
+        "config": {"workload": workload_name(sp, st), "global_batch": sp.num_seqs * world,
+                   "seq_len": max_ctx, "parallelism": f"dp{world}",
+                   "partition_tokens": eff_part if split else None,
+                   "l2": f"inputs larger than L2: {wl.kv_bytes(sp) / 1e9:.2f} GB of K/V "
+                         "per step vs 126 MB L2; no flush"},
+        "pct_of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+        "tokens_per_s_per_layer": round(world * sp.num_seqs / (step_ms * 1e-3), 1),
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode" +
+                     (" + partition combine)" if split else ")"),
+                     "achieved": round(achieved, 2), "peak": peak,
+                     "peak_kind": f"{peak_kind} HBM copy GB/s", "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": recorded_traffic(sp.name),
+                     "algorithmic_bytes_per_launch": dbytes,
+                     "launch_ms": round(dec_ms, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e:
+        line["e2e"] = {"value": round(job_throughput_gbs(world, dbytes, e2e["ms_per_step"]), 2),
+                       "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
+                       "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e["ms_per_step"], 5),
+                       "copies": "one packed host-to-device copy of the step's inputs and one "
+                                 "device-to-host copy of its output per step, on a copy stream, "
+                                 "double-buffered so they overlap the neighbouring steps"}
+    return line
+
+
+class E2EStep:
+    """One decode step through the public API from pinned host memory: the
+    step's inputs (query, new K/V, block table, context lengths, slots) are
+    packed in one pinned buffer and uploaded by one copy, and the output is
+    read back by one copy, both on a copy stream. Two device buffers of each
+    alternate, so the upload of step k+1 and the read-back of step k run under
+    the decode of the neighbouring step."""
+
+    NAMES = ("query", "new_key", "new_value", "bt", "cl", "sl")
+
+    def __init__(self, host: dict, out_like, run_step, device):
+        import torch
+        offs, at = {}, 0
+        for k in self.NAMES:
+            offs[k] = at
+            at = (at + host[k].numel() * host[k].element_size() + 255) // 256 * 256
+        self.nbytes = at
+        self.pin_in = torch.empty(at, dtype=torch.uint8).pin_memory()
+        for k in self.NAMES:
+            t = host[k].contiguous().view(-1).view(torch.uint8)
+            self.pin_in[offs[k]:offs[k] + t.numel()].copy_(t)
+        self.h2d = sum(host[k].numel() * host[k].element_size() for k in self.NAMES)
+        self.dev_in = [torch.empty(at, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.views = []
+        for b in range(2):
+            v = {}
+            for k in self.NAMES:
+                n = host[k].numel() * host[k].element_size()
+                v[k] = self.dev_in[b][offs[k]:offs[k] + n].view(host[k].dtype).view(host[k].shape)
+            self.views.append(v)
+        self.out = [torch.empty_like(out_like) for _ in range(2)]
+        self.pin_out = [torch.empty(out_like.shape, dtype=out_like.dtype).pin_memory()
+                        for _ in range(2)]
+        self.d2h = out_like.numel() * out_like.element_size()
+        self.copy = torch.cuda.Stream(device=device)
+        self.compute = torch.cuda.current_stream(device)
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        self.uploaded, self.consumed, self.produced, self.read = (
+            [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()])
+        self.run_step = run_step
+        self.k = 0
+        for b in range(2):  # every buffer starts free
+            self.consumed[b].record(self.compute)
+            self.read[b].record(self.copy)
+
+    def __call__(self):
+        import torch
+        b = self.k & 1
+        with torch.cuda.stream(self.copy):
+            self.copy.wait_event(self.consumed[b])        # the decode of step k-2 read it
+            self.dev_in[b].copy_(self.pin_in, non_blocking=True)
+            self.uploaded[b].record(self.copy)
+        self.compute.wait_event(self.uploaded[b])
+        self.compute.wait_event(self.read[b])             # step k-2's output was read back
+        v = self.views[b]
+        self.run_step(v["query"], v["new_key"], v["new_value"], v["bt"], v["cl"], v["sl"],
+                      self.out[b])
+        self.consumed[b].record(self.compute)
+        self.produced[b].record(self.compute)
+        with torch.cuda.stream(self.copy):
+            self.copy.wait_event(self.produced[b])
+            self.pin_out[b].copy_(self.out[b], non_blocking=True)
+            self.read[b].record(self.copy)
+        self.k += 1
+
+    def finish(self):
+        """Make the compute stream wait for the last read-backs."""
+        for b in range(2):
+            self.compute.wait_event(self.read[b])
+
+
 def main():
     args = parse()
     if args.op == "prefill":
@@ -549,8 +698,11 @@ def main():
     if args.op in ("copy_blocks", "swap"):
         run_copy(args)
         return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args))
     sp = wl.spec(args.config)
     st = wl.structure(sp)
+    world, rank, local = world_of(args)
     if args.impl == "reference":
         run_reference(args, sp, st)
         return
@@ -559,9 +711,6 @@ def main():
     import torch.distributed as dist
     import paged_kv_cache_448_b200 as pk
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -625,80 +774,38 @@ def main():
     # e2e: the same step through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
-        pin = {k: d[k].cpu().pin_memory() for k in ("query", "new_key", "new_value")}
-        pin["bt"] = torch.from_numpy(st.block_tables).pin_memory()
-        pin["cl"] = torch.from_numpy(sp.context_lens).pin_memory()
-        pin["sl"] = torch.from_numpy(slots).pin_memory()
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        dq, dnk, dnv = (torch.empty_like(d[k]) for k in ("query", "new_key", "new_value"))
-        dbt, dcl, dsl = torch.empty_like(bt), torch.empty_like(cl), torch.empty_like(sl)
-        h2d = sum(t.numel() * t.element_size() for t in pin.values())
-        d2h = out_h.numel() * out_h.element_size()
+        host = {k: d[k].cpu() for k in ("query", "new_key", "new_value")}
+        host["bt"] = torch.from_numpy(st.block_tables)
+        host["cl"] = torch.from_numpy(sp.context_lens)
+        host["sl"] = torch.from_numpy(slots)
+        e2e_step = E2EStep(host, out, step, dev)
         e2e_steps = max(1, min(args.steps, 2000))
-
-        def e2e_step():
-            dq.copy_(pin["query"], non_blocking=True)
-            dnk.copy_(pin["new_key"], non_blocking=True)
-            dnv.copy_(pin["new_value"], non_blocking=True)
-            dbt.copy_(pin["bt"], non_blocking=True)
-            dcl.copy_(pin["cl"], non_blocking=True)
-            dsl.copy_(pin["sl"], non_blocking=True)
-            step(dq, dnk, dnv, dbt, dcl, dsl, out)
-            out_h.copy_(out, non_blocking=True)
-
         for _ in range(3):
             e2e_step()
+        e2e_step.finish()
         torch.cuda.synchronize()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         for _ in range(e2e_steps):
             e2e_step()
+        e2e_step.finish()
         b.record()
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = a.elapsed_time(b) / e2e_steps
-        e2e = {"ms_per_step": e2e_ms, "h2d": h2d, "d2h": d2h}
+        e2e = {"ms_per_step": a.elapsed_time(b) / e2e_steps, "h2d": e2e_step.h2d,
+               "d2h": e2e_step.d2h}
+        pk.decode_check(ws)
 
     # max over ranks
     step_ms, dec_ms, e2e_ms = max_over_ranks(
         [elapsed_ms / args.steps, dec_ms, e2e["ms_per_step"] if e2e else 0.0], world, dev)
+    if e2e:
+        e2e["ms_per_step"] = e2e_ms
 
     if rank == 0:
-        dbytes = wl.decode_bytes(sp, st)
-        peak, peak_kind = measured_peaks()
-        value = job_throughput_gbs(world, dbytes, step_ms)
-        achieved = dbytes / (dec_ms * 1e-3) / 1e9
-        traffic = recorded_traffic(sp.name)
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": sp.cache_dtype, "data": "synthetic",
-            "config": {"workload": workload_name(sp, st), "global_batch": sp.num_seqs * world,
-                       "seq_len": max_ctx, "parallelism": f"dp{world}",
-                       "partition_tokens": eff_part if split else None,
-                       "l2": f"inputs larger than L2: {wl.kv_bytes(sp) / 1e9:.2f} GB of K/V "
-                             "per step vs 126 MB L2; no flush"},
-            "pct_of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2),
-            "pct_of_measured_hbm": round(100 * value / world / peak, 2),
-            "tokens_per_s_per_layer": round(world * sp.num_seqs / (step_ms * 1e-3), 1),
-            "roofline": {"bound": "hbm", "kernel": "pa_decode (decode" +
-                         (" + partition combine)" if split else ")"),
-                         "achieved": round(achieved, 2), "peak": peak,
-                         "peak_kind": f"{peak_kind} HBM copy GB/s", "unit": "GB/s",
-                         "frac": round(achieved / peak, 4),
-                         "traffic": traffic,
-                         "algorithmic_bytes_per_launch": dbytes,
-                         "launch_ms": round(dec_ms, 5)},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks,
-        }
-        if e2e:
-            line["e2e"] = {"value": round(job_throughput_gbs(world, dbytes, e2e_ms), 2),
-                           "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
-                           "d2h_bytes_per_step": e2e["d2h"],
-                           "ms_per_step": round(e2e_ms, 5)}
+        line = decode_line(args, sp, st, world, step_ms, dec_ms, eff_part, launches_per_step,
+                           clocks, e2e)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(sp, args.cpu_seconds)
         print(json.dumps(line), flush=True)

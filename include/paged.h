@@ -168,12 +168,16 @@ PA_API pa_status pa_decode(void* out, const void* query,
  * than 32 MiB (pa_decode_workspace_size > 32 MiB) return PA_ERR_UNSUPPORTED
  * without launching; use pa_decode for them.
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture. Every call shares the one array and leaves its contents behind:
- * two calls whose kernels overlap on the GPU (e.g. on two streams) race on it
- * and give wrong results, so serialise them. Nothing in it needs clearing
- * between calls (every partial result is written before it is read). Table
- * errors are made harmless as in pa_decode but are not reported.
+ * device, with that device current, and again only if the device's context
+ * was replaced, e.g. after cudaDeviceReset); make that first call before any
+ * stream capture. Every call shares the one array and leaves its contents
+ * behind: two calls whose kernels overlap on the GPU (e.g. on two streams)
+ * race on it and give wrong results, so serialise them. Nothing in it needs
+ * clearing between calls: every partial result a call combines is written by
+ * that call, and a work unit whose pipeline wait gave up writes an empty
+ * partial (or zeros) rather than leaving another call's data to be combined.
+ * Table errors and waits that gave up are made harmless as in pa_decode and
+ * recorded in the array's error word: read them with pa_decode_noalloc_check.
  */
 PA_API pa_status pa_decode_noalloc(void* out, const void* query,
                     const void* key_cache, const void* value_cache,
@@ -184,6 +188,16 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* query,
                     float scale, pa_dtype q_dtype, pa_dtype cache_dtype,
                     const float* k_scale, const float* v_scale,
                     int32_t partition_tokens, pa_stream_t stream);
+
+/*
+ * pa_decode_check for pa_decode_noalloc: synchronises `stream`, then reads and
+ * clears the error word of this device's static scratch. Same results as
+ * pa_decode_check (PA_OK, PA_ERR_BAD_TABLE, or PA_ERR_CUDA for a wait that
+ * gave up, with the first failure's record in pa_last_error()). It allocates
+ * nothing either. The word collects every pa_decode_noalloc call on this
+ * device since the last check.
+ */
+PA_API pa_status pa_decode_noalloc_check(pa_stream_t stream);
 
 /*
  * Attention of several query tokens per sequence over the paged cache
@@ -267,7 +281,9 @@ PA_API int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads, i
  * Returns PA_OK, or PA_ERR_BAD_TABLE if a previous pa_decode or
  * pa_chunked_prefill on this workspace met an out-of-range table entry or
  * context length or a query longer than its context, or PA_ERR_CUDA (a wait
- * that gave up, or a CUDA error).
+ * that gave up, or a CUDA error). For a wait that gave up, pa_last_error()
+ * names the first failure: its site (decode tile, multi-token tile or step,
+ * FP8 decode tile), the CTA and the pipeline position where it stopped.
  */
 PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream);
 
@@ -276,6 +292,25 @@ PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream);
  * pa_decode never needs the rest of the workspace cleared.
  */
 PA_API pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * Test hook of the failure detection (no counterpart on the pages). Every
+ * pipeline wait inside the decode and multi-token kernels is bounded by wall
+ * time (1 s by default); a wait that runs out makes the kernel record the
+ * failure, set the timeout bit of the error word, let its own loads and
+ * tensor-core operations in flight complete, free its tensor memory and
+ * return, leaving zeros (or an empty partial result) for the rows it could
+ * not finish. Nothing faults, traps or hangs.
+ * This call makes the NEXT pa_decode, pa_decode_noalloc or pa_chunked_prefill
+ * made on the calling thread leave out the loads of one 16-token tile, `tile`
+ * (counted from 0 within the key range of the launch's first work unit:
+ * sequence 0, kv-head 0, first partition and query tile), and bound every wait
+ * of that launch by wait_limit_ns instead. The wait for the left-out tile then
+ * runs out and pa_decode_check / pa_decode_noalloc_check return PA_ERR_CUDA
+ * with the failure record. The request is used up by that call; tile < 0
+ * cancels a pending one. PA_ERR_INVALID_ARG if tile >= 0 and wait_limit_ns is 0.
+ */
+PA_API pa_status pa_inject_wait_timeout(int32_t tile, uint64_t wait_limit_ns);
 
 /*
  * Copy whole blocks: for each pair i, block block_pairs[2i] of the source

@@ -20,7 +20,8 @@ import numpy as np
 from . import _native
 from ._native import PagedError, check
 
-__all__ = ["reshape_and_cache", "decode", "decode_noalloc", "decode_workspace",
+__all__ = ["reshape_and_cache", "decode", "decode_noalloc", "decode_noalloc_check",
+           "inject_wait_timeout", "decode_workspace",
            "decode_workspace_size",
            "decode_partition_tokens", "decode_check", "chunked_prefill",
            "chunked_prefill_workspace", "chunked_prefill_workspace_size", "copy_blocks", "sha256", "block_hash",
@@ -124,8 +125,24 @@ def decode_noalloc(out, query, key_cache, value_cache, block_tables, context_len
 
 
 def decode_check(workspace, stream=None) -> None:
-    """Synchronise and raise PagedError if a decode on `workspace` met a bad table entry."""
+    """Synchronise and raise PagedError if a decode on `workspace` met a bad
+    table entry (PA_ERR_BAD_TABLE) or a pipeline wait gave up (PA_ERR_CUDA)."""
     check(_native.lib().pa_decode_check(_ptr(workspace), _stream_handle(stream)))
+
+
+def decode_noalloc_check(stream=None) -> None:
+    """decode_check for decode_noalloc: reads and clears the error word of the
+    library's static scratch on the current device (pa_decode_noalloc_check)."""
+    check(_native.lib().pa_decode_noalloc_check(_stream_handle(stream)))
+
+
+def inject_wait_timeout(tile: int, wait_limit_ns: int) -> None:
+    """Failure-detection test hook (pa_inject_wait_timeout): the next decode,
+    decode_noalloc or chunked_prefill on this thread leaves out the loads of
+    16-token tile `tile` of its first work unit and bounds every wait by
+    `wait_limit_ns`; the wait for that tile runs out and the check call
+    reports it. tile < 0 cancels."""
+    check(_native.lib().pa_inject_wait_timeout(int(tile), int(wait_limit_ns)))
 
 
 # ---------------------------------------------------------------- host side

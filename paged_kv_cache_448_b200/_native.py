@@ -29,6 +29,7 @@ SIGNATURES = [
                         _f32, _st, _st, _P, _P, _i32, _P, _sz, _P]),
     ("pa_decode_noalloc", _st, [_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i32,
                                 _i32, _i64, _f32, _st, _st, _P, _P, _i32, _P]),
+    ("pa_decode_noalloc_check", _st, [_P]),
     ("pa_chunked_prefill", _st, [_P, _P, _P, _i32, _i32, _P, _P, _P, _i32, _P, _i32, _i32,
                                  _i32, _i32, _i32, _i32, _i64, _f32, _st, _st, _P, _P, _P, _sz,
                                  _P]),
@@ -37,6 +38,7 @@ SIGNATURES = [
     ("pa_decode_partition_tokens", _i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
     ("pa_decode_check", _st, [_P, _P]),
     ("pa_workspace_init", _st, [_P, _sz, _P]),
+    ("pa_inject_wait_timeout", _st, [_i32, ctypes.c_uint64]),
     ("pa_copy_blocks", _st, [_P, _P, _P, _P, _P, _i32, _i64, _i64, _i64, _P, _P]),
     ("pa_sha256", _st, [_P, _i64, _P]),
     ("pa_block_hash", _st, [_P, _P, _i32, _P]),

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "decode_args.h"
+#include "device_common.cuh"
 #include "prefill_args.h"
 #include "paged.h"
 #include "status.h"
@@ -185,6 +186,22 @@ bool shape_supported(int32_t head_dim, int32_t block_size) {
   return (head_dim == 64 || head_dim == 128) && (block_size == 16 || block_size == 32);
 }
 
+// A failure-detection test's request for the next launch on this thread
+// (pa_inject_wait_timeout): the tile whose loads are left out, and the bound
+// of every wait. Taken, and cleared, by the next decode or multi-token launch.
+struct Injection {
+  int32_t tile = -1;
+  uint64_t limit_ns = 0;
+};
+thread_local Injection g_injection;
+
+void take_injection(int32_t* skip_tile, uint64_t* wait_limit_ns) {
+  *skip_tile = g_injection.tile;
+  *wait_limit_ns = g_injection.tile >= 0 && g_injection.limit_ns > 0 ? g_injection.limit_ns
+                                                                      : kWaitLimitNs;
+  g_injection = Injection{};
+}
+
 }  // namespace
 }  // namespace paged
 
@@ -256,16 +273,38 @@ PA_API pa_status pa_workspace_init(void* workspace, size_t workspace_bytes, pa_s
       "workspace_init");
 }
 
+PA_API pa_status pa_inject_wait_timeout(int32_t tile, uint64_t wait_limit_ns) {
+  clear_error();
+  if (tile >= 0 && wait_limit_ns == 0)
+    return fail(PA_ERR_INVALID_ARG, "inject_wait_timeout: wait limit must be positive");
+  g_injection.tile = tile < 0 ? -1 : tile;
+  g_injection.limit_ns = tile < 0 ? 0 : wait_limit_ns;
+  return PA_OK;
+}
+
 PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream) {
   clear_error();
   if (!workspace) return fail(PA_ERR_INVALID_ARG, "decode_check: null workspace");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int32_t word = 0;
+  // error word (int 0) and the first failure's record (ints 8..15)
+  int32_t head[16] = {};
   cudaError_t e = cudaStreamSynchronize(st);
-  if (e == cudaSuccess) e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(head, workspace, sizeof(head), cudaMemcpyDeviceToHost);
+  const int32_t word = head[kWordError];
   if (e == cudaSuccess && word != 0) e = cudaMemset(workspace, 0, 64);  // error + failure record
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode_check: %s", cudaGetErrorString(e));
-  if (word & kErrWaitTimeout) return fail(PA_ERR_CUDA, "decode: a pipeline wait timed out");
+  if (word & kErrWaitTimeout) {
+    const int32_t* r = head + kWordDiag;
+    const char* site = r[0] == kSiteTile       ? "decode tile"
+                       : r[0] == kSitePrefill  ? "multi-token (mma.sync) tile"
+                       : r[0] == kSiteTcStep   ? "multi-token (tcgen05) step"
+                       : r[0] == kSiteFp8Tile  ? "decode (tcgen05 FP8) tile"
+                                               : "unknown site";
+    return fail(PA_ERR_CUDA,
+                "decode: a pipeline wait timed out; first failure: site %d (%s), CTA (%d, %d, "
+                "%d), values %d %d %d %d",
+                r[0], site, r[1], r[2], r[3], r[4], r[5], r[6], r[7]);
+  }
   if (word & (kErrBadBlockId | kErrContextClipped | kErrQueryLonger))
     return fail(PA_ERR_BAD_TABLE, "decode: %s%s%s",
                 (word & kErrBadBlockId) ? "block-table entry outside the pool; " : "",
@@ -361,6 +400,7 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
   a.max_parts = plan.max_parts;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.block_size = block_size;
+  take_injection(&a.skip_tile, &a.wait_limit_ns);
 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   DecodeFn fn = nullptr;
@@ -584,6 +624,7 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
   a.q_tiles = plan.q_tiles;
   a.partition_tiles = plan.partition_tiles;
   a.max_parts = plan.max_parts;
+  take_injection(&a.skip_tile, &a.wait_limit_ns);
   if (plan.max_parts > 1) {
     const size_t rows = static_cast<size_t>(num_tokens) * num_heads * plan.max_parts;
     a.ws_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + kHeaderBytes);

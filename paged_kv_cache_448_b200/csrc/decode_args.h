@@ -18,9 +18,16 @@ enum : int32_t {
   kErrQueryLonger = 16,    // multi-token query: more query rows than context (rows are zeros)
 };
 
-// Failure sites recorded in the diagnostic words.
+// Failure sites recorded in the diagnostic words (the first word of the record).
 enum : int32_t {
-  kSiteTile = 4,        // a tile's loads never completed
+  kSiteTile = 4,        // decode: a tile's loads never completed
+                        //   (values: kv-head, sequence, partition, warp, warp's tile, its count)
+  kSitePrefill = 5,     // multi-token query on mma.sync: a tile or a stage release
+                        //   (values: CTA x, y, z, warp or step, tile, tiles, 0 / 1 = producer)
+  kSiteTcStep = 6,      // multi-token query on tcgen05: an MMA-warp wait
+                        //   (values: CTA x, y, z, K steps received, V steps received, steps, groups)
+  kSiteFp8Tile = 7,     // decode on tcgen05 (E4M3 cache): a role's wait
+                        //   (values: kv-head, sequence, partition, role, tile, tiles)
 };
 
 // Words of the workspace header (int32): the error word and, from kWordDiag,
@@ -49,6 +56,8 @@ struct DecodeArgs {
   int32_t max_parts;            // partitions per sequence in the launch (1 = single pass)
   float scale_log2;             // softmax scale * log2(e)
   int32_t block_size;           // tokens per cache block (a multiple of 16)
+  int32_t skip_tile;            // failure-detection test: tile of CTA (0,0,0) not loaded; -1 none
+  uint64_t wait_limit_ns;       // bound of every pipeline wait
 };
 
 // Per (q dtype, cache dtype) dispatchers, defined in decode_<q>_<c>.cu.

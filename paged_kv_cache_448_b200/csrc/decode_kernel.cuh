@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(NW_ * 32)
     const int32_t bid = ids[t / tpb];
     const int32_t row0 = bid >= 0 ? bid * a.block_size + (t % tpb) * TR : -TR;
     uint8_t* kt = my_stages + stage * STAGE;
+    if (skip_for_test(a.skip_tile, t)) return;
     mbar_arrive_expect_tx(&my_bars[stage], STAGE);
     tma_load_4d(kt, &kmap, &my_bars[stage], 0, row0, kvh, 0, policy);
     tma_load_4d(kt + T::BYTES, &vmap, &my_bars[stage], 0, row0, kvh, 0, policy);
@@ -161,7 +162,8 @@ __global__ void __launch_bounds__(NW_ * 32)
   int k = 0;
   for (; k < my_count; ++k) {
     const int stage = k % R;
-    if (!__all_sync(FULL, mbar_wait(&my_bars[stage], (k / R) & 1, &aborted))) break;
+    if (!__all_sync(FULL, mbar_wait(&my_bars[stage], (k / R) & 1, a.wait_limit_ns, &aborted)))
+      break;
     uint8_t* kt = my_stages + stage * STAGE;
     const int t = warp + k * NW;
     c.block(kt, kt + T::BYTES, max(0, min(TR, ctx - (tok0 + t * TR))), lane);
@@ -172,18 +174,32 @@ __global__ void __launch_bounds__(NW_ * 32)
     // A wait gave up (never expected): record it, let this warp's loads still
     // in flight land (bounded again), and stop the CTA after the barrier.
     if (lane == 0) {
-      aborted = 1;
+      // the record first: a warp stopped by the flag below must not take it
       record_failure(a.diag, kSiteTile, blockIdx.x, blockIdx.y, blockIdx.z, warp, k, my_count,
                      0);
+      aborted = 1;
     }
-    for (int kk = k; kk < min(k + R, my_count); ++kk) mbar_wait(&my_bars[kk % R], (kk / R) & 1);
+    for (int kk = k; kk < min(k + R, my_count); ++kk)
+      mbar_wait(&my_bars[kk % R], (kk / R) & 1, a.wait_limit_ns);
   }
 
   // Merge the warps through shared memory (the rings are idle: every issued
   // load has been waited for).
   __syncthreads();
+  const bool single = parts == 1;
+  const int64_t row0 = static_cast<int64_t>(s) * a.num_heads + kvh * G;
   if (aborted) {
+    // The unit's result is lost: leave zeros (single pass) or an empty
+    // partial that the combine kernel gives no weight, never stale data.
     if (threadIdx.x == 0) report(a.err, kErrWaitTimeout);
+    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+      const int g = idx / D, d = idx % D;
+      if (single) {
+        store_out(typename Consumer::QF{}, a.out, (row0 + g) * D + d, 0.f);
+      } else if (d == 0) {
+        a.ws_ml[(row0 + g) * a.max_parts + part] = make_float2(-CUDART_INF_F, 0.f);
+      }
+    }
     return;
   }
   float* mbuf = reinterpret_cast<float*>(smem);              // [NW][G][2]: m, l
@@ -191,9 +207,7 @@ __global__ void __launch_bounds__(NW_ * 32)
   c.finish(mbuf + warp * G * 2, obuf + warp * G * D, lane);
   __syncthreads();
 
-  const bool single = parts == 1;
   const float vs = a.v_scale ? a.v_scale[kvh] : 1.f;
-  const int64_t row0 = static_cast<int64_t>(s) * a.num_heads + kvh * G;
   for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
     const int g = idx / D, d = idx % D;
     float M = -CUDART_INF_F;

@@ -13,9 +13,10 @@
 
 namespace paged {
 
-// Wall-clock bound of every pipeline wait: far above any real TMA or
-// hand-over latency, yet a wait that can never complete ends in about a second
-// (the kernel then reports kErrWaitTimeout instead of hanging).
+// Default wall-clock bound of every pipeline wait (the launch passes it in
+// the kernel arguments): far above any real TMA or hand-over latency, yet a
+// wait that can never complete ends in about a second (the kernel then
+// reports kErrWaitTimeout instead of hanging).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
@@ -76,17 +77,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for phase `parity` of `bar` to complete. Gives up (returns false) after
-// kWaitLimitNs of wall time, or at once when *abort is set (another warp of the
+// limit_ns of wall time, or at once when *abort is set (another warp of the
 // CTA has given up already).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                           const volatile int* abort = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// True for the one load a failure-detection test asked to leave out: tile
+// `tile` of the launch's first CTA (skip_tile < 0: none). The wait for that
+// tile then runs out, which exercises the abort and drain path.
+__device__ __forceinline__ bool skip_for_test(int32_t skip_tile, int tile) {
+  return skip_tile >= 0 && tile == skip_tile && blockIdx.x == 0 && blockIdx.y == 0 &&
+         blockIdx.z == 0;
 }
 
 // First failure of a launch: where it happened and the state there, written

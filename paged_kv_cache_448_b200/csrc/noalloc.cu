@@ -8,6 +8,7 @@
 // allocation API at all. For them the scratch lives here, in a file-scope
 // __device__ array of fixed size that every GPU loading this library holds
 // until the process exits. No allocation call of any kind is made.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -27,26 +28,56 @@ __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+struct ScratchSlot {
+  void* ctx = nullptr;   // the context the address was resolved in
+  void* addr = nullptr;  // device address of g_decode_scratch there
+};
+ScratchSlot g_scratch[kMaxDevices];
 
-// Device address of g_decode_scratch on the current device; resolved once
-// per device, with that device current.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of g_decode_scratch on the current device. Resolved once
+// per device, with that device current, and again only when the device's
+// current context changed (a cudaDeviceReset destroys the old context and
+// with it the module holding the array).
 pa_status scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode_noalloc: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices)
     return fail(PA_ERR_UNSUPPORTED, "decode_noalloc: device index %d", dev);
+  auto current = [] {
+    CUcontext c = nullptr;
+    if (auto get = ctx_get_current()) get(&c);
+    return static_cast<void*>(c);
+  };
+  void* ctx = current();  // null before the runtime made its context current
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
+  ScratchSlot& slot = g_scratch[dev];
+  if (!slot.addr || !ctx || slot.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess || !p)
       return fail(PA_ERR_CUDA, "decode_noalloc: cudaGetSymbolAddress failed: %s",
                   cudaGetErrorString(e));
-    g_scratch_addr[dev] = p;
+    slot.addr = p;
+    slot.ctx = current();  // the lookup made the device's context current
   }
-  *out = g_scratch_addr[dev];
+  *out = slot.addr;
   return PA_OK;
 }
 
@@ -73,10 +104,21 @@ extern "C" PA_API pa_status pa_decode_noalloc(
   void* scratch = nullptr;
   pa_status st = scratch_address(&scratch);
   if (st != PA_OK) return st;
-  // Every partial result is written before it is read, so nothing in the
-  // scratch has to start at zero; the error word there is never reported.
+  // Every partial result the combine kernel reads is written by this call
+  // (a unit whose wait gave up writes an empty partial), so nothing in the
+  // scratch has to start at zero. Errors accumulate in the scratch's error
+  // word until pa_decode_noalloc_check reads and clears it.
   return pa_decode(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
                    context_lens, max_context_len, num_seqs, num_heads, num_kv_heads, head_dim,
                    block_size, num_blocks, scale, q_dtype, cache_dtype, k_scale, v_scale,
                    partition_tokens, scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" PA_API pa_status pa_decode_noalloc_check(pa_stream_t stream) {
+  using namespace paged;
+  clear_error();
+  void* scratch = nullptr;
+  pa_status st = scratch_address(&scratch);
+  if (st != PA_OK) return st;
+  return pa_decode_check(scratch, stream);
 }

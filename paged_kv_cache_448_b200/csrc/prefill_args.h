@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "decode_args.h"
+
 namespace paged {
 
 struct PrefillArgs {
@@ -31,10 +33,10 @@ struct PrefillArgs {
   int32_t max_parts;
   float* ws_o;                   // [T * H][max_parts][D] partial outputs (normalised)
   float2* ws_ml;                 // [T * H][max_parts] (max, sum) in base-2 units
+  int32_t skip_tile;             // failure-detection test: 16-token tile of CTA (0,0,0)
+                                 // whose loads are left out; -1 none
+  uint64_t wait_limit_ns;        // bound of every pipeline wait
 };
-
-// Failure site of a prefill wait that gave up.
-enum : int32_t { kSitePrefill = 5 };
 
 // Query tokens per CTA of the mma.sync kernel (64 rows = tokens x group).
 __host__ __device__ constexpr int prefill_tokens_per_cta(int group) { return 64 / group; }

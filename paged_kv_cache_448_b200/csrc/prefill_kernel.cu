@@ -165,6 +165,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
     }
     const int32_t row0 = bid >= 0 ? bid * a.block_size + ((tbase + t) * TR) % a.block_size : -TR;
     uint8_t* kt = smem + stage * STAGE;
+    if (skip_for_test(a.skip_tile, t)) return;
     mbar_arrive_expect_tx(&full[stage], STAGE);
     tma_load_4d(kt, &kmap, &full[stage], 0, row0, kvh, 0, policy);
     tma_load_4d(kt + T::BYTES, &vmap, &full[stage], 0, row0, kvh, 0, policy);
@@ -243,14 +244,14 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
       bool ok = true;
       for (int j = 0; j < kPrefillTps && ok; ++j) {
         const int tp = t0 - kPrefillTps + j;
-        ok = mbar_wait(&empty[tp % R], (tp / R) & 1, &aborted);
+        ok = mbar_wait(&empty[tp % R], (tp / R) & 1, a.wait_limit_ns, &aborted);
       }
       if (ok) {
         issue_step(k + kPrefillRs - 1);
       } else {
-        aborted = 1;
         record_failure(a.diag, kSitePrefill, blockIdx.x, blockIdx.y, blockIdx.z, k, t0, ntiles,
                        1);
+        aborted = 1;
       }
     }
     // ---- S = Q K^T over the step's tiles (16 tokens each)
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
       for (int nt = 0; nt < 2; ++nt)
         sacc[j][nt][0] = sacc[j][nt][1] = sacc[j][nt][2] = sacc[j][nt][3] = 0.f;
       if (tt >= ntiles) continue;
-      if (!__all_sync(FULL, mbar_wait(&full[tt % R], (tt / R) & 1, &aborted))) {
+      if (!__all_sync(FULL, mbar_wait(&full[tt % R], (tt / R) & 1, a.wait_limit_ns, &aborted))) {
         failed = true;
         break;
       }
@@ -423,15 +424,29 @@ __global__ void __launch_bounds__(kPrefillWarps * 32)
     // A wait gave up (never expected): record it and let the loads this CTA
     // issued land (bounded) before its shared memory goes away.
     if (lane == 0) {
-      aborted = 1;
+      // the record first: a warp stopped by the flag below must not take it
       record_failure(a.diag, kSitePrefill, blockIdx.x, blockIdx.y, blockIdx.z, warp, t, ntiles,
                      0);
+      aborted = 1;
       report(a.err, kErrWaitTimeout);
     }
     if (producer) {
       // issued so far: steps 0 .. min(k + RS - 1, nsteps - 1) at most
       const int last = min(ntiles, (min(k + kPrefillRs - 1, nsteps - 1) + 1) * kPrefillTps);
-      for (int tt = t; tt < last; ++tt) mbar_wait(&full[tt % R], (tt / R) & 1);
+      for (int tt = t; tt < last; ++tt) mbar_wait(&full[tt % R], (tt / R) & 1, a.wait_limit_ns);
+    }
+    // The rows' results are lost: leave zeros (whole key range) or an empty
+    // part that the combine kernel gives no weight, never stale data.
+    if (parts == 1) {
+      uint32_t* out32 = static_cast<uint32_t*>(a.out);
+      for (int j = 0; j < NO; ++j) {
+        if (v_lo) out32[(row_lo + j * 8 + 2 * c) / 2] = 0u;
+        if (v_hi) out32[(row_hi + j * 8 + 2 * c) / 2] = 0u;
+      }
+    } else if (c == 0) {
+      const int64_t pl = (row_lo / D) * a.max_parts + part, ph = (row_hi / D) * a.max_parts + part;
+      if (v_lo) a.ws_ml[pl] = make_float2(-CUDART_INF_F, 0.f);
+      if (v_hi) a.ws_ml[ph] = make_float2(-CUDART_INF_F, 0.f);
     }
     return;
   }

@@ -58,7 +58,6 @@ constexpr int kTcNT = 64;          // tokens per step
 constexpr int kTcStages = 2;
 constexpr uint32_t kTmemGroup = 256;  // tensor-memory columns per row group: S x 2, then O
 constexpr uint32_t kTmemO = 128;      // column of O within the group (S buffers at 0 and 64)
-constexpr int kSiteTc = 6;
 
 // NG row groups of 128 rows share each K/V step (NG = 2: 256 rows, eight
 // softmax warps, and two independent MMA streams per step).
@@ -162,6 +161,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   const int z = blockIdx.x % a.q_tiles, part = blockIdx.x / a.q_tiles;
   const int kvh = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint64_t lim = a.wait_limit_ns;
   if (tid == 0) {
     for (int r = 0; r < KR; ++r) {
       mbar_init(&kfull[r], 1);
@@ -297,6 +297,9 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
         uint64_t* bar = is_v ? &vfull[k % VR] : &kfull[k % KR];
         const CUtensorMap* map = is_v ? &vmap : &kmap;
         const int t_begin = (kbase + k) * (NT / TR), t_end = min(tend, t_begin + NT / TR);
+        if (!is_v && a.skip_tile >= t_begin - tbase && a.skip_tile < t_end - tbase &&
+            skip_for_test(a.skip_tile, a.skip_tile))
+          return;
         mbar_arrive_expect_tx(bar, static_cast<uint32_t>(NSEG * (t_end - t_begin) * TR * 128));
 #pragma unroll
         for (int j = 0; j < NT / TR; ++j) {
@@ -327,14 +330,14 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       for (int k = 0; ok && k <= nsteps; ++k) {
         if (k < nsteps) {
           load_ids(k, bid);
-          if (k >= KR) ok = mbar_wait(&kempty[k % KR], ((k - KR) / KR) & 1, &aborted);
+          if (k >= KR) ok = mbar_wait(&kempty[k % KR], ((k - KR) / KR) & 1, lim, &aborted);
           if (ok) {
             issue(k, bid, false);
             kk_issued = k + 1;
           }
         }
         if (ok && k >= 1) {
-          if (k - 1 >= VR) ok = mbar_wait(&vempty[(k - 1) % VR], ((k - 1 - VR) / VR) & 1, &aborted);
+          if (k - 1 >= VR) ok = mbar_wait(&vempty[(k - 1) % VR], ((k - 1 - VR) / VR) & 1, lim, &aborted);
           if (ok) {
             issue(k - 1, pbid, true);
             vv_issued = k;
@@ -350,9 +353,9 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       // before the CTA's shared memory goes away every issued load must have
       // landed (the last use of each stage; earlier ones completed already)
       for (int j = max(0, kk_issued - KR); j < kk_issued; ++j)
-        mbar_wait(&kfull[j % KR], (j / KR) & 1);
+        mbar_wait(&kfull[j % KR], (j / KR) & 1, lim);
       for (int j = max(0, vv_issued - VR); j < vv_issued; ++j)
-        mbar_wait(&vfull[j % VR], (j / VR) & 1);
+        mbar_wait(&vfull[j % VR], (j / VR) & 1, lim);
     }
   } else if (warp == kMma) {
     // ================= MMA issue (one thread) =================
@@ -365,7 +368,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       const uint64_t kd0 = tc::sw128_desc(sk(0), 16, 1024);
       const uint64_t vd0 = tc::sw128_desc(sv(0), NT * 128, 1024);
       auto issue_s = [&](int k) {  // S of step k for every group
-        if (!mbar_wait(&kfull[k % KR], (k / KR) & 1, &aborted)) return false;
+        if (!mbar_wait(&kfull[k % KR], (k / KR) & 1, lim, &aborted)) return false;
         k_waited = k + 1;
         tc::fence_after_sync();
         const uint64_t kd = kd0 + static_cast<uint64_t>(((k % KR) * C::KV_BYTES) >> 4);
@@ -401,16 +404,16 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
         // S and wrote P there, and O += P V of step k-1 read P
         if (k + 1 < nsteps) {
           for (int g = 0; ok && g < NG && k >= 1; ++g)
-            ok = mbar_wait(&p_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted) &&
-                 mbar_wait(&pv_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, &aborted);
+            ok = mbar_wait(&p_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted) &&
+                 mbar_wait(&pv_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted);
           ok = ok && issue_s(k + 1);
         }
-        if (ok) ok = mbar_wait(&vfull[k % VR], (k / VR) & 1, &aborted);
+        if (ok) ok = mbar_wait(&vfull[k % VR], (k / VR) & 1, lim, &aborted);
         if (ok) v_waited = k + 1;
         // O += P V of each group once its softmax warps wrote P of step k
         const uint64_t vd = vd0 + static_cast<uint64_t>(((k % VR) * C::KV_BYTES) >> 4);
         for (int g = 0; ok && g < NG; ++g) {
-          ok = mbar_wait(&p_bar[g][k & 1], (k >> 1) & 1, &aborted);
+          ok = mbar_wait(&p_bar[g][k & 1], (k >> 1) & 1, lim, &aborted);
           if (!ok) break;
           tc::fence_after_sync();
           // P of step k in tensor memory: the S buffer's columns 0-31 (and the
@@ -440,12 +443,12 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       if (!ok) {
         // A wait gave up (never expected): let this CTA's MMAs finish (bounded)
         // before its tensor and shared memory go away.
-        aborted = 1;
-        record_failure(a.diag, kSiteTc, blockIdx.x, blockIdx.y, blockIdx.z, k_waited, v_waited,
+        record_failure(a.diag, kSiteTcStep, blockIdx.x, blockIdx.y, blockIdx.z, k_waited, v_waited,
                        nsteps, NG);
+        aborted = 1;
         report(a.err, kErrWaitTimeout);
         tc::commit(&drain_bar);
-        mbar_wait(&drain_bar, 0);
+        mbar_wait(&drain_bar, 0, lim);
       }
     }
   } else {
@@ -460,7 +463,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
     float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int k = 0; ok && k < nsteps; ++k) {
-      ok = mbar_wait(&s_bar[g][k & 1], (k >> 1) & 1, &aborted);
+      ok = mbar_wait(&s_bar[g][k & 1], (k >> 1) & 1, lim, &aborted);
       if (!ok) break;
       tc::fence_after_sync();
       float x[NT];
@@ -494,7 +497,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       // O may be rescaled only once O += P V of step k-1 completed (rare: the
       // maximum moves lazily), otherwise that MMA keeps running under this softmax
       if (k >= 1 && rescale) {
-        ok = mbar_wait(&pv_bar[g][(k - 1) & 1], ((k - 1) >> 1) & 1, &aborted);
+        ok = mbar_wait(&pv_bar[g][(k - 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted);
         if (!ok) break;
         tc::fence_after_sync();
 #pragma unroll
@@ -538,7 +541,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       const int vrows = max(0, min(NT, kv_valid - tk0));
       if (vrows < NT) {
         uint8_t* vs = sv(k);
-        ok = mbar_wait(&vfull[k % VR], (k / VR) & 1, &aborted);  // the TMA writes come first
+        ok = mbar_wait(&vfull[k % VR], (k / VR) & 1, lim, &aborted);  // the TMA writes come first
         if (!ok) break;
         for (int i = rr; i < (NT - vrows) * NSEG * 8; i += kTcRows) {
           const int r = vrows + i / (NSEG * 8), sg = (i / 8) % NSEG, c = i % 8;
@@ -552,9 +555,19 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       if (lane == 0) mbar_arrive(&p_bar[g][k & 1]);
     }
     if (ok)
-      ok = mbar_wait(&pv_bar[g][(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, &aborted);
+      ok = mbar_wait(&pv_bar[g][(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, lim, &aborted);
     if (!ok) {
+      // The row's result is lost: leave zeros (whole key range) or an empty
+      // part that the combine kernel gives no weight, never stale data.
       aborted = 1;
+      if (valid) {
+        if (parts == 1) {
+          uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
+          for (int c = 0; c < D / 8; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          a.ws_ml[(row_off / D) * a.max_parts + part] = make_float2(-CUDART_INF_F, 0.f);
+        }
+      }
     } else {
       // ---- epilogue: out = O / l, rounded to the q dtype; or, for a part of
       // a split key range, (max, sum) and O / l in fp32 for the combine

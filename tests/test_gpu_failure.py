@@ -1,0 +1,150 @@
+"""Failure detection on the GPU without a fault: every pipeline wait of the
+decode and multi-token kernels is bounded by wall time. pa_inject_wait_timeout
+makes the next launch leave out the loads of one tile of its first CTA and
+bounds its waits by a short limit; the wait for that tile then runs out. The
+kernel must record the failure (site and CTA), set the timeout bit that the
+check call reports as PA_ERR_CUDA, let its loads (and, on tcgen05, its MMAs)
+in flight complete before its shared and tensor memory go away, and leave
+zeros (or an empty partial) for the rows it could not finish. Every other row
+must still match the oracle, and a clean call right after on the same stream
+must pass parity: the context stays usable.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_448_b200 as pk
+from paged_kv_cache_448_b200 import _native
+from paged_kv_cache_448_b200 import workloads as wl
+from gpu_helpers import GpuStep, assert_close, dev, f32, i32
+
+pytestmark = pytest.mark.gpu
+
+LIMIT_NS = 20_000_000  # 20 ms: far above any real load latency, keeps the test short
+
+
+def _expect_timeout(check, site):
+    with pytest.raises(pk.PagedError) as e:
+        check()
+    msg = str(e.value)
+    assert e.value.status == _native.PA_ERR_CUDA, msg
+    assert "timed out" in msg and f"site {site} " in msg and "CTA (0, 0, 0)" in msg, msg
+
+
+def _decode_step(G, cache, seed):
+    ctxs = [700, 33, 1500, 2, 0, 900]
+    D = 128
+    qdt = "bf16"
+    sp = wl.Spec("failure", len(ctxs), 2 * G, 2, D, 16, qdt, cache, 1.0 / math.sqrt(D),
+                 np.array(ctxs, np.int32), spare_blocks=4, seed=seed)
+    st = wl.structure(sp)
+    hd = wl.host_data(sp, st)
+    return GpuStep(sp, st, hd)
+
+
+@pytest.mark.parametrize("cache", ["bf16", "e4m3"])
+@pytest.mark.parametrize("G,part", [(1, 0), (2, 128), (4, 256), (8, 0)])
+def test_decode_wait_that_runs_out(G, part, cache):
+    g = _decode_step(G, cache, seed=50 + G)
+    g.reshape()
+    sp = g.sp
+    _, _, ref = oracle_ref(g)
+    ws = pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                             sp.block_size, g.max_ctx, part)
+    split = pk.decode_partition_tokens(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                                       sp.block_size, g.max_ctx, part) < g.max_ctx
+    g.out.fill_(float("nan"))
+    pk.inject_wait_timeout(3, LIMIT_NS)        # tile 3 of (kv-head 0, sequence 0, part 0)
+    pk.decode(g.out, g.q, g.kc, g.vc, g.bt, g.cl, g.max_ctx, sp.scale, k_scale=g.ks,
+              v_scale=g.vs, partition_tokens=part, workspace=ws)
+    _expect_timeout(lambda: pk.decode_check(ws), 4)
+    out = g.out_f64()
+    assert np.isfinite(out).all()
+    lost = np.zeros(out.shape[:2], bool)
+    lost[0, :G] = True                          # the rows of the unit that stopped
+    if not split:
+        assert (out[lost] == 0).all()
+    assert_close(out[~lost], ref[~lost], cache, "rows of the other units")
+    # the same call again, without the injection: parity, and a clean check
+    g.out.fill_(float("nan"))
+    pk.decode(g.out, g.q, g.kc, g.vc, g.bt, g.cl, g.max_ctx, sp.scale, k_scale=g.ks,
+              v_scale=g.vs, partition_tokens=part, workspace=ws)
+    pk.decode_check(ws)
+    assert_close(g.out_f64(), ref, cache, "clean call after the timeout")
+
+
+def oracle_ref(g):
+    from gpu_helpers import oracle_step
+    return oracle_step(g.sp, g.st, g.hd)
+
+
+def _prefill(ctxs, qlens, G, D, dt, seed, cache=None):
+    sp = wl.Spec("failure", len(ctxs), 2 * G, 2, D, 16, dt, cache or dt, 1.0 / math.sqrt(D),
+                 np.array(ctxs, np.int32), spare_blocks=3, seed=seed)
+    st = wl.structure(sp)
+    hd = wl.host_data(sp, st)
+    qlens = np.array(qlens, np.int32)
+    q = wl.prefill_queries_host(sp, qlens)
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    ref = oracle.chunked_prefill(q, hd.key_cache, hd.value_cache, st.block_tables,
+                                 sp.context_lens, cu, scale=np.float32(sp.scale),
+                                 q_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype,
+                                 k_scale=hd.k_scale, v_scale=hd.v_scale)
+    gq = dev(q, dt)
+    kc, vc = dev(hd.key_cache, sp.cache_dtype), dev(hd.value_cache, sp.cache_dtype)
+    ws = pk.chunked_prefill_workspace(sp.num_seqs, int(qlens.sum()), sp.num_heads,
+                                      sp.num_kv_heads, D, int(qlens.max()), int(max(ctxs)),
+                                      pk.dtype_code(kc))
+    out = torch.full_like(gq, float("nan"))
+
+    def call():
+        pk.chunked_prefill(out, gq, i32(cu), int(qlens.max()), kc, vc, i32(st.block_tables),
+                           i32(sp.context_lens), int(max(ctxs)), sp.scale,
+                           k_scale=f32(hd.k_scale), v_scale=f32(hd.v_scale), workspace=ws)
+    return sp, out, ws, call, ref
+
+
+@pytest.mark.parametrize("kernel,site", [("mma_sync", 5), ("tcgen05", 6)])
+@pytest.mark.parametrize("cache", ["f16", "e4m3"])
+def test_multi_token_wait_that_runs_out(kernel, site, cache):
+    """mma.sync: 4-token chunks (4 rows per kv-head); tcgen05: a 128-token
+    chunk (128 rows), whose MMA warp must drain its MMAs before the tensor
+    memory is freed."""
+    G, D = 1, 128
+    if kernel == "mma_sync":
+        ctxs, qlens = [300, 90, 41], [4, 4, 2]
+    else:
+        ctxs, qlens = [300, 150, 128], [128, 100, 7]
+    sp, out, ws, call, ref = _prefill(ctxs, qlens, G, D, "f16", seed=60 + site,
+                                      cache=None if cache == "f16" else "e4m3")
+    pk.inject_wait_timeout(5, LIMIT_NS)        # tile 5 of (sequence 0, kv-head 0, first tile)
+    call()
+    _expect_timeout(lambda: pk.decode_check(ws), site)
+    o = out.double().cpu().numpy()
+    assert np.isfinite(o).all()
+    # rows of the first CTA: the first query tokens of sequence 0, heads of kv-head 0
+    qt = 64 // G if kernel == "mma_sync" else 128 // G
+    lost = np.zeros(o.shape[:2], bool)
+    lost[:min(qt, qlens[0]), :G] = True
+    assert (o[lost] == 0).all()
+    assert_close(o[~lost], ref[~lost], cache, "rows of the other CTAs")
+    out.fill_(float("nan"))
+    call()
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), ref, cache, "clean call after the timeout")
+
+
+def test_injection_is_used_up_and_can_be_cancelled():
+    g = _decode_step(4, "bf16", seed=70)
+    g.reshape()
+    _, _, ref = oracle_ref(g)
+    pk.inject_wait_timeout(2, LIMIT_NS)
+    pk.inject_wait_timeout(-1, 0)               # cancelled: the next call is clean
+    g.decode(partition_tokens=0)
+    assert_close(g.out_f64(), ref, "bf16", "after a cancelled injection")
+    with pytest.raises(pk.PagedError) as e:
+        pk.inject_wait_timeout(1, 0)
+    assert e.value.status == _native.PA_ERR_INVALID_ARG

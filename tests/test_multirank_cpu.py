@@ -51,6 +51,98 @@ def test_two_ranks_agree_on_the_slowest_time_and_use_distinct_batches():
     assert res[0][1] != res[1][1]
 
 
+def _line_worker(rank, world, port, out):
+    """One rank of a decode run on CPU stubs: the real seeds, max-over-ranks
+    and line assembly of bench.py, with made-up device times."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import argparse
+
+        import bench
+        from paged_kv_cache_448_b200 import workloads as wl
+        sp = wl.spec(2)
+        st = wl.structure(sp)
+        args = argparse.Namespace(steps=10, warmup=3, gpus=world)
+        # rank 1 is the slower one
+        step_ms, dec_ms, e2e_ms = bench.max_over_ranks(
+            [0.20 + 0.05 * rank, 0.18 + 0.04 * rank, 0.25 + 0.01 * rank], world, "cpu")
+        e2e = {"ms_per_step": e2e_ms, "h2d": 1, "d2h": 2}
+        line = bench.decode_line(args, sp, st, world, step_ms, dec_ms, 1024, 3,
+                                 {"sm_mhz": None}, e2e) if rank == 0 else None
+        out.put((rank, bench.rank_seed(sp, rank), line))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_decode_line_counts_both_batches_over_the_slowest_rank():
+    import bench
+    from paged_kv_cache_448_b200 import workloads as wl
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_line_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in procs:
+        rank, seed, line = q.get(timeout=120)
+        res[rank] = (seed, line)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0][0] != res[1][0]                     # each rank its own batch
+    line = res[0][1]
+    sp = wl.spec(2)
+    nbytes = wl.decode_bytes(sp, wl.structure(sp))
+    assert line["n_gpus"] == 2 and line["config"]["global_batch"] == 2 * sp.num_seqs
+    assert line["config"]["parallelism"] == "dp2" and line["scaling"] == "weak"
+    assert line["ms_per_step"] == pytest.approx(0.25)
+    assert line["value"] == pytest.approx(2 * nbytes / 0.25e-3 / 1e9, rel=1e-3)
+    assert line["roofline"]["launch_ms"] == pytest.approx(0.22)
+    assert line["e2e"]["value"] == pytest.approx(2 * nbytes / 0.26e-3 / 1e9, rel=1e-3)
+    assert bench.job_throughput_gbs(2, nbytes, 0.25) == pytest.approx(line["value"], rel=1e-3)
+
+
+def test_gpus_n_starts_n_ranks_itself():
+    """`python bench.py --gpus 2` without a launcher starts two ranks through
+    torch.distributed.run; here on the reference arm, which needs no GPU:
+    exactly one JSON line (rank 0's), with n_gpus 2."""
+    import json
+    import subprocess
+    import sys
+
+    import bench
+    cmd = bench.relaunch_command(2, 12345, ["--gpus", "2"])
+    i = cmd.index("-m")
+    assert cmd[:4] == ["timeout", "-k", "60", "3600"]
+    assert cmd[i + 1] == "torch.distributed.run" and "--nproc-per-node=2" in cmd
+    assert cmd[-3].endswith("bench.py") and cmd[-2:] == ["--gpus", "2"]
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl",
+                        "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+                        "--cpu-seconds", "0.2"], capture_output=True, text=True, env=env,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
+
+
+def test_rank_count_must_match_gpus():
+    import argparse
+
+    import bench
+    os.environ["WORLD_SIZE"] = "3"
+    try:
+        with pytest.raises(SystemExit):
+            bench.world_of(argparse.Namespace(gpus=2))
+    finally:
+        del os.environ["WORLD_SIZE"]
+
+
 def test_job_throughput_counts_every_rank():
     import bench
     one = bench.job_throughput_gbs(1, 1_000_000_000, 100.0)
