@@ -403,11 +403,17 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
   take_injection(&a.skip_tile, &a.wait_limit_ns);
 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  DecodeFn fn = nullptr;
-  if (q_dtype == PA_F16) fn = fp8 ? decode_f16_e4m3 : decode_f16_f16;
-  else fn = fp8 ? decode_bf16_e4m3 : decode_bf16_bf16;
-  const int warps = plan.max_parts > 1 && plan.partition_tokens <= kNarrowTokens ? 2 : 4;
-  st = cuda_status(fn(a, kmap, vmap, head_dim, group, warps, cs), "decode");
+  if (fp8 && head_dim == 128) {
+    // E4M3 rows of 128 bytes: the tcgen05 kernel takes the tiles as stored
+    st = cuda_status(decode_fp8_tc(a, kmap, vmap, q_dtype == PA_F16 ? kF16 : kBF16, group, cs),
+                     "decode");
+  } else {
+    DecodeFn fn = nullptr;
+    if (q_dtype == PA_F16) fn = fp8 ? decode_f16_e4m3 : decode_f16_f16;
+    else fn = fp8 ? decode_bf16_e4m3 : decode_bf16_bf16;
+    const int warps = plan.max_parts > 1 && plan.partition_tokens <= kNarrowTokens ? 2 : 4;
+    st = cuda_status(fn(a, kmap, vmap, head_dim, group, warps, cs), "decode");
+  }
   if (st != PA_OK || plan.max_parts <= 1) return st;
   return cuda_status(launch_reduce(a, q_dtype, head_dim, cs), "decode combine");
 }

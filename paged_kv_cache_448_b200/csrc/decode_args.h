@@ -77,6 +77,11 @@ cudaError_t decode_bf16_e4m3(const DecodeArgs&, const CUtensorMap&, const CUtens
 
 cudaError_t launch_reduce(const DecodeArgs& a, int q_dtype, int head_dim, cudaStream_t stream);
 
+// Decode over an E4M3 cache with head_dim 128 on tcgen05 (tokens on M), any
+// query group up to 8; cudaErrorNotSupported otherwise.
+cudaError_t decode_fp8_tc(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                          int q_dtype, int group, cudaStream_t stream);
+
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
                                      void* value_cache, const int32_t* slot_mapping,
                                      int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,

@@ -107,32 +107,6 @@ __device__ __forceinline__ float2 unpack_q(uint32_t w) {
   return __half22float2(h);
 }
 
-// Four values -> E4M3 hi parts and 8-bit residuals (E4M3 or E5M2), four bytes
-// each in order. The values go through f16 (exact for the inputs here: bf16 /
-// f16 queries times a power of two, probabilities of at most 2^8); the
-// residual h - hi is exact in f16.
-template <bool LO_E5M2>
-__device__ __forceinline__ void split_fp8x4(float a, float b, float c, float d, uint32_t& hi,
-                                            uint32_t& lo) {
-  const __half2 h01 = __floats2half2_rn(a, b), h23 = __floats2half2_rn(c, d);
-  const __nv_fp8x2_storage_t hi01 = __nv_cvt_halfraw2_to_fp8x2(
-      *reinterpret_cast<const __half2_raw*>(&h01), __NV_SATFINITE, __NV_E4M3);
-  const __nv_fp8x2_storage_t hi23 = __nv_cvt_halfraw2_to_fp8x2(
-      *reinterpret_cast<const __half2_raw*>(&h23), __NV_SATFINITE, __NV_E4M3);
-  const __half2_raw b01 = __nv_cvt_fp8x2_to_halfraw2(hi01, __NV_E4M3);
-  const __half2_raw b23 = __nv_cvt_fp8x2_to_halfraw2(hi23, __NV_E4M3);
-  const __half2 r01 = __hsub2(h01, *reinterpret_cast<const __half2*>(&b01));
-  const __half2 r23 = __hsub2(h23, *reinterpret_cast<const __half2*>(&b23));
-  constexpr __nv_fp8_interpretation_t LO = LO_E5M2 ? __NV_E5M2 : __NV_E4M3;
-  const __nv_fp8x2_storage_t lo01 =
-      __nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r01), __NV_SATFINITE, LO);
-  const __nv_fp8x2_storage_t lo23 =
-      __nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r23), __NV_SATFINITE, LO);
-  hi = static_cast<uint32_t>(hi01) | (static_cast<uint32_t>(hi23) << 16);
-  lo = static_cast<uint32_t>(lo01) | (static_cast<uint32_t>(lo23) << 16);
-}
-
-
 template <class QF, class CF, int D, int G, int NG>
 __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
     paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap kmap,
@@ -269,7 +243,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const float2 f0 = unpack_q<QF>(w[2 * j]), f1 = unpack_q<QF>(w[2 * j + 1]);
-            split_fp8x4<false>(ldexpf(f0.x, e), ldexpf(f0.y, e), ldexpf(f1.x, e),
+            tc::split_fp8x4<false>(ldexpf(f0.x, e), ldexpf(f0.y, e), ldexpf(f1.x, e),
                                ldexpf(f1.y, e), hw[j], lw[j]);
           }
         }
@@ -515,7 +489,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
         uint32_t w[NT / 4], wl[NT / 4];
 #pragma unroll
         for (int i = 0; i < NT / 4; ++i)
-          split_fp8x4<true>(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3], w[i], wl[i]);
+          tc::split_fp8x4<true>(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3], w[i], wl[i]);
         const uint32_t t_p = t_grp + (k & 1) * NT + lane_base;
         tc::st16u(t_p, w);
         tc::st16u(t_p + 16, wl);

@@ -51,6 +51,24 @@ __device__ __forceinline__ constexpr uint32_t idesc_f8() {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same with the major-ness of A chosen as well (bit 15: A MN-major), for
+// an A operand whose M index runs along the rows in shared memory.
+template <int A_FMT, int B_FMT, int M, int N, bool A_MN_MAJOR, bool B_MN_MAJOR>
+__device__ __forceinline__ constexpr uint32_t idesc_f8_ab() {
+  return idesc_f8<A_FMT, B_FMT, M, N, B_MN_MAJOR>() | ((A_MN_MAJOR ? 1u : 0u) << 15);
+}
+
+// Shared-memory matrix descriptor of an operand without swizzle (layout 0):
+// 8 x 16-byte core matrices, rows of one core matrix 16 bytes apart. With
+// both offsets 128 bytes and 16 bytes of the MN index per row (an MN-major
+// operand N = 16 of 8-bit values), the operand is simply [K rows][16 bytes].
+__device__ __forceinline__ uint64_t plain_desc(const void* smem, uint32_t lbo_bytes,
+                                               uint32_t sbo_bytes) {
+  const uint64_t a = (smem_addr(smem) >> 4) & 0x3FFFu;
+  return a | (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
 // D (tensor memory) (+)= A . B, 8-bit operands (K = 32 per instruction), both
 // from shared memory.
 __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -152,6 +170,36 @@ __device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 8 / 16 consecutive fp32 columns of this thread's lane; the caller waits
+// (tcgen05.wait::ld) before using them.
+__device__ __forceinline__ void ld8_nowait(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void st8u(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+      : "memory");
+}
+
 // Two 32-column loads in flight before one wait (columns taddr .. taddr+63).
 __device__ __forceinline__ void ld64(uint32_t taddr, float (&v)[64]) {
   uint32_t r[64];
@@ -176,6 +224,31 @@ __device__ __forceinline__ void ld64(uint32_t taddr, float (&v)[64]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Four values -> E4M3 hi parts and 8-bit residuals (E4M3 or E5M2), four bytes
+// each in order. The values go through f16 (exact for the inputs here: bf16 /
+// f16 queries times a power of two, probabilities of at most 2^8); the
+// residual h - hi is exact in f16.
+template <bool LO_E5M2>
+__device__ __forceinline__ void split_fp8x4(float a, float b, float c, float d, uint32_t& hi,
+                                            uint32_t& lo) {
+  const __half2 h01 = __floats2half2_rn(a, b), h23 = __floats2half2_rn(c, d);
+  const __nv_fp8x2_storage_t hi01 = __nv_cvt_halfraw2_to_fp8x2(
+      *reinterpret_cast<const __half2_raw*>(&h01), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi23 = __nv_cvt_halfraw2_to_fp8x2(
+      *reinterpret_cast<const __half2_raw*>(&h23), __NV_SATFINITE, __NV_E4M3);
+  const __half2_raw b01 = __nv_cvt_fp8x2_to_halfraw2(hi01, __NV_E4M3);
+  const __half2_raw b23 = __nv_cvt_fp8x2_to_halfraw2(hi23, __NV_E4M3);
+  const __half2 r01 = __hsub2(h01, *reinterpret_cast<const __half2*>(&b01));
+  const __half2 r23 = __hsub2(h23, *reinterpret_cast<const __half2*>(&b23));
+  constexpr __nv_fp8_interpretation_t LO = LO_E5M2 ? __NV_E5M2 : __NV_E4M3;
+  const __nv_fp8x2_storage_t lo01 =
+      __nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r01), __NV_SATFINITE, LO);
+  const __nv_fp8x2_storage_t lo23 =
+      __nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r23), __NV_SATFINITE, LO);
+  hi = static_cast<uint32_t>(hi01) | (static_cast<uint32_t>(hi23) << 16);
+  lo = static_cast<uint32_t>(lo01) | (static_cast<uint32_t>(lo23) << 16);
 }
 
 // 2^x by the MUFU instruction (flushes subnormal results to zero, which the

@@ -96,6 +96,40 @@ def assert_close(gpu: np.ndarray, ref: np.ndarray, cache_dtype: str, what="", ou
                              f"gpu={gpu[i]!r} ref={ref[i]!r} (max {ulps:.3g} ulp)")
 
 
+GUARD = 4096            # bytes of sentinel before and after a guarded buffer
+SENTINEL = 0xA7
+
+
+class Guarded:
+    """A device buffer with GUARD sentinel bytes on either side, standing in
+    for an out-of-bounds checker: any stray write of a kernel just before or
+    after the buffer changes a sentinel. `t` is the buffer itself (aligned to
+    256 bytes within the allocation)."""
+
+    def __init__(self, shape, dtype, device="cuda", fill=None):
+        esz = torch.empty((), dtype=dtype).element_size()
+        n = int(np.prod(shape)) * esz
+        self.raw = torch.full((GUARD + n + GUARD,), SENTINEL, dtype=torch.uint8, device=device)
+        self.n = n
+        self.t = self.raw[GUARD:GUARD + n].view(dtype).view(shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, what=""):
+        head = self.raw[:GUARD]
+        tail = self.raw[GUARD + self.n:]
+        assert bool((head == SENTINEL).all()) and bool((tail == SENTINEL).all()), \
+            f"{what}: a write landed outside the buffer (guard bytes changed)"
+
+
+def guarded_workspace(nbytes, device="cuda"):
+    """A workspace of nbytes inside guard bytes, error word zeroed."""
+    g = Guarded((max(nbytes, 256),), torch.uint8, device=device)
+    g.t.fill_(0xFF)              # everything past the header starts as garbage
+    g.t[:256].zero_()
+    return g
+
+
 class GpuStep:
     """Device copies of a workload and the library calls of one decode step."""
 
@@ -111,7 +145,8 @@ class GpuStep:
         self.cl = i32(sp.context_lens, device)
         slots = pk.build_slot_mapping(st.block_tables, st.positions, sp.block_size)
         self.slots = i32(slots, device)
-        self.out = torch.empty_like(self.q)
+        self.out_g = Guarded(tuple(self.q.shape), self.q.dtype, device)
+        self.out = self.out_g.t
         self.max_ctx = int(sp.context_lens.max())
 
     def reshape(self):
@@ -123,13 +158,19 @@ class GpuStep:
         table error or a pipeline wait that gave up raises PagedError)."""
         sp = self.sp
         p = sp.partition_tokens if partition_tokens is None else partition_tokens
+        wsg = None
         if workspace is None:
-            workspace = pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads,
-                                            sp.head_dim, sp.block_size, self.max_ctx, p)
+            wsg = guarded_workspace(pk.decode_workspace_size(
+                sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size,
+                self.max_ctx, p))
+            workspace = wsg.t
         out = pk.decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, self.max_ctx,
                         sp.scale, k_scale=self.ks, v_scale=self.vs, partition_tokens=p,
                         workspace=workspace)
         pk.decode_check(workspace)
+        self.out_g.check("decode output")
+        if wsg is not None:
+            wsg.check("decode workspace")
         return out
 
     def out_f64(self) -> np.ndarray:

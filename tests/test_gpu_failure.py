@@ -60,7 +60,8 @@ def test_decode_wait_that_runs_out(G, part, cache):
     pk.inject_wait_timeout(3, LIMIT_NS)        # tile 3 of (kv-head 0, sequence 0, part 0)
     pk.decode(g.out, g.q, g.kc, g.vc, g.bt, g.cl, g.max_ctx, sp.scale, k_scale=g.ks,
               v_scale=g.vs, partition_tokens=part, workspace=ws)
-    _expect_timeout(lambda: pk.decode_check(ws), 4)
+    # an E4M3 cache with head_dim 128 runs on the tcgen05 kernel (site 7)
+    _expect_timeout(lambda: pk.decode_check(ws), 7 if cache == "e4m3" else 4)
     out = g.out_f64()
     assert np.isfinite(out).all()
     lost = np.zeros(out.shape[:2], bool)

@@ -13,24 +13,31 @@ import torch
 import oracle
 import paged_kv_cache_448_b200 as pk
 from paged_kv_cache_448_b200 import workloads as wl
-from gpu_helpers import assert_close, dev, f32, host_codes, i32
+from gpu_helpers import Guarded, assert_close, dev, f32, guarded_workspace, host_codes, i32
 
 pytestmark = pytest.mark.gpu
 
 
 def run_gpu(sp, st, hd, q, qlens, table=None, ctx=None):
+    """One pa_chunked_prefill call; its output and workspace sit inside guard
+    bytes that must be unchanged afterwards."""
     cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
     ctx = sp.context_lens if ctx is None else ctx
     table = st.block_tables if table is None else table
     gq = dev(q, sp.q_dtype)
-    out = torch.full_like(gq, float("nan"))
+    out_g = Guarded(tuple(gq.shape), gq.dtype, fill=float("nan"))
+    out = out_g.t
     kc, vc = dev(hd.key_cache, sp.cache_dtype), dev(hd.value_cache, sp.cache_dtype)
-    ws = pk.chunked_prefill_workspace(sp.num_seqs, int(qlens.sum()), sp.num_heads,
-                                      sp.num_kv_heads, sp.head_dim, int(qlens.max()),
-                                      int(np.max(ctx)), pk.dtype_code(kc))
+    ws_g = guarded_workspace(pk.chunked_prefill_workspace_size(
+        sp.num_seqs, int(qlens.sum()), sp.num_heads, sp.num_kv_heads, sp.head_dim,
+        int(qlens.max()), int(np.max(ctx)), pk.dtype_code(kc)))
+    ws = ws_g.t
     pk.chunked_prefill(out, gq, i32(cu), int(qlens.max()), kc, vc, i32(table), i32(ctx),
                        int(np.max(ctx)), sp.scale, k_scale=f32(hd.k_scale),
                        v_scale=f32(hd.v_scale), workspace=ws)
+    torch.cuda.synchronize()
+    out_g.check("multi-token output")
+    ws_g.check("multi-token workspace")
     return out, ws, cu
 
 
