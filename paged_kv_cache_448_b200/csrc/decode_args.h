@@ -28,6 +28,8 @@ enum : int32_t {
                         //   (values: CTA x, y, z, K steps received, V steps received, steps, groups)
   kSiteFp8Tile = 7,     // decode on tcgen05 (E4M3 cache): a role's wait
                         //   (values: kv-head, sequence, partition, role, tile, tiles)
+  kSiteTmTile = 8,      // multi-token query with the key tokens on M: a role's wait
+                        //   (values: CTA x, y, z, role, tile, tiles)
 };
 
 // Words of the workspace header (int32): the error word and, from kWordDiag,

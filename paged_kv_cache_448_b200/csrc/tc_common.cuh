@@ -39,6 +39,12 @@ __device__ __forceinline__ constexpr uint32_t idesc_f16() {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same with the major-ness of A chosen as well (bit 15: A MN-major).
+template <bool BF, int M, int N, bool A_MN_MAJOR, bool B_MN_MAJOR>
+__device__ __forceinline__ constexpr uint32_t idesc_f16_ab() {
+  return idesc_f16<BF, M, N, B_MN_MAJOR>() | ((A_MN_MAJOR ? 1u : 0u) << 15);
+}
+
 // Instruction descriptor of kind::f8f6f4 with fp32 accumulators; operand
 // formats 0 = E4M3, 1 = E5M2 (bits 7-9 for A, 10-12 for B), the other fields
 // as in idesc_f16.

@@ -108,26 +108,30 @@ def _prefill(ctxs, qlens, G, D, dt, seed, cache=None):
     return sp, out, ws, call, ref
 
 
-@pytest.mark.parametrize("kernel,site", [("mma_sync", 5), ("tcgen05", 6)])
-@pytest.mark.parametrize("cache", ["f16", "e4m3"])
-def test_multi_token_wait_that_runs_out(kernel, site, cache):
-    """mma.sync: 4-token chunks (4 rows per kv-head); tcgen05: a 128-token
-    chunk (128 rows), whose MMA warp must drain its MMAs before the tensor
-    memory is freed."""
-    G, D = 1, 128
-    if kernel == "mma_sync":
-        ctxs, qlens = [300, 90, 41], [4, 4, 2]
-    else:
+@pytest.mark.parametrize("kernel,cache,D,site", [
+    ("mma_sync", "f16", 64, 5), ("mma_sync", "e4m3", 128, 5),
+    ("keys_on_m", "f16", 128, 8), ("keys_on_m", "bf16", 128, 8),
+    ("tcgen05", "f16", 128, 6), ("tcgen05", "e4m3", 128, 6)])
+def test_multi_token_wait_that_runs_out(kernel, cache, D, site):
+    """mma.sync: 4-token chunks with head_dim 64, or over an E4M3 cache; keys
+    on M: the same short chunks over a 16-bit cache with head_dim 128;
+    tcgen05 rows on M: a 128-token chunk. The tcgen05 kernels' MMA warp must
+    drain its MMAs before the tensor memory is freed."""
+    G = 1
+    if kernel == "tcgen05":
         ctxs, qlens = [300, 150, 128], [128, 100, 7]
-    sp, out, ws, call, ref = _prefill(ctxs, qlens, G, D, "f16", seed=60 + site,
-                                      cache=None if cache == "f16" else "e4m3")
+    else:
+        ctxs, qlens = [300, 90, 41], [4, 4, 2]
+    dt = "bf16" if cache == "bf16" else "f16"
+    sp, out, ws, call, ref = _prefill(ctxs, qlens, G, D, dt, seed=60 + site,
+                                      cache=None if cache != "e4m3" else "e4m3")
     pk.inject_wait_timeout(5, LIMIT_NS)        # tile 5 of (sequence 0, kv-head 0, first tile)
     call()
     _expect_timeout(lambda: pk.decode_check(ws), site)
     o = out.double().cpu().numpy()
     assert np.isfinite(o).all()
     # rows of the first CTA: the first query tokens of sequence 0, heads of kv-head 0
-    qt = 64 // G if kernel == "mma_sync" else 128 // G
+    qt = {"mma_sync": 64 // G, "keys_on_m": qlens[0], "tcgen05": 128 // G}[kernel]
     lost = np.zeros(o.shape[:2], bool)
     lost[:min(qt, qlens[0]), :G] = True
     assert (o[lost] == 0).all()
