@@ -83,6 +83,8 @@ cudaError_t launch_reduce(const DecodeArgs& a, int q_dtype, int head_dim, cudaSt
 // query group up to 8; cudaErrorNotSupported otherwise.
 cudaError_t decode_fp8_tc(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           int q_dtype, int group, cudaStream_t stream);
+// kv-heads per CTA of that kernel (its TMA boxes span as many heads).
+int decode_fp8_tc_heads_per_cta(int num_kv_heads, int group);
 
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
                                      void* value_cache, const int32_t* slot_mapping,

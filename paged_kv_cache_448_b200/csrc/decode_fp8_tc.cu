@@ -23,7 +23,7 @@
 // the two O^T products (hi with E4M3, residual with E5M2) add into the same
 // accumulator. V's scale multiplies the output.
 //
-// A CTA is one work unit (kv-head, sequence, context partition) with six
+// A CTA is one work unit (kv-head, sequence, context partition) with nine
 // warps:
 //  * four softmax warps: thread i owns tensor-memory lane i, i.e. token i of
 //    the tile in S^T and dimension i of O^T. Per tile it loads its S^T row,
@@ -37,9 +37,9 @@
 //  * the MMA warp (one thread) owns the tensor memory: two 16-column S^T
 //    buffers and 16 columns of O^T. It issues S^T of tile k+1 before
 //    O^T += V^T P'^T of tile k, so S is computed under the softmax of tile k;
-//  * the TMA warp (one thread) loads K and V tiles into 3-stage rings (one
-//    16-row box per 16 tokens through the block table) and refills a stage
-//    when the MMAs that read it completed.
+//  * four TMA warps (one thread each, every fourth tile) load K and V tiles
+//    into 3-stage rings (one 16-row box per 16 tokens through the block
+//    table) and refill a stage when the MMAs that read it completed.
 // Every wait is bounded by wall time, and no barrier between the softmax
 // warps is an unbounded one: their exchanges go through mbarriers. A wait
 // that gives up records the failure, sets a shared abort flag that ends the
@@ -57,18 +57,18 @@
 namespace paged {
 namespace {
 
-constexpr int kTok = 128;                // tokens per tile (M of S^T)
-constexpr int kN = 16;                   // N of both products: 2G <= 16 query rows
+constexpr int kTok = 128;                // rows per tile (M of S^T): tokens x kv-heads
+constexpr int kN = 16;                   // N of O^T: query heads of the CTA, padded
 constexpr int kStages = 3;               // K and V ring depth
 constexpr int kTileBytes = kTok * 128;   // one K (or V) tile: 128 rows of 128 B
 constexpr int kSoftmaxWarps = 4;
-constexpr int kMmaWarp = 4, kTmaWarp = 5, kThreads = 192;
-constexpr uint32_t kTmemCols = 64;       // S^T x 2 (columns 0, 16), O^T (32)
-constexpr uint32_t kColO = 32;
+constexpr int kMmaWarp = 4, kTmaWarp = 5;  // TMA warps 5 .. 5 + kProducers - 1
+constexpr int kProducers = 4;               // tile k is loaded by TMA warp k % kProducers
+constexpr int kThreads = (kTmaWarp + kProducers) * 32;
 // shared memory from the 1024-aligned base
 constexpr int kOffV = kStages * kTileBytes;
 constexpr int kOffQ = 2 * kStages * kTileBytes;
-constexpr int kOffP = kOffQ + kN * 128;            // [2 buffers][hi, lo][128 tokens][16 B]
+constexpr int kOffP = kOffQ + 32 * 128;            // [2 buffers][hi, lo][128 rows][16 B]
 constexpr int kPBuf = 2 * kTok * 16;
 constexpr int kOffIds = kOffP + 2 * kPBuf;
 constexpr float kLazy = 8.f;             // base-2 margin of the lazy maximum
@@ -96,13 +96,21 @@ __device__ __forceinline__ float2 q_pair(uint32_t w) {
   return __half22float2(h);
 }
 
-template <class QF, int G>
+// H2 kv-heads per CTA (1 or 2): one TMA box carries 16 tokens of all H2
+// heads, [head][16 rows][128 B], so tile row i is head (i / 16) % H2, token
+// (i / (16 H2)) * 16 + i % 16 of the tile; the HG = H2 G query heads of the
+// CTA are the columns, and a row uses those of its own kv-head.
+template <class QF, int G, int H2>
 __global__ void __launch_bounds__(kThreads, 2)
     paged_decode_fp8_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
                                const __grid_constant__ CUtensorMap vmap) {
-  static_assert(G >= 1 && 2 * G <= kN, "query group");
-  constexpr int NL = G <= 4 ? 8 : 16;   // S^T / O^T columns a thread loads
-  constexpr int TR = kTileRows;         // 16 tokens per TMA box
+  constexpr int HG = G * H2;             // query heads of the CTA
+  static_assert(G >= 1 && (H2 == 1 || H2 == 2) && 2 * HG <= 16, "query group");
+  constexpr int NS = 16;                  // S^T columns: per query head hi and lo parts
+  constexpr uint32_t kTmemCols = 64;      // S^T x 2 (columns 0, 16), then O^T (32)
+  constexpr uint32_t kColO = 2 * NS;
+  constexpr int TT = kTok / H2;           // context tokens per tile
+  constexpr int TR = kTileRows;           // 16 tokens per TMA box
   constexpr unsigned FULL = 0xffffffffu;
 
   extern __shared__ uint8_t smem_raw[];
@@ -122,11 +130,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       s_full[2], s_free[2], p_full[2], p_free[2], red_bar[2], sum_bar, drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int aborted;
-  __shared__ float qscale_s[G];
-  __shared__ float red[2][kSoftmaxWarps][G];
-  __shared__ float lsum[kSoftmaxWarps][G];
+  __shared__ int last_k[kStages], last_v[kStages];  // last tile loaded into each stage
+  __shared__ float qscale_s[HG];
+  __shared__ float red[2][kSoftmaxWarps][HG];
+  __shared__ float lsum[kSoftmaxWarps][HG];
 
-  const int kvh = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
+  const int kvh = blockIdx.x * H2, s = blockIdx.y, part = blockIdx.z;  // first kv-head
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint64_t lim = a.wait_limit_ns;
   if (tid == 0) {
@@ -147,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
     aborted = 0;
+    for (int r = 0; r < kStages; ++r) last_k[r] = last_v[r] = -1;
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
   }
@@ -166,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int nlocal = min(b_begin + a.partition_blocks, nblk) - b_begin;
   const int tok0 = b_begin * a.block_size;
   const int ntok = max(0, min(ctx, (b_begin + nlocal) * a.block_size) - tok0);
-  const int ntiles = (ntok + kTok - 1) / kTok;
+  const int ntiles = (ntok + TT - 1) / TT;
 
   // Block ids of this unit -> shared memory, validated once.
   const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
@@ -178,12 +188,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     ids[i] = id;
   }
-  // Q' -> shared memory: one warp per query head; lane l holds dims 4l..4l+3
+  // Q' -> shared memory: one warp per query head n (of kv-head kvh + n / G);
+  // its hi and lo rows are 2G (n / G) + n % G and that + G; lane l holds
+  // dims 4l..4l+3
   if (warp < kSoftmaxWarps) {
-    for (int g = warp; g < G; g += kSoftmaxWarps) {
+    for (int n = warp; n < HG; n += kSoftmaxWarps) {
+      const int g = (n / G) * 2 * G + n % G;  // hi row
       const uint2 raw = *reinterpret_cast<const uint2*>(
           static_cast<const uint8_t*>(a.query) +
-          ((static_cast<int64_t>(s) * a.num_heads + kvh * G + g) * 128 + 4 * lane) * 2);
+          ((static_cast<int64_t>(s) * a.num_heads + kvh * G + n) * 128 + 4 * lane) * 2);
       const float2 f0 = q_pair<QF>(raw.x), f1 = q_pair<QF>(raw.y);
       float mq = fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y)));
 #pragma unroll
@@ -200,10 +213,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int c = lane >> 2, b = (lane & 3) * 4;
       *reinterpret_cast<uint32_t*>(sq + sw128_off(g, c) + b) = hi;
       *reinterpret_cast<uint32_t*>(sq + sw128_off(G + g, c) + b) = lo;
-      if (lane == 0) qscale_s[g] = a.scale_log2 * a.k_scale[kvh] * ldexpf(1.f, -e);
+      if (lane == 0) qscale_s[n] = a.scale_log2 * a.k_scale[kvh + n / G] * ldexpf(1.f, -e);
     }
-    for (int i = tid; i < (kN - 2 * G) * 8; i += kSoftmaxWarps * 32)
-      *reinterpret_cast<uint4*>(sq + sw128_off(2 * G + i / 8, i % 8)) = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < (NS - 2 * HG) * 8; i += kSoftmaxWarps * 32)
+      *reinterpret_cast<uint4*>(sq + sw128_off(2 * HG + i / 8, i % 8)) = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
   __syncthreads();  // barrier initialisation, ids and Q' visible to every thread
@@ -213,56 +226,66 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc::fence_after_sync();
   const uint32_t tmem = tmem_slot;
 
-  if (warp == kTmaWarp) {
-    // ================= TMA loads (one thread) =================
+  if (warp >= kTmaWarp) {
+    // ================= TMA loads (one thread per TMA warp) =================
+    // Issuing a tensor load costs its thread hundreds of cycles, and a tile is
+    // 16 boxes of 2 KB: the tiles are dealt to kProducers warps so that
+    // enough loads are issued per SM.
+    const int producer = warp - kTmaWarp;
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
       auto issue = [&](int k, bool is_v) {
         uint8_t* dst = is_v ? sv(k) : sk(k);
         uint64_t* bar = is_v ? &vfull[k % kStages] : &kfull[k % kStages];
         const CUtensorMap* map = is_v ? &vmap : &kmap;
-        const int u0 = k * kTok;
-        const int nsub = (min(kTok, ntok - u0) + TR - 1) / TR;  // boxes holding context tokens
+        const int u0 = k * TT;
+        const int nsub = (min(TT, ntok - u0) + TR - 1) / TR;  // boxes holding context tokens
         if (!is_v && a.skip_tile >= u0 / TR && a.skip_tile < u0 / TR + nsub &&
             skip_for_test(a.skip_tile, a.skip_tile))
           return;
-        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nsub * TR * 128));
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nsub * H2 * TR * 128));
         for (int j = 0; j < nsub; ++j) {
           const int u = u0 + j * TR;
           const int32_t bid = ids[u / a.block_size];
           const int32_t row0 = bid >= 0 ? bid * a.block_size + u % a.block_size : -TR;
-          tma_load_4d(dst + j * TR * 128, map, bar, 0, row0, kvh, 0, policy);
+          tma_load_4d(dst + j * H2 * TR * 128, map, bar, 0, row0, kvh, 0, policy);
         }
       };
       bool ok = true;
-      int k_issued = 0, v_issued = 0, k = 0;
-      for (; ok && k < ntiles; ++k) {
+      int k = producer;
+      for (; ok && k < ntiles; k += kProducers) {
         if (k >= kStages)
           ok = mbar_wait(&kempty[k % kStages], ((k - kStages) / kStages) & 1, lim, &aborted);
         if (!ok) break;
         issue(k, false);
-        k_issued = k + 1;
+        atomicMax(&last_k[k % kStages], k);
         if (k >= kStages)
           ok = mbar_wait(&vempty[k % kStages], ((k - kStages) / kStages) & 1, lim, &aborted);
         if (!ok) break;
         issue(k, true);
-        v_issued = k + 1;
+        atomicMax(&last_v[k % kStages], k);
       }
       if (!ok) {
         record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 0, k, ntiles, 0);
         aborted = 1;
         report(a.err, kErrWaitTimeout);
       }
-      // every issued load lands before the CTA's shared memory goes away
-      for (int j = max(0, k_issued - kStages); j < k_issued; ++j)
-        mbar_wait(&kfull[j % kStages], (j / kStages) & 1, lim);
-      for (int j = max(0, v_issued - kStages); j < v_issued; ++j)
-        mbar_wait(&vfull[j % kStages], (j / kStages) & 1, lim);
+    }
+    // Every issued load lands before the CTA's shared memory goes away: once
+    // all TMA warps stopped (their loops end in bounded time), the last load
+    // of each stage is waited for (earlier ones were consumed before the stage
+    // was reused).
+    asm volatile("bar.sync 1, %0;" ::"n"(kProducers * 32) : "memory");
+    if (producer == 0 && lane == 0) {
+      for (int r = 0; r < kStages; ++r) {
+        if (last_k[r] >= 0) mbar_wait(&kfull[r], (last_k[r] / kStages) & 1, lim);
+        if (last_v[r] >= 0) mbar_wait(&vfull[r], (last_v[r] / kStages) & 1, lim);
+      }
     }
   } else if (warp == kMmaWarp) {
     // ================= MMA issue (one thread) =================
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = tc::idesc_f8_ab<0, 0, kTok, kN, false, false>();
+      constexpr uint32_t IDESC_S = tc::idesc_f8_ab<0, 0, kTok, NS, false, false>();
       constexpr uint32_t IDESC_O_HI = tc::idesc_f8_ab<0, 0, kTok, kN, true, true>();
       constexpr uint32_t IDESC_O_LO = tc::idesc_f8_ab<0, 1, kTok, kN, true, true>();
       // descriptors computed once; a k-step or stage offset is added to the
@@ -282,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint64_t kd = kd0 + static_cast<uint64_t>(((kk_tile % kStages) * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 32 dims (bytes) per K step
-          tc::mma_f8(tmem + (kk_tile & 1) * kN, kd + 2 * kk, qd + 2 * kk, IDESC_S, kk > 0);
+          tc::mma_f8(tmem + (kk_tile & 1) * NS, kd + 2 * kk, qd + 2 * kk, IDESC_S, kk > 0);
         tc::commit(&s_full[kk_tile & 1]);
         tc::commit(&kempty[kk_tile % kStages]);
         return true;
@@ -321,12 +344,14 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else {
     // ================= softmax warps =================
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float m[G], l[G], qs[G];
+    const int h = (tid / TR) % H2;                        // this row's kv-head (of the CTA)
+    const int utok = (tid / (TR * H2)) * TR + tid % TR;   // and its token in the tile
+    float m[HG], l[HG], qs[HG];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      m[g] = -CUDART_INF_F;
-      l[g] = 0.f;
-      qs[g] = qscale_s[g];
+    for (int n = 0; n < HG; ++n) {
+      m[n] = -CUDART_INF_F;
+      l[n] = 0.f;
+      qs[n] = qscale_s[n];
     }
     bool ok = true;
     int k = 0;
@@ -334,52 +359,55 @@ __global__ void __launch_bounds__(kThreads, 2)
       ok = __all_sync(FULL, mbar_wait(&s_full[k & 1], (k >> 1) & 1, lim, &aborted));
       if (!ok) break;
       tc::fence_after_sync();
-      uint32_t r[NL];
-      if constexpr (NL == 8) tc::ld8_nowait(tmem + (k & 1) * kN + lane_base, r);
-      else tc::ld16_nowait(tmem + (k & 1) * kN + lane_base, r);
+      uint32_t r[NS];
+      tc::ld16_nowait(tmem + (k & 1) * NS + lane_base, r);
       tc::wait_ld();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[k & 1]);
-      const int vk = min(kTok, ntok - k * kTok);  // context tokens in this tile
-      const bool live = tid < vk;
-      float x[G];
+      const int vk = min(TT, ntok - k * TT);  // context tokens in this tile
+      const bool live = utok < vk;
+      // logits (base 2) of the query heads of this row's kv-head; -inf elsewhere
+      float x[HG];
 #pragma unroll
-      for (int g = 0; g < G; ++g)
-        x[g] = live ? (__uint_as_float(r[g]) + __uint_as_float(r[G + g])) * qs[g]
-                    : -CUDART_INF_F;
-      // the tile's maximum per head over the CTA
+      for (int n = 0; n < HG; ++n) {
+        const int c = (n / G) * 2 * G + n % G;
+        x[n] = live && n / G == h
+                   ? (__uint_as_float(r[c]) + __uint_as_float(r[c + G])) * qs[n]
+                   : -CUDART_INF_F;
+      }
+      // the tile's maximum per query head over the CTA
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const int mx = __reduce_max_sync(FULL, ord_of(x[g]));
-        if (lane == 0) red[k & 1][warp][g] = float_of(mx);
+      for (int n = 0; n < HG; ++n) {
+        const int mx = __reduce_max_sync(FULL, ord_of(x[n]));
+        if (lane == 0) red[k & 1][warp][n] = float_of(mx);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&red_bar[k & 1]);
       ok = __all_sync(FULL, mbar_wait(&red_bar[k & 1], (k >> 1) & 1, lim, &aborted));
       if (!ok) break;
-      float alpha[G];
+      float alpha[HG];
       bool rescale = false;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float tmax = red[k & 1][0][g];
+      for (int n = 0; n < HG; ++n) {
+        float tmax = red[k & 1][0][n];
 #pragma unroll
-        for (int w = 1; w < kSoftmaxWarps; ++w) tmax = fmaxf(tmax, red[k & 1][w][g]);
-        alpha[g] = 1.f;
-        if (tmax > m[g] + kLazy) {  // false while the head has seen nothing
-          alpha[g] = tc::ex2(m[g] - tmax);
-          m[g] = tmax;
+        for (int w = 1; w < kSoftmaxWarps; ++w) tmax = fmaxf(tmax, red[k & 1][w][n]);
+        alpha[n] = 1.f;
+        if (tmax > m[n] + kLazy) {  // false while the head has seen nothing
+          alpha[n] = tc::ex2(m[n] - tmax);
+          m[n] = tmax;
           rescale = true;
         }
       }
-      float p[8];
+      float p[16];
 #pragma unroll
-      for (int g = 0; g < 8; ++g) p[g] = 0.f;
+      for (int n = 0; n < 16; ++n) p[n] = 0.f;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float mu = m[g] == -CUDART_INF_F ? 0.f : m[g];
-        p[g] = tc::ex2(x[g] - mu);
-        l[g] = fmaf(l[g], alpha[g], p[g]);
+      for (int n = 0; n < HG; ++n) {
+        const float mu = m[n] == -CUDART_INF_F ? 0.f : m[n];
+        p[n] = tc::ex2(x[n] - mu);
+        l[n] = fmaf(l[n], alpha[n], p[n]);
       }
       // O^T may be rescaled only once O += P V of tile k-1 completed (rare:
       // the maximum moves lazily); the same for every thread of the CTA
@@ -387,14 +415,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         ok = __all_sync(FULL, mbar_wait(&p_free[(k - 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted));
         if (!ok) break;
         tc::fence_after_sync();
-        uint32_t o[NL];
-        if constexpr (NL == 8) tc::ld8_nowait(tmem + kColO + lane_base, o);
-        else tc::ld16_nowait(tmem + kColO + lane_base, o);
+        uint32_t o[16];
+        tc::ld16_nowait(tmem + kColO + lane_base, o);
         tc::wait_ld();
 #pragma unroll
-        for (int g = 0; g < G; ++g) o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
-        if constexpr (NL == 8) tc::st8u(tmem + kColO + lane_base, o);
-        else tc::st16u(tmem + kColO + lane_base, o);
+        for (int n = 0; n < HG; ++n) o[n] = __float_as_uint(__uint_as_float(o[n]) * alpha[n]);
+        tc::st16u(tmem + kColO + lane_base, o);
         tc::wait_st();
       }
       // P' buffer k & 1 is free once O += P V of tile k-2 completed
@@ -402,21 +428,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         ok = __all_sync(FULL, mbar_wait(&p_free[k & 1], ((k - 2) >> 1) & 1, lim, &aborted));
         if (!ok) break;
       }
-      uint32_t hw[4], lw[4];
-      tc::split_fp8x4<true>(p[0], p[1], p[2], p[3], hw[0], lw[0]);
-      if constexpr (G > 4) {
-        tc::split_fp8x4<true>(p[4], p[5], p[6], p[7], hw[1], lw[1]);
-      } else {
-        hw[1] = lw[1] = 0u;
-      }
-      hw[2] = hw[3] = lw[2] = lw[3] = 0u;
+      uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int q = 0; q < (HG + 3) / 4; ++q)
+        tc::split_fp8x4<true>(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3], hw[q], lw[q]);
       uint8_t* prow = sp + (k & 1) * kPBuf + tid * 16;
       *reinterpret_cast<uint4*>(prow) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4*>(prow + kTok * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       // V rows without context tokens (end of the unit) may hold anything,
       // even NaN codes, and 0 * NaN is NaN inside the MMA: clear them once
       // the tile's loads landed
-      if (vk < kTok) {
+      if (vk < TT) {
         ok = __all_sync(FULL, mbar_wait(&vfull[k % kStages], (k / kStages) & 1, lim, &aborted));
         if (!ok) break;
         if (!live) {
@@ -442,11 +464,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     // the partial sums over the CTA (every softmax warp posts its own)
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float v = l[g];
+    for (int n = 0; n < HG; ++n) {
+      float v = l[n];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-      if (lane == 0) lsum[warp][g] = v;
+      if (lane == 0) lsum[warp][n] = v;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sum_bar);
@@ -464,38 +486,32 @@ __global__ void __launch_bounds__(kThreads, 2)
       // The unit's result is lost: leave zeros (single pass) or an empty
       // partial that the combine kernel gives no weight, never stale data.
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        if (single) store_out(QF{}, a.out, (row0 + g) * 128 + tid, 0.f);
-        else if (tid == 0) a.ws_ml[(row0 + g) * a.max_parts + part] = make_float2(-CUDART_INF_F, 0.f);
+      for (int n = 0; n < HG; ++n) {
+        if (single) store_out(QF{}, a.out, (row0 + n) * 128 + tid, 0.f);
+        else if (tid == 0) a.ws_ml[(row0 + n) * a.max_parts + part] = make_float2(-CUDART_INF_F, 0.f);
       }
     } else {
-      // ---- epilogue: thread i holds dimension i of every head's O
-      float L[G];
+      // ---- epilogue: thread i holds dimension i of every query head's O
+      uint32_t o[16];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        L[g] = 0.f;
-#pragma unroll
-        for (int w = 0; w < kSoftmaxWarps; ++w) L[g] += lsum[w][g];
-      }
-      uint32_t o[NL];
-#pragma unroll
-      for (int i = 0; i < NL; ++i) o[i] = 0u;
+      for (int i = 0; i < 16; ++i) o[i] = 0u;
       if (ntiles > 0) {
         tc::fence_after_sync();
-        if constexpr (NL == 8) tc::ld8_nowait(tmem + kColO + lane_base, o);
-        else tc::ld16_nowait(tmem + kColO + lane_base, o);
+        tc::ld16_nowait(tmem + kColO + lane_base, o);
         tc::wait_ld();
       }
-      const float vs = a.v_scale[kvh];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float val = L[g] > 0.f ? __uint_as_float(o[g]) / L[g] * vs : 0.f;
+      for (int n = 0; n < HG; ++n) {
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSoftmaxWarps; ++w) L += lsum[w][n];
+        const float val = L > 0.f ? __uint_as_float(o[n]) / L * a.v_scale[kvh + n / G] : 0.f;
         if (single) {
-          store_out(QF{}, a.out, (row0 + g) * 128 + tid, val);
+          store_out(QF{}, a.out, (row0 + n) * 128 + tid, val);
         } else {
-          const int64_t pi = (row0 + g) * a.max_parts + part;
+          const int64_t pi = (row0 + n) * a.max_parts + part;
           a.ws_o[pi * 128 + tid] = val;
-          if (tid == 0) a.ws_ml[pi] = make_float2(m[g], L[g]);
+          if (tid == 0) a.ws_ml[pi] = make_float2(m[n], L);
         }
       }
     }
@@ -508,28 +524,40 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <class QF, int G>
+template <class QF, int G, int H2>
 cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                        cudaStream_t stream) {
-  if (a.partition_blocks > kMaxUnitBlocks) return cudaErrorNotSupported;
+  if (a.partition_blocks > kMaxUnitBlocks || a.num_kv_heads % H2 != 0)
+    return cudaErrorNotSupported;
   const size_t smem = 1024 + kOffIds + 4 * static_cast<size_t>(a.partition_blocks);
-  auto kern = paged_decode_fp8_tc_kernel<QF, G>;
+  auto kern = paged_decode_fp8_tc_kernel<QF, G, H2>;
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(a.num_kv_heads, a.num_seqs, a.max_parts), kThreads, smem, stream,
-                    a, kmap, vmap);
+  return launch_pdl(kern, dim3(a.num_kv_heads / H2, a.num_seqs, a.max_parts), kThreads, smem,
+                    stream, a, kmap, vmap);
 }
 
 }  // namespace
 
+// Two kv-heads per CTA (4 KB boxes: half the loads to issue per byte) while
+// their query heads fit the 16 columns of S^T's hi and lo parts.
+int decode_fp8_tc_heads_per_cta(int num_kv_heads, int group) {
+  return num_kv_heads % 2 == 0 && group <= 4 ? 2 : 1;
+}
+
 cudaError_t decode_fp8_tc(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           int q_dtype, int group, cudaStream_t stream) {
-#define PAGED_FP8TC(QF, g) \
-  if (group == g) return launch_one<QF, g>(a, kmap, vmap, stream);
+  const int h2 = decode_fp8_tc_heads_per_cta(a.num_kv_heads, group);
+#define PAGED_FP8TC(QF, g)                                           \
+  if (group == g)                                                    \
+    return h2 == 2 ? launch_one<QF, g, 2>(a, kmap, vmap, stream)     \
+                   : launch_one<QF, g, 1>(a, kmap, vmap, stream);
   if (q_dtype == kF16) {
-    PAGED_FP8TC(F16, 1) PAGED_FP8TC(F16, 2) PAGED_FP8TC(F16, 4) PAGED_FP8TC(F16, 8)
+    PAGED_FP8TC(F16, 1) PAGED_FP8TC(F16, 2) PAGED_FP8TC(F16, 4)
+    if (group == 8) return launch_one<F16, 8, 1>(a, kmap, vmap, stream);
   } else if (q_dtype == kBF16) {
-    PAGED_FP8TC(BF16, 1) PAGED_FP8TC(BF16, 2) PAGED_FP8TC(BF16, 4) PAGED_FP8TC(BF16, 8)
+    PAGED_FP8TC(BF16, 1) PAGED_FP8TC(BF16, 2) PAGED_FP8TC(BF16, 4)
+    if (group == 8) return launch_one<BF16, 8, 1>(a, kmap, vmap, stream);
   }
 #undef PAGED_FP8TC
   return cudaErrorNotSupported;

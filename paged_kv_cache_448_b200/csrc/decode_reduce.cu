@@ -38,7 +38,10 @@ __global__ void __launch_bounds__(128) paged_decode_reduce(const DecodeArgs a) {
   const float* o = a.ws_o + row * a.max_parts * D;
   for (int p = 0; p < parts; ++p) {
     const float2 v = ml[p];
-    const float w = v.x == -CUDART_INF_F ? 0.f : v.y * exp2f(v.x - M);
+    // a partition that saw no token (or gave up) has no weight, and its o
+    // was never written: it is not read
+    if (v.x == -CUDART_INF_F || !(v.y > 0.f)) continue;
+    const float w = v.y * exp2f(v.x - M);
     L += w;
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, o[p * D + lane + 32 * i], acc[i]);

@@ -539,7 +539,10 @@ __global__ void __launch_bounds__(128) paged_prefill_combine(const PrefillArgs a
   const float* op = a.ws_o + row * a.max_parts * D;
   for (int p = 0; p < parts; ++p) {
     const float2 v = ml[p];
-    const float w = v.x == -CUDART_INF_F ? 0.f : v.y * exp2f(v.x - M);
+    // a part that saw no token of this row (or gave up) has no weight, and
+    // its o may never have been written: it is not read
+    if (v.x == -CUDART_INF_F || !(v.y > 0.f)) continue;
+    const float w = v.y * exp2f(v.x - M);
     L += w;
 #pragma unroll
     for (int j = 0; j < PER; ++j) acc[j] = fmaf(w, op[p * D + lane + 32 * j], acc[j]);

@@ -280,16 +280,10 @@ def test_chunked_prefill_workspace_plan():
     n = pk.chunked_prefill_workspace_size(16, 16 * 8, 64, 8, 128, 8, 4096)
     rows = 16 * 8 * 64
     assert n > 256 and (n - 256) % (rows * (8 + 128 * 4)) < 256
-    # short chunks over a 16-bit cache with head_dim 128 (at most 64 rows per
-    # kv-head) run with the key tokens on M, one CTA per SM: 64 x 8 CTAs are
-    # below six waves of 148, so each key range of 32 tiles splits in two;
-    # the same for 2 rows per kv-head
-    n = pk.chunked_prefill_workspace_size(64, 64 * 8, 64, 8, 128, 8, 4096)
-    rows = 64 * 8 * 64
-    assert n > 256 and (n - 256) == 2 * rows * (8 + 128 * 4)
+    # short chunks whose tcgen05 CTAs fill a wave (64 x 8 >= 2 per SM) run
+    # there, unsplit; with 2 rows per kv-head they stay on mma.sync, split
+    assert pk.chunked_prefill_workspace_size(64, 64 * 8, 64, 8, 128, 8, 4096) == 256
     assert pk.chunked_prefill_workspace_size(16, 16 * 2, 32, 32, 128, 2, 4096) > 256
-    # with head_dim 64 they stay on the row-major kernels: 64 x 8 tcgen05
-    # CTAs fill a wave (>= 2 per SM), unsplit
     assert pk.chunked_prefill_workspace_size(64, 64 * 8, 64, 8, 64, 8, 4096) == 256
     assert pk.chunked_prefill_workspace_size(1, 1, 3, 2, 128, 1, 10) == 0   # H % Hkv != 0
     # an E4M3 cache takes tcgen05 only with head_dim 128: 4 sequences' long

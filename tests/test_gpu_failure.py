@@ -65,7 +65,9 @@ def test_decode_wait_that_runs_out(G, part, cache):
     out = g.out_f64()
     assert np.isfinite(out).all()
     lost = np.zeros(out.shape[:2], bool)
-    lost[0, :G] = True                          # the rows of the unit that stopped
+    # the rows of the unit that stopped: sequence 0, the query heads of kv-head 0
+    # (and of kv-head 1 where the tcgen05 FP8 kernel takes two kv-heads per CTA)
+    lost[0, :G * (2 if cache == "e4m3" and G <= 4 else 1)] = True
     if not split:
         assert (out[lost] == 0).all()
     assert_close(out[~lost], ref[~lost], cache, "rows of the other units")
@@ -109,14 +111,12 @@ def _prefill(ctxs, qlens, G, D, dt, seed, cache=None):
 
 
 @pytest.mark.parametrize("kernel,cache,D,site", [
-    ("mma_sync", "f16", 64, 5), ("mma_sync", "e4m3", 128, 5),
-    ("keys_on_m", "f16", 128, 8), ("keys_on_m", "bf16", 128, 8),
+    ("mma_sync", "f16", 64, 5), ("mma_sync", "f16", 128, 5), ("mma_sync", "e4m3", 128, 5),
     ("tcgen05", "f16", 128, 6), ("tcgen05", "e4m3", 128, 6)])
 def test_multi_token_wait_that_runs_out(kernel, cache, D, site):
-    """mma.sync: 4-token chunks with head_dim 64, or over an E4M3 cache; keys
-    on M: the same short chunks over a 16-bit cache with head_dim 128;
-    tcgen05 rows on M: a 128-token chunk. The tcgen05 kernels' MMA warp must
-    drain its MMAs before the tensor memory is freed."""
+    """mma.sync: 4-token chunks (4 rows per kv-head); tcgen05 rows on M: a
+    128-token chunk, whose MMA warp must drain its MMAs before the tensor
+    memory is freed."""
     G = 1
     if kernel == "tcgen05":
         ctxs, qlens = [300, 150, 128], [128, 100, 7]
@@ -131,7 +131,7 @@ def test_multi_token_wait_that_runs_out(kernel, cache, D, site):
     o = out.double().cpu().numpy()
     assert np.isfinite(o).all()
     # rows of the first CTA: the first query tokens of sequence 0, heads of kv-head 0
-    qt = {"mma_sync": 64 // G, "keys_on_m": qlens[0], "tcgen05": 128 // G}[kernel]
+    qt = {"mma_sync": 64 // G, "tcgen05": 128 // G}[kernel]
     lost = np.zeros(o.shape[:2], bool)
     lost[:min(qt, qlens[0]), :G] = True
     assert (o[lost] == 0).all()
