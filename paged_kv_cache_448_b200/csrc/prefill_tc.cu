@@ -331,6 +331,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
       for (int j = max(0, vv_issued - VR); j < vv_issued; ++j)
         mbar_wait(&vfull[j % VR], (j / VR) & 1, lim);
     }
+    __syncwarp();  // whole warps reach the CTA barrier below
   } else if (warp == kMma) {
     // ================= MMA issue (one thread) =================
     if (lane == 0) {
@@ -425,6 +426,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
         mbar_wait(&drain_bar, 0, lim);
       }
     }
+    __syncwarp();  // whole warps reach the CTA barrier below
   } else {
     // ================= softmax warps: one row per thread =================
     const int g = warp / 4;                      // row group

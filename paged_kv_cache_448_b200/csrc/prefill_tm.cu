@@ -254,6 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, v_issued - kStages); j < v_issued; ++j)
         mbar_wait(&vfull[j % kStages], (j / kStages) & 1, lim);
     }
+    __syncwarp();  // whole warps reach the CTA barrier below
   } else if (warp == kMmaWarp) {
     // ================= MMA issue (one thread) =================
     if (lane == 0) {
@@ -308,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&drain_bar, 0, lim);
       }
     }
+    __syncwarp();  // whole warps reach the CTA barrier below
   } else {
     // ================= softmax warps =================
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
