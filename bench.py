@@ -726,10 +726,11 @@ def main():
     sl = torch.from_numpy(slots).to(dev)
     out = torch.empty_like(d["query"])
     max_ctx = int(sp.context_lens.max())
+    cdt = pk.dtype_code(d["key_cache"])
     ws = pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
-                             sp.block_size, max_ctx, part, device=dev)
+                             sp.block_size, max_ctx, part, device=dev, cache_dtype=cdt)
     eff_part = pk.decode_partition_tokens(sp.num_seqs, sp.num_heads, sp.num_kv_heads,
-                                          sp.head_dim, sp.block_size, max_ctx, part)
+                                          sp.head_dim, sp.block_size, max_ctx, part, cdt)
     split = eff_part < max_ctx
     launches_per_step = 2 + (1 if split else 0)
 

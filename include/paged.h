@@ -260,21 +260,25 @@ PA_API size_t pa_chunked_prefill_workspace_size(int32_t num_seqs, int32_t num_to
                                                 int32_t max_context_len, pa_dtype cache_dtype);
 
 /*
- * Bytes of workspace pa_decode needs for these sizes on the current device
- * (the automatic partition choice depends on the device's SM count).
+ * Bytes of workspace pa_decode needs for these sizes and cache dtype on the
+ * current device (the automatic partition choice depends on the device's SM
+ * count and on the kernel the cache dtype and head_dim select).
  * Returns 0 for invalid sizes.
  */
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                 int32_t head_dim, int32_t block_size,
-                                int32_t max_context_len, int32_t partition_tokens);
+                                int32_t max_context_len, int32_t partition_tokens,
+                                pa_dtype cache_dtype);
 
 /*
- * The partition length (tokens) pa_decode will use for these sizes on the
- * current device; a result >= max_context_len means the single-pass path.
+ * The partition length (tokens) pa_decode will use for these sizes and cache
+ * dtype on the current device; a result >= max_context_len means the
+ * single-pass path.
  */
 PA_API int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                    int32_t head_dim, int32_t block_size,
-                                   int32_t max_context_len, int32_t partition_tokens);
+                                   int32_t max_context_len, int32_t partition_tokens,
+                                   pa_dtype cache_dtype);
 
 /*
  * Synchronises `stream`, reads and clears the error word of `workspace`.

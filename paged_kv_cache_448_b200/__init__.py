@@ -65,25 +65,30 @@ def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, *, k_sca
 
 
 def decode_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                            max_context_len, partition_tokens=0) -> int:
+                            max_context_len, partition_tokens=0,
+                            cache_dtype: int = _native.PA_F16) -> int:
+    """Partition length pa_decode uses (>= max_context_len: one pass);
+    cache_dtype is a pa_dtype code."""
     return int(_native.lib().pa_decode_partition_tokens(
         num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
-        partition_tokens))
+        partition_tokens, int(cache_dtype)))
 
 
 def decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                          max_context_len, partition_tokens=0) -> int:
+                          max_context_len, partition_tokens=0,
+                          cache_dtype: int = _native.PA_F16) -> int:
     return int(_native.lib().pa_decode_workspace_size(
         num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
-        partition_tokens))
+        partition_tokens, int(cache_dtype)))
 
 
 def decode_workspace(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
-                     partition_tokens=0, device="cuda", stream=None):
+                     partition_tokens=0, device="cuda", stream=None,
+                     cache_dtype: int = _native.PA_F16):
     """A device workspace (torch uint8) of the size pa_decode needs, error word zeroed."""
     import torch
     n = decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                              max_context_len, partition_tokens)
+                              max_context_len, partition_tokens, cache_dtype)
     ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
     check(_native.lib().pa_workspace_init(_ptr(ws), ws.numel(), _stream_handle(stream)))
     return ws
@@ -99,7 +104,8 @@ def decode(out, query, key_cache, value_cache, block_tables, context_lens, max_c
     NB, BS, Hkv = key_cache.shape[:3]
     if workspace is None:
         workspace = decode_workspace(S, H, Hkv, D, BS, max_context_len, partition_tokens,
-                                     device=query.device, stream=stream)
+                                     device=query.device, stream=stream,
+                                     cache_dtype=dtype_code(key_cache))
     check(_native.lib().pa_decode(
         _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
         block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, H, Hkv, D, BS, NB,

@@ -34,8 +34,8 @@ SIGNATURES = [
                                  _i32, _i32, _i32, _i32, _i64, _f32, _st, _st, _P, _P, _P, _sz,
                                  _P]),
     ("pa_chunked_prefill_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _st]),
-    ("pa_decode_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
-    ("pa_decode_partition_tokens", _i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    ("pa_decode_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _st]),
+    ("pa_decode_partition_tokens", _i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _st]),
     ("pa_decode_check", _st, [_P, _P]),
     ("pa_workspace_init", _st, [_P, _sz, _P]),
     ("pa_inject_wait_timeout", _st, [_i32, ctypes.c_uint64]),

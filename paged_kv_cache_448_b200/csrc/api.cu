@@ -109,8 +109,14 @@ struct Plan {
 
 constexpr int32_t kMaxParts = 65535;  // partitions per sequence (grid z extent)
 
+// fp8_tc: the E4M3 tcgen05 kernel (two CTAs per SM, two tiles of 128 tokens
+// in flight in each), which runs best on few, long units: measured on B200 on
+// the shared-prefix E4M3 workload (1 024 sequence x kv-head pairs of 1 100 to
+// 1 500 tokens), one pass 77 us against 98 / 120 / 175 us with partitions of
+// 1 024 / 512 / 256 tokens. It is cut into partitions only below one wave of
+// units. The other decode kernels (three CTAs per SM) want about four waves.
 Plan make_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
-               int32_t max_context_len, int32_t requested) {
+               int32_t max_context_len, int32_t requested, bool fp8_tc) {
   const int32_t blocks_max = std::max<int32_t>(1, (max_context_len + block_size - 1) / block_size);
   Plan p{};
   int32_t pb;
@@ -120,7 +126,7 @@ Plan make_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
     // Enough independent work units to keep every SM busy through the end of
     // the launch; otherwise cut the context into partitions (>= 256 tokens).
     const int64_t pairs = static_cast<int64_t>(num_seqs) * num_kv_heads;
-    const int64_t want = 4LL * sm_count() * 3;
+    const int64_t want = fp8_tc ? 2LL * sm_count() : 4LL * sm_count() * 3;
     pb = blocks_max;
     if (pairs < want && static_cast<int64_t>(blocks_max) * block_size > kMinAutoPartition) {
       const int32_t min_pb = std::max(1, kMinAutoPartition / block_size);
@@ -246,21 +252,23 @@ PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, void* 
 PA_API int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads,
                                           int32_t num_kv_heads, int32_t head_dim,
                                           int32_t block_size, int32_t max_context_len,
-                                          int32_t partition_tokens) {
+                                          int32_t partition_tokens, pa_dtype cache_dtype) {
   (void)num_heads;
-  (void)head_dim;
   if (num_seqs < 0 || num_kv_heads <= 0 || block_size <= 0 || max_context_len < 0) return 0;
-  Plan p = make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
+  Plan p = make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens,
+                     cache_dtype == PA_FP8_E4M3 && head_dim == 128);
   return p.max_parts <= 1 ? std::max(p.partition_tokens, max_context_len) : p.partition_tokens;
 }
 
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                        int32_t head_dim, int32_t block_size,
-                                       int32_t max_context_len, int32_t partition_tokens) {
+                                       int32_t max_context_len, int32_t partition_tokens,
+                                       pa_dtype cache_dtype) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
       max_context_len < 0)
     return 0;
-  Plan p = make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
+  Plan p = make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens,
+                     cache_dtype == PA_FP8_E4M3 && head_dim == 128);
   (void)num_kv_heads;
   return layout_for(p, num_seqs, num_heads, head_dim).total;
 }
@@ -357,8 +365,8 @@ PA_API pa_status pa_decode(void* out, const void* query, const void* key_cache,
       (k_scale && !aligned(k_scale, 4)) || (v_scale && !aligned(v_scale, 4)))
     return fail(PA_ERR_INVALID_ARG, "decode: misaligned pointer");
 
-  const Plan plan =
-      make_plan(num_seqs, num_kv_heads, block_size, max_context_len, partition_tokens);
+  const Plan plan = make_plan(num_seqs, num_kv_heads, block_size, max_context_len,
+                              partition_tokens, fp8 && head_dim == 128);
   if (num_seqs > 65535 || plan.max_parts > kMaxParts)
     return fail(PA_ERR_UNSUPPORTED, "decode: %d sequences x %d partitions exceed the grid",
                 num_seqs, plan.max_parts);

@@ -23,28 +23,32 @@
 // the two O^T products (hi with E4M3, residual with E5M2) add into the same
 // accumulator. V's scale multiplies the output.
 //
-// A CTA is one work unit (kv-head, sequence, context partition) with nine
-// warps:
-//  * four softmax warps: thread i owns tensor-memory lane i, i.e. token i of
-//    the tile in S^T and dimension i of O^T. Per tile it loads its S^T row,
-//    forms the G logits (masking tokens past the context), and the CTA takes
-//    each head's tile maximum (an ordered-integer warp reduction, then the
-//    four warps through shared memory behind an mbarrier). The running
-//    maximum moves only when a tile's maximum passes it by more than 8
-//    (base 2), so probabilities stay below 2^8 and O is rarely rescaled (in
-//    tensor memory, after the previous O += P V completed). Each thread keeps
-//    its own partial sums; they are added across the CTA at the end;
-//  * the MMA warp (one thread) owns the tensor memory: two 16-column S^T
-//    buffers and 16 columns of O^T. It issues S^T of tile k+1 before
-//    O^T += V^T P'^T of tile k, so S is computed under the softmax of tile k;
-//  * four TMA warps (one thread each, every fourth tile) load K and V tiles
+// A CTA is one work unit (kv-head, sequence, context partition). The time
+// of a tile is the latency of its softmax chain (S load, the CTA-wide tile
+// maximum, P store, then O += P V), so a CTA keeps two tiles in that chain at
+// once: two softmax groups take the tiles in turn, each with its own S
+// buffers, P buffer, running maxima, sums and O accumulator, merged at the
+// end like two parts of the context. Twelve warps:
+//  * two groups of four softmax warps: thread i of a group owns tensor-memory
+//    lane i, i.e. token i of its tiles in S^T and dimension i of its O^T. Per
+//    tile it loads its S^T row, forms the G logits (masking tokens past the
+//    context), and the group takes each head's tile maximum (an ordered-
+//    integer warp reduction, then its four warps through shared memory
+//    behind an mbarrier). The running maximum moves only when a tile's
+//    maximum passes it by more than 8 (base 2), so probabilities stay below
+//    2^8 and O is rarely rescaled (in tensor memory, after the group's
+//    previous O += P V completed). Each thread keeps its own partial sums;
+//  * the MMA warp (one thread) owns the tensor memory: per group two
+//    16-column S^T buffers and 16 columns of O^T. It issues S^T two tiles
+//    ahead (the next tile of the same group), then O^T += V^T P'^T of tile k;
+//  * three TMA warps (one thread each, every third tile) load K and V tiles
 //    into 3-stage rings (one 16-row box per 16 tokens through the block
 //    table) and refill a stage when the MMAs that read it completed.
-// Every wait is bounded by wall time, and no barrier between the softmax
-// warps is an unbounded one: their exchanges go through mbarriers. A wait
-// that gives up records the failure, sets a shared abort flag that ends the
-// other waits, and the roles drain their loads and MMAs before the tensor
-// memory is freed; the unit then leaves zeros (or an empty partial).
+// Every wait is bounded by wall time, and no barrier between softmax warps
+// is an unbounded one: their exchanges go through mbarriers. A wait that
+// gives up records the failure, sets a shared abort flag that ends the other
+// waits, and the roles drain their loads and MMAs before the tensor memory is
+// freed; the unit then leaves zeros (or an empty partial).
 #include <math_constants.h>
 
 #include <type_traits>
@@ -57,20 +61,24 @@
 namespace paged {
 namespace {
 
-constexpr int kTok = 128;                // rows per tile (M of S^T): tokens x kv-heads
-constexpr int kN = 16;                   // N of O^T: query heads of the CTA, padded
+constexpr int kTok = 128;                // tokens per tile (M of S^T)
+constexpr int kN = 16;                   // N of both products: hi and lo query rows, padded
 constexpr int kStages = 3;               // K and V ring depth
 constexpr int kTileBytes = kTok * 128;   // one K (or V) tile: 128 rows of 128 B
-constexpr int kSoftmaxWarps = 4;
-constexpr int kMmaWarp = 4, kTmaWarp = 5;  // TMA warps 5 .. 5 + kProducers - 1
-constexpr int kProducers = 4;               // tile k is loaded by TMA warp k % kProducers
+constexpr int kGroups = 2, kGroupWarps = 4;
+constexpr int kMmaWarp = kGroups * kGroupWarps;   // 8
+constexpr int kTmaWarp = kMmaWarp + 1;            // TMA warps 9 .. 9 + kProducers - 1
+constexpr int kProducers = 3;                     // tile k is loaded by TMA warp k % kProducers
 constexpr int kThreads = (kTmaWarp + kProducers) * 32;
+constexpr uint32_t kTmemCols = 128;      // per group 64: S^T x 2 (columns 0, 16), O^T (32)
+constexpr uint32_t kGroupCols = 64;
+constexpr uint32_t kColO = 32;
 // shared memory from the 1024-aligned base
 constexpr int kOffV = kStages * kTileBytes;
 constexpr int kOffQ = 2 * kStages * kTileBytes;
-constexpr int kOffP = kOffQ + 32 * 128;            // [2 buffers][hi, lo][128 rows][16 B]
+constexpr int kOffP = kOffQ + kN * 128;            // [group][hi, lo][128 tokens][16 B]
 constexpr int kPBuf = 2 * kTok * 16;
-constexpr int kOffIds = kOffP + 2 * kPBuf;
+constexpr int kOffIds = kOffP + kGroups * kPBuf;
 constexpr float kLazy = 8.f;             // base-2 margin of the lazy maximum
 
 // Byte offset of 16-byte chunk c of row r of a 128-byte-swizzled K-major
@@ -96,46 +104,41 @@ __device__ __forceinline__ float2 q_pair(uint32_t w) {
   return __half22float2(h);
 }
 
-// H2 kv-heads per CTA (1 or 2): one TMA box carries 16 tokens of all H2
-// heads, [head][16 rows][128 B], so tile row i is head (i / 16) % H2, token
-// (i / (16 H2)) * 16 + i % 16 of the tile; the HG = H2 G query heads of the
-// CTA are the columns, and a row uses those of its own kv-head.
-template <class QF, int G, int H2>
+template <class QF, int G>
 __global__ void __launch_bounds__(kThreads, 2)
     paged_decode_fp8_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
                                const __grid_constant__ CUtensorMap vmap) {
-  constexpr int HG = G * H2;             // query heads of the CTA
-  static_assert(G >= 1 && (H2 == 1 || H2 == 2) && 2 * HG <= 16, "query group");
-  constexpr int NS = 16;                  // S^T columns: per query head hi and lo parts
-  constexpr uint32_t kTmemCols = 64;      // S^T x 2 (columns 0, 16), then O^T (32)
-  constexpr uint32_t kColO = 2 * NS;
-  constexpr int TT = kTok / H2;           // context tokens per tile
-  constexpr int TR = kTileRows;           // 16 tokens per TMA box
+  static_assert(G >= 1 && 2 * G <= kN, "query group");
+  constexpr int NL = G <= 4 ? 8 : 16;   // S^T / O^T columns a thread loads
+  constexpr int TR = kTileRows;         // 16 tokens per TMA box
   constexpr unsigned FULL = 0xffffffffu;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sq = smem + kOffQ;
-  uint8_t* sp = smem + kOffP;
   int32_t* ids = reinterpret_cast<int32_t*>(smem + kOffIds);
   auto sk = [&](int k) { return smem + (k % kStages) * kTileBytes; };
   auto sv = [&](int k) { return smem + kOffV + (k % kStages) * kTileBytes; };
+  auto sp = [&](int g) { return smem + kOffP + g * kPBuf; };
   // kfull/vfull: a tile's boxes landed; kempty/vempty: the MMAs reading the
-  // stage completed; s_full[b]: S^T buffer b computed; s_free[b]: the softmax
-  // warps read it; p_full[b]: P' buffer b written (and O rescaled);
-  // p_free[b]: O += P V that read it completed; red_bar[b]: the four warps'
-  // tile maxima posted; sum_bar: their partial sums posted.
+  // stage completed. Per group g: s_full[g][b] S^T buffer b computed;
+  // s_free[g][b] the group read it; p_full[g] the group wrote P' (and
+  // rescaled O); p_free[g] O += P V that read it completed; red_bar[g][b] the
+  // group's tile maxima posted; sum_bar[g] its partial sums posted;
+  // merge_bar the second group's result posted for the first.
   __shared__ uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages],
-      s_full[2], s_free[2], p_full[2], p_free[2], red_bar[2], sum_bar, drain_bar;
+      s_full[kGroups][2], s_free[kGroups][2], p_full[kGroups], p_free[kGroups],
+      red_bar[kGroups][2], sum_bar[kGroups], merge_bar, drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int aborted;
   __shared__ int last_k[kStages], last_v[kStages];  // last tile loaded into each stage
-  __shared__ float qscale_s[HG];
-  __shared__ float red[2][kSoftmaxWarps][HG];
-  __shared__ float lsum[kSoftmaxWarps][HG];
+  __shared__ float qscale_s[G];
+  __shared__ float red[kGroups][2][kGroupWarps][G];
+  __shared__ float lsum[kGroups][kGroupWarps][G];
+  __shared__ float merge_ml[2][G];                   // second group: (max, sum) per head
 
-  const int kvh = blockIdx.x * H2, s = blockIdx.y, part = blockIdx.z;  // first kv-head
+  const int kvh = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint64_t lim = a.wait_limit_ns;
   if (tid == 0) {
@@ -145,14 +148,17 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&vfull[r], 1);
       mbar_init(&vempty[r], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], kSoftmaxWarps);
-      mbar_init(&p_full[b], kSoftmaxWarps);
-      mbar_init(&p_free[b], 1);
-      mbar_init(&red_bar[b], kSoftmaxWarps);
+    for (int g = 0; g < kGroups; ++g) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&s_full[g][b], 1);
+        mbar_init(&s_free[g][b], kGroupWarps);
+        mbar_init(&red_bar[g][b], kGroupWarps);
+      }
+      mbar_init(&p_full[g], kGroupWarps);
+      mbar_init(&p_free[g], 1);
+      mbar_init(&sum_bar[g], kGroupWarps);
     }
-    mbar_init(&sum_bar, kSoftmaxWarps);
+    mbar_init(&merge_bar, kGroupWarps);
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
     aborted = 0;
@@ -176,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int nlocal = min(b_begin + a.partition_blocks, nblk) - b_begin;
   const int tok0 = b_begin * a.block_size;
   const int ntok = max(0, min(ctx, (b_begin + nlocal) * a.block_size) - tok0);
-  const int ntiles = (ntok + TT - 1) / TT;
+  const int ntiles = (ntok + kTok - 1) / kTok;
 
   // Block ids of this unit -> shared memory, validated once.
   const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
@@ -188,15 +194,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     ids[i] = id;
   }
-  // Q' -> shared memory: one warp per query head n (of kv-head kvh + n / G);
-  // its hi and lo rows are 2G (n / G) + n % G and that + G; lane l holds
-  // dims 4l..4l+3
-  if (warp < kSoftmaxWarps) {
-    for (int n = warp; n < HG; n += kSoftmaxWarps) {
-      const int g = (n / G) * 2 * G + n % G;  // hi row
+  // Q' -> shared memory: one warp per query head; lane l holds dims 4l..4l+3
+  if (warp < kGroups * kGroupWarps) {
+    for (int g = warp; g < G; g += kGroups * kGroupWarps) {
       const uint2 raw = *reinterpret_cast<const uint2*>(
           static_cast<const uint8_t*>(a.query) +
-          ((static_cast<int64_t>(s) * a.num_heads + kvh * G + n) * 128 + 4 * lane) * 2);
+          ((static_cast<int64_t>(s) * a.num_heads + kvh * G + g) * 128 + 4 * lane) * 2);
       const float2 f0 = q_pair<QF>(raw.x), f1 = q_pair<QF>(raw.y);
       float mq = fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y)));
 #pragma unroll
@@ -213,10 +216,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int c = lane >> 2, b = (lane & 3) * 4;
       *reinterpret_cast<uint32_t*>(sq + sw128_off(g, c) + b) = hi;
       *reinterpret_cast<uint32_t*>(sq + sw128_off(G + g, c) + b) = lo;
-      if (lane == 0) qscale_s[n] = a.scale_log2 * a.k_scale[kvh + n / G] * ldexpf(1.f, -e);
+      if (lane == 0) qscale_s[g] = a.scale_log2 * a.k_scale[kvh] * ldexpf(1.f, -e);
     }
-    for (int i = tid; i < (NS - 2 * HG) * 8; i += kSoftmaxWarps * 32)
-      *reinterpret_cast<uint4*>(sq + sw128_off(2 * HG + i / 8, i % 8)) = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < (kN - 2 * G) * 8; i += kGroups * kGroupWarps * 32)
+      *reinterpret_cast<uint4*>(sq + sw128_off(2 * G + i / 8, i % 8)) = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
   __syncthreads();  // barrier initialisation, ids and Q' visible to every thread
@@ -238,17 +241,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint8_t* dst = is_v ? sv(k) : sk(k);
         uint64_t* bar = is_v ? &vfull[k % kStages] : &kfull[k % kStages];
         const CUtensorMap* map = is_v ? &vmap : &kmap;
-        const int u0 = k * TT;
-        const int nsub = (min(TT, ntok - u0) + TR - 1) / TR;  // boxes holding context tokens
+        const int u0 = k * kTok;
+        const int nsub = (min(kTok, ntok - u0) + TR - 1) / TR;  // boxes holding context tokens
         if (!is_v && a.skip_tile >= u0 / TR && a.skip_tile < u0 / TR + nsub &&
             skip_for_test(a.skip_tile, a.skip_tile))
           return;
-        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nsub * H2 * TR * 128));
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nsub * TR * 128));
         for (int j = 0; j < nsub; ++j) {
           const int u = u0 + j * TR;
           const int32_t bid = ids[u / a.block_size];
           const int32_t row0 = bid >= 0 ? bid * a.block_size + u % a.block_size : -TR;
-          tma_load_4d(dst + j * H2 * TR * 128, map, bar, 0, row0, kvh, 0, policy);
+          tma_load_4d(dst + j * TR * 128, map, bar, 0, row0, kvh, 0, policy);
         }
       };
       bool ok = true;
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == kMmaWarp) {
     // ================= MMA issue (one thread) =================
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = tc::idesc_f8_ab<0, 0, kTok, NS, false, false>();
+      constexpr uint32_t IDESC_S = tc::idesc_f8_ab<0, 0, kTok, kN, false, false>();
       constexpr uint32_t IDESC_O_HI = tc::idesc_f8_ab<0, 0, kTok, kN, true, true>();
       constexpr uint32_t IDESC_O_LO = tc::idesc_f8_ab<0, 1, kTok, kN, true, true>();
       // descriptors computed once; a k-step or stage offset is added to the
@@ -296,42 +299,47 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t qd = tc::sw128_desc(sq, 16, 1024);
       const uint64_t kd0 = tc::sw128_desc(smem, 16, 1024);
       const uint64_t vd0 = tc::sw128_desc(smem + kOffV, kTileBytes, 1024);
-      const uint64_t pd0 = tc::plain_desc(sp, 128, 128);
+      const uint64_t pd0 = tc::plain_desc(smem + kOffP, 128, 128);
       int k = 0;
-      auto issue_s = [&](int kk_tile) {  // S^T of tile kk_tile into buffer kk_tile & 1
-        if (kk_tile >= 2 &&
-            !mbar_wait(&s_free[kk_tile & 1], ((kk_tile - 2) >> 1) & 1, lim, &aborted))
+      // tile t belongs to group t & 1 as its (t >> 1)-th tile
+      auto issue_s = [&](int t) {
+        const int g = t & 1, j = t >> 1;
+        if (j >= 2 && !mbar_wait(&s_free[g][j & 1], ((j - 2) >> 1) & 1, lim, &aborted))
           return false;
-        if (!mbar_wait(&kfull[kk_tile % kStages], (kk_tile / kStages) & 1, lim, &aborted))
-          return false;
+        if (!mbar_wait(&kfull[t % kStages], (t / kStages) & 1, lim, &aborted)) return false;
         tc::fence_after_sync();
-        const uint64_t kd = kd0 + static_cast<uint64_t>(((kk_tile % kStages) * kTileBytes) >> 4);
+        const uint64_t kd = kd0 + static_cast<uint64_t>(((t % kStages) * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 32 dims (bytes) per K step
-          tc::mma_f8(tmem + (kk_tile & 1) * NS, kd + 2 * kk, qd + 2 * kk, IDESC_S, kk > 0);
-        tc::commit(&s_full[kk_tile & 1]);
-        tc::commit(&kempty[kk_tile % kStages]);
+          tc::mma_f8(tmem + g * kGroupCols + (j & 1) * kN, kd + 2 * kk, qd + 2 * kk, IDESC_S,
+                     kk > 0);
+        tc::commit(&s_full[g][j & 1]);
+        tc::commit(&kempty[t % kStages]);
         return true;
       };
-      bool ok = ntiles == 0 || issue_s(0);
+      bool ok = true;
+      for (int t = 0; ok && t < min(2, ntiles); ++t) ok = issue_s(t);
       for (; ok && k < ntiles; ++k) {
-        if (k + 1 < ntiles) ok = issue_s(k + 1);
+        // S of the group's next tile first, then O += P V of tile k
+        if (k + 2 < ntiles) ok = issue_s(k + 2);
         if (!ok) break;
+        const int g = k & 1, j = k >> 1;
         ok = mbar_wait(&vfull[k % kStages], (k / kStages) & 1, lim, &aborted) &&
-             mbar_wait(&p_full[k & 1], (k >> 1) & 1, lim, &aborted);
+             mbar_wait(&p_full[g], j & 1, lim, &aborted);
         if (!ok) break;
         tc::fence_after_sync();
         const uint64_t vd = vd0 + static_cast<uint64_t>(((k % kStages) * kTileBytes) >> 4);
-        const uint64_t ph = pd0 + static_cast<uint64_t>(((k & 1) * kPBuf) >> 4);
+        const uint64_t ph = pd0 + static_cast<uint64_t>((g * kPBuf) >> 4);
         const uint64_t pl = ph + static_cast<uint64_t>((kTok * 16) >> 4);
+        const uint32_t to = tmem + g * kGroupCols + kColO;
 #pragma unroll
         for (int kk = 0; kk < kTok / 32; ++kk) {  // 32 tokens per K step
           const uint64_t av = vd + static_cast<uint64_t>((kk * 32 * 128) >> 4);
           const uint64_t off = static_cast<uint64_t>((kk * 32 * 16) >> 4);
-          tc::mma_f8(tmem + kColO, av, ph + off, IDESC_O_HI, k > 0 || kk > 0);
-          tc::mma_f8(tmem + kColO, av, pl + off, IDESC_O_LO, true);
+          tc::mma_f8(to, av, ph + off, IDESC_O_HI, j > 0 || kk > 0);
+          tc::mma_f8(to, av, pl + off, IDESC_O_LO, true);
         }
-        tc::commit(&p_free[k & 1]);
+        tc::commit(&p_free[g]);
         tc::commit(&vempty[k % kStages]);
       }
       if (!ok) {
@@ -346,107 +354,111 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncwarp();  // whole warps reach the CTA barrier below
   } else {
-    // ================= softmax warps =================
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int h = (tid / TR) % H2;                        // this row's kv-head (of the CTA)
-    const int utok = (tid / (TR * H2)) * TR + tid % TR;   // and its token in the tile
-    float m[HG], l[HG], qs[HG];
+    // ================= softmax warps (two groups) =================
+    const int grp = warp / kGroupWarps, gw = warp % kGroupWarps;
+    const int gtid = tid - grp * kGroupWarps * 32;      // token / dimension of this thread
+    const uint32_t lane_base = static_cast<uint32_t>(gw * 32) << 16;
+    const uint32_t tbase = tmem + grp * kGroupCols;
+    const int ntg = ntiles > grp ? (ntiles - grp + 1) / 2 : 0;  // tiles of this group
+    uint8_t* pbuf = sp(grp);
+    float m[G], l[G], qs[G];
 #pragma unroll
-    for (int n = 0; n < HG; ++n) {
-      m[n] = -CUDART_INF_F;
-      l[n] = 0.f;
-      qs[n] = qscale_s[n];
+    for (int g = 0; g < G; ++g) {
+      m[g] = -CUDART_INF_F;
+      l[g] = 0.f;
+      qs[g] = qscale_s[g];
     }
     bool ok = true;
-    int k = 0;
-    for (; ok && k < ntiles; ++k) {
-      ok = __all_sync(FULL, mbar_wait(&s_full[k & 1], (k >> 1) & 1, lim, &aborted));
+    int j = 0;
+    for (; ok && j < ntg; ++j) {
+      const int k = 2 * j + grp;  // the tile
+      ok = __all_sync(FULL, mbar_wait(&s_full[grp][j & 1], (j >> 1) & 1, lim, &aborted));
       if (!ok) break;
       tc::fence_after_sync();
-      uint32_t r[NS];
-      tc::ld16_nowait(tmem + (k & 1) * NS + lane_base, r);
+      uint32_t r[NL];
+      if constexpr (NL == 8) tc::ld8_nowait(tbase + (j & 1) * kN + lane_base, r);
+      else tc::ld16_nowait(tbase + (j & 1) * kN + lane_base, r);
       tc::wait_ld();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[k & 1]);
-      const int vk = min(TT, ntok - k * TT);  // context tokens in this tile
-      const bool live = utok < vk;
-      // logits (base 2) of the query heads of this row's kv-head; -inf elsewhere
-      float x[HG];
+      if (lane == 0) mbar_arrive(&s_free[grp][j & 1]);
+      const int vk = min(kTok, ntok - k * kTok);  // context tokens in this tile
+      const bool live = gtid < vk;
+      float x[G];
 #pragma unroll
-      for (int n = 0; n < HG; ++n) {
-        const int c = (n / G) * 2 * G + n % G;
-        x[n] = live && n / G == h
-                   ? (__uint_as_float(r[c]) + __uint_as_float(r[c + G])) * qs[n]
-                   : -CUDART_INF_F;
-      }
-      // the tile's maximum per query head over the CTA
+      for (int g = 0; g < G; ++g)
+        x[g] = live ? (__uint_as_float(r[g]) + __uint_as_float(r[G + g])) * qs[g]
+                    : -CUDART_INF_F;
+      // the tile's maximum per head over the group
 #pragma unroll
-      for (int n = 0; n < HG; ++n) {
-        const int mx = __reduce_max_sync(FULL, ord_of(x[n]));
-        if (lane == 0) red[k & 1][warp][n] = float_of(mx);
+      for (int g = 0; g < G; ++g) {
+        const int mx = __reduce_max_sync(FULL, ord_of(x[g]));
+        if (lane == 0) red[grp][j & 1][gw][g] = float_of(mx);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&red_bar[k & 1]);
-      ok = __all_sync(FULL, mbar_wait(&red_bar[k & 1], (k >> 1) & 1, lim, &aborted));
+      if (lane == 0) mbar_arrive(&red_bar[grp][j & 1]);
+      ok = __all_sync(FULL, mbar_wait(&red_bar[grp][j & 1], (j >> 1) & 1, lim, &aborted));
       if (!ok) break;
-      float alpha[HG];
+      float alpha[G];
       bool rescale = false;
 #pragma unroll
-      for (int n = 0; n < HG; ++n) {
-        float tmax = red[k & 1][0][n];
+      for (int g = 0; g < G; ++g) {
+        float tmax = red[grp][j & 1][0][g];
 #pragma unroll
-        for (int w = 1; w < kSoftmaxWarps; ++w) tmax = fmaxf(tmax, red[k & 1][w][n]);
-        alpha[n] = 1.f;
-        if (tmax > m[n] + kLazy) {  // false while the head has seen nothing
-          alpha[n] = tc::ex2(m[n] - tmax);
-          m[n] = tmax;
+        for (int w = 1; w < kGroupWarps; ++w) tmax = fmaxf(tmax, red[grp][j & 1][w][g]);
+        alpha[g] = 1.f;
+        if (tmax > m[g] + kLazy) {  // false while the head has seen nothing
+          alpha[g] = tc::ex2(m[g] - tmax);
+          m[g] = tmax;
           rescale = true;
         }
       }
-      float p[16];
+      float p[8];
 #pragma unroll
-      for (int n = 0; n < 16; ++n) p[n] = 0.f;
+      for (int g = 0; g < 8; ++g) p[g] = 0.f;
 #pragma unroll
-      for (int n = 0; n < HG; ++n) {
-        const float mu = m[n] == -CUDART_INF_F ? 0.f : m[n];
-        p[n] = tc::ex2(x[n] - mu);
-        l[n] = fmaf(l[n], alpha[n], p[n]);
+      for (int g = 0; g < G; ++g) {
+        const float mu = m[g] == -CUDART_INF_F ? 0.f : m[g];
+        p[g] = tc::ex2(x[g] - mu);
+        l[g] = fmaf(l[g], alpha[g], p[g]);
       }
-      // O^T may be rescaled only once O += P V of tile k-1 completed (rare:
-      // the maximum moves lazily); the same for every thread of the CTA
-      if (rescale && k >= 1) {
-        ok = __all_sync(FULL, mbar_wait(&p_free[(k - 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted));
+      // The group's P' buffer is free, and its O^T may be rescaled, once
+      // O += P V of its previous tile completed
+      if (j >= 1) {
+        ok = __all_sync(FULL, mbar_wait(&p_free[grp], (j - 1) & 1, lim, &aborted));
         if (!ok) break;
+      }
+      if (rescale && j >= 1) {  // rare: the maximum moves lazily; uniform over the group
         tc::fence_after_sync();
-        uint32_t o[16];
-        tc::ld16_nowait(tmem + kColO + lane_base, o);
+        uint32_t o[NL];
+        if constexpr (NL == 8) tc::ld8_nowait(tbase + kColO + lane_base, o);
+        else tc::ld16_nowait(tbase + kColO + lane_base, o);
         tc::wait_ld();
 #pragma unroll
-        for (int n = 0; n < HG; ++n) o[n] = __float_as_uint(__uint_as_float(o[n]) * alpha[n]);
-        tc::st16u(tmem + kColO + lane_base, o);
+        for (int g = 0; g < G; ++g) o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
+        if constexpr (NL == 8) tc::st8u(tbase + kColO + lane_base, o);
+        else tc::st16u(tbase + kColO + lane_base, o);
         tc::wait_st();
       }
-      // P' buffer k & 1 is free once O += P V of tile k-2 completed
-      if (k >= 2) {
-        ok = __all_sync(FULL, mbar_wait(&p_free[k & 1], ((k - 2) >> 1) & 1, lim, &aborted));
-        if (!ok) break;
+      uint32_t hw[4], lw[4];
+      tc::split_fp8x4<true>(p[0], p[1], p[2], p[3], hw[0], lw[0]);
+      if constexpr (G > 4) {
+        tc::split_fp8x4<true>(p[4], p[5], p[6], p[7], hw[1], lw[1]);
+      } else {
+        hw[1] = lw[1] = 0u;
       }
-      uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int q = 0; q < (HG + 3) / 4; ++q)
-        tc::split_fp8x4<true>(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3], hw[q], lw[q]);
-      uint8_t* prow = sp + (k & 1) * kPBuf + tid * 16;
-      *reinterpret_cast<uint4*>(prow) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(prow + kTok * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      hw[2] = hw[3] = lw[2] = lw[3] = 0u;
+      *reinterpret_cast<uint4*>(pbuf + gtid * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(pbuf + kTok * 16 + gtid * 16) =
+          make_uint4(lw[0], lw[1], lw[2], lw[3]);
       // V rows without context tokens (end of the unit) may hold anything,
       // even NaN codes, and 0 * NaN is NaN inside the MMA: clear them once
       // the tile's loads landed
-      if (vk < TT) {
+      if (vk < kTok) {
         ok = __all_sync(FULL, mbar_wait(&vfull[k % kStages], (k / kStages) & 1, lim, &aborted));
         if (!ok) break;
         if (!live) {
-          uint4* row = reinterpret_cast<uint4*>(sv(k) + tid * 128);
+          uint4* row = reinterpret_cast<uint4*>(sv(k) + gtid * 128);
 #pragma unroll
           for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -454,68 +466,105 @@ __global__ void __launch_bounds__(kThreads, 2)
       fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[k & 1]);
+      if (lane == 0) mbar_arrive(&p_full[grp]);
     }
-    if (ok && ntiles > 0)
-      ok = __all_sync(FULL, mbar_wait(&p_free[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, lim,
-                                      &aborted));
+    if (ok && ntg > 0)
+      ok = __all_sync(FULL, mbar_wait(&p_free[grp], (ntg - 1) & 1, lim, &aborted));
     // A warp that gave up says so before it posts its sums, so that the
     // others, which wait for those, see the flag.
     if (!ok && lane == 0) {
-      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 2, k, ntiles, 0);
+      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 2 + grp, 2 * j + grp, ntiles, 0);
       aborted = 1;
       report(a.err, kErrWaitTimeout);
     }
-    // the partial sums over the CTA (every softmax warp posts its own)
+    // the group's partial sums (every warp of the group posts its own)
 #pragma unroll
-    for (int n = 0; n < HG; ++n) {
-      float v = l[n];
+    for (int g = 0; g < G; ++g) {
+      float v = l[g];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-      if (lane == 0) lsum[warp][n] = v;
+      if (lane == 0) lsum[grp][gw][g] = v;
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sum_bar);
-    const bool sums = __all_sync(FULL, mbar_wait(&sum_bar, 0, lim, &aborted));
+    if (lane == 0) mbar_arrive(&sum_bar[grp]);
+    const bool sums = __all_sync(FULL, mbar_wait(&sum_bar[grp], 0, lim, &aborted));
     if (!sums && lane == 0) {
-      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 3, k, ntiles, 0);
+      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 4 + grp, 2 * j + grp, ntiles, 0);
       aborted = 1;
       report(a.err, kErrWaitTimeout);
     }
-    __syncwarp();
-    ok = __all_sync(FULL, ok && sums && *static_cast<volatile int*>(&aborted) == 0);
-    const bool single = parts == 1;
-    const int64_t row0 = static_cast<int64_t>(s) * a.num_heads + kvh * G;
-    if (!ok) {
-      // The unit's result is lost: leave zeros (single pass) or an empty
-      // partial that the combine kernel gives no weight, never stale data.
+    // thread i holds dimension i of the group's O for every head: normalised
+    // by the group's sum (0 where the group saw no token)
+    float L[G], on[G];
 #pragma unroll
-      for (int n = 0; n < HG; ++n) {
-        if (single) store_out(QF{}, a.out, (row0 + n) * 128 + tid, 0.f);
-        else if (tid == 0) a.ws_ml[(row0 + n) * a.max_parts + part] = make_float2(-CUDART_INF_F, 0.f);
+    for (int g = 0; g < G; ++g) {
+      L[g] = 0.f;
+#pragma unroll
+      for (int w = 0; w < kGroupWarps; ++w) L[g] += lsum[grp][w][g];
+      on[g] = 0.f;
+    }
+    if (ok && sums && ntg > 0) {
+      tc::fence_after_sync();
+      uint32_t o[NL];
+      if constexpr (NL == 8) tc::ld8_nowait(tbase + kColO + lane_base, o);
+      else tc::ld16_nowait(tbase + kColO + lane_base, o);
+      tc::wait_ld();
+#pragma unroll
+      for (int g = 0; g < G; ++g) on[g] = L[g] > 0.f ? __uint_as_float(o[g]) / L[g] : 0.f;
+    }
+    // the second group hands (max, sum, O / sum) to the first through shared
+    // memory: the first K stage, which is idle once the group's last
+    // O += P V completed (every S, issued before it, is done then, and no K
+    // load follows); a group without a tile, or that gave up, posts sum 0 and
+    // leaves that memory alone
+    float* mo = reinterpret_cast<float*>(smem);   // [128 dims][G]
+    if (grp == 1) {
+      const bool has = ok && sums && ntg > 0;
+      if (has) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) mo[gtid * G + g] = on[g];
       }
+      if (gtid == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          merge_ml[0][g] = m[g];
+          merge_ml[1][g] = has ? L[g] : 0.f;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&merge_bar);
     } else {
-      // ---- epilogue: thread i holds dimension i of every query head's O
-      uint32_t o[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) o[i] = 0u;
-      if (ntiles > 0) {
-        tc::fence_after_sync();
-        tc::ld16_nowait(tmem + kColO + lane_base, o);
-        tc::wait_ld();
+      const bool merged = __all_sync(FULL, mbar_wait(&merge_bar, 0, lim, &aborted));
+      if (!merged && lane == 0) {
+        record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 6, ntiles, ntiles, 0);
+        aborted = 1;
+        report(a.err, kErrWaitTimeout);
       }
+      __syncwarp();
+      const bool good =
+          __all_sync(FULL, ok && sums && merged && *static_cast<volatile int*>(&aborted) == 0);
+      const bool single = parts == 1;
+      const int64_t row0 = static_cast<int64_t>(s) * a.num_heads + kvh * G;
+      const float vs = a.v_scale[kvh];
 #pragma unroll
-      for (int n = 0; n < HG; ++n) {
-        float L = 0.f;
-#pragma unroll
-        for (int w = 0; w < kSoftmaxWarps; ++w) L += lsum[w][n];
-        const float val = L > 0.f ? __uint_as_float(o[n]) / L * a.v_scale[kvh + n / G] : 0.f;
+      for (int g = 0; g < G; ++g) {
+        // the two groups as two parts of the context: weights L 2^(m - M)
+        const float m1 = merge_ml[0][g], L1 = merge_ml[1][g];
+        const float M = fmaxf(m[g], m1);
+        const float w0 = L[g] > 0.f ? L[g] * tc::ex2(m[g] - M) : 0.f;
+        const float w1 = L1 > 0.f ? L1 * tc::ex2(m1 - M) : 0.f;
+        const float W = w0 + w1;
+        float val = w0 * on[g];
+        if (w1 > 0.f) val += w1 * mo[gtid * G + g];
+        val = W > 0.f ? val / W * vs : 0.f;
+        if (!good) val = 0.f;
         if (single) {
-          store_out(QF{}, a.out, (row0 + n) * 128 + tid, val);
+          store_out(QF{}, a.out, (row0 + g) * 128 + gtid, val);
         } else {
-          const int64_t pi = (row0 + n) * a.max_parts + part;
-          a.ws_o[pi * 128 + tid] = val;
-          if (tid == 0) a.ws_ml[pi] = make_float2(m[n], L);
+          const int64_t pi = (row0 + g) * a.max_parts + part;
+          a.ws_o[pi * 128 + gtid] = val;
+          if (gtid == 0)
+            a.ws_ml[pi] = good && W > 0.f ? make_float2(M, W) : make_float2(-CUDART_INF_F, 0.f);
         }
       }
     }
@@ -528,31 +577,26 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <class QF, int G, int H2>
+template <class QF, int G>
 cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                        cudaStream_t stream) {
-  if (a.partition_blocks > kMaxUnitBlocks || a.num_kv_heads % H2 != 0)
-    return cudaErrorNotSupported;
+  if (a.partition_blocks > kMaxUnitBlocks) return cudaErrorNotSupported;
   const size_t smem = 1024 + kOffIds + 4 * static_cast<size_t>(a.partition_blocks);
-  auto kern = paged_decode_fp8_tc_kernel<QF, G, H2>;
+  auto kern = paged_decode_fp8_tc_kernel<QF, G>;
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(a.num_kv_heads / H2, a.num_seqs, a.max_parts), kThreads, smem,
-                    stream, a, kmap, vmap);
+  return launch_pdl(kern, dim3(a.num_kv_heads, a.num_seqs, a.max_parts), kThreads, smem, stream,
+                    a, kmap, vmap);
 }
 
 }  // namespace
 
-// One kv-head per CTA. (A form with two kv-heads per CTA, one 4 KB box per
-// 16 tokens, is written above as H2 = 2; it is not launched: on B200 it
-// ended in an unspecified launch failure on the full-size shared-prefix
-// workload with units of 8 or more of its tiles, with the cause not found.)
 int decode_fp8_tc_heads_per_cta(int, int) { return 1; }
 
 cudaError_t decode_fp8_tc(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           int q_dtype, int group, cudaStream_t stream) {
 #define PAGED_FP8TC(QF, g) \
-  if (group == g) return launch_one<QF, g, 1>(a, kmap, vmap, stream);
+  if (group == g) return launch_one<QF, g>(a, kmap, vmap, stream);
   if (q_dtype == kF16) {
     PAGED_FP8TC(F16, 1) PAGED_FP8TC(F16, 2) PAGED_FP8TC(F16, 4) PAGED_FP8TC(F16, 8)
   } else if (q_dtype == kBF16) {

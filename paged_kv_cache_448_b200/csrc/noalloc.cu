@@ -94,7 +94,8 @@ extern "C" PA_API pa_status pa_decode_noalloc(
   using namespace paged;
   clear_error();
   const size_t need = pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
-                                               block_size, max_context_len, partition_tokens);
+                                               block_size, max_context_len, partition_tokens,
+                                               cache_dtype);
   if (need == 0) return fail(PA_ERR_INVALID_ARG, "decode_noalloc: invalid sizes");
   if (need > kNoAllocScratchBytes)
     return fail(PA_ERR_UNSUPPORTED,

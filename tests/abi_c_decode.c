@@ -124,7 +124,7 @@ int main(int argc, char** argv) {
   CHECK_CUDA(cudaMalloc(&d_table, sizeof table));
   CHECK_CUDA(cudaMalloc(&d_ctx, sizeof ctx));
   CHECK_CUDA(cudaMalloc(&d_slots, sizeof slots));
-  const size_t ws_bytes = pa_decode_workspace_size(S, H, HKV, D, BS, 300, 0);
+  const size_t ws_bytes = pa_decode_workspace_size(S, H, HKV, D, BS, 300, 0, PA_F16);
   if (ws_bytes < 256) return 1;
   CHECK_CUDA(cudaMalloc(&d_ws, ws_bytes));
   CHECK_CUDA(cudaMemcpy(d_kc, kc, cache_elems * 2, cudaMemcpyHostToDevice));

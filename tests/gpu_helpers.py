@@ -162,7 +162,7 @@ class GpuStep:
         if workspace is None:
             wsg = guarded_workspace(pk.decode_workspace_size(
                 sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size,
-                self.max_ctx, p))
+                self.max_ctx, p, pk.dtype_code(self.kc)))
             workspace = wsg.t
         out = pk.decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, self.max_ctx,
                         sp.scale, k_scale=self.ks, v_scale=self.vs, partition_tokens=p,

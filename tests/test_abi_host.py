@@ -360,6 +360,17 @@ def test_workspace_sizes_and_partition_plan():
     assert pk.decode_partition_tokens(32, 32, 32, 128, 16, 2048, 512) == 512
     # partitions are whole blocks
     assert pk.decode_partition_tokens(2, 8, 8, 128, 32, 4096, 300) == 320
+    # the E4M3 tcgen05 kernel (head_dim 128) wants one wave of units (two
+    # CTAs per SM): 128 sequences x 8 kv-heads of up to 1534 tokens run in one
+    # pass, where the 16-bit kernels cut them into 1024-token partitions;
+    # with 8 sequences both cut
+    fp8 = _native.PA_FP8_E4M3
+    assert pk.decode_partition_tokens(128, 32, 8, 128, 16, 1534, 0, fp8) >= 1534
+    assert pk.decode_workspace_size(128, 32, 8, 128, 16, 1534, 0, fp8) == 256
+    assert pk.decode_partition_tokens(128, 32, 8, 128, 16, 1534, 0) == 1024
+    assert pk.decode_partition_tokens(8, 32, 8, 128, 16, 1534, 0, fp8) < 1534
+    # head_dim 64 over E4M3 keeps the mma.sync kernel and its plan
+    assert pk.decode_partition_tokens(128, 32, 8, 64, 16, 1534, 0, fp8) == 1024
 
 
 def test_slot_mapping_agrees_with_oracle_on_random_tables():

@@ -52,10 +52,11 @@ def test_decode_wait_that_runs_out(G, part, cache):
     g.reshape()
     sp = g.sp
     _, _, ref = oracle_ref(g)
+    cdt = pk.dtype_code(g.kc)
     ws = pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
-                             sp.block_size, g.max_ctx, part)
+                             sp.block_size, g.max_ctx, part, cache_dtype=cdt)
     split = pk.decode_partition_tokens(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
-                                       sp.block_size, g.max_ctx, part) < g.max_ctx
+                                       sp.block_size, g.max_ctx, part, cdt) < g.max_ctx
     g.out.fill_(float("nan"))
     pk.inject_wait_timeout(3, LIMIT_NS)        # tile 3 of (kv-head 0, sequence 0, part 0)
     pk.decode(g.out, g.q, g.kc, g.vc, g.bt, g.cl, g.max_ctx, sp.scale, k_scale=g.ks,

@@ -302,7 +302,8 @@ def test_full_size_workload_sampled(cfg):
     pk.reshape_and_cache(d["new_key"], d["new_value"], d["key_cache"], d["value_cache"],
                          i32(slots), k_scale=d["k_scale"], v_scale=d["v_scale"])
     ws = pk.decode_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
-                             sp.block_size, int(lens.max()), sp.partition_tokens)
+                             sp.block_size, int(lens.max()), sp.partition_tokens,
+                             cache_dtype=pk.dtype_code(d["key_cache"]))
     pk.decode(out, d["query"], d["key_cache"], d["value_cache"], i32(st.block_tables),
               i32(lens), int(lens.max()), sp.scale, k_scale=d["k_scale"], v_scale=d["v_scale"],
               partition_tokens=sp.partition_tokens, workspace=ws)
