@@ -100,12 +100,20 @@ def measured_tensor_peak():
     return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def decode_sources() -> list:
-    """The files the decode kernels are built from: the decode_*.cu units,
-    everything they include (transitively), and api.cu, which launches them."""
+# The units each bench row's kernels are built from (plus everything they
+# include, and api.cu, which launches them).
+OP_UNITS = {"decode": ("decode_*.cu",), "prefill": ("prefill_*.cu",),
+            "copy_blocks": ("copy_blocks.cu",)}
+
+
+def op_sources(op: str = "decode") -> list:
+    """The files the kernels of a bench row are built from: its units,
+    everything they include (transitively), and api.cu."""
     import re
     csrc = os.path.join(ROOT, "paged_kv_cache_448_b200", "csrc")
-    todo = sorted(glob.glob(os.path.join(csrc, "decode_*.cu"))) + [os.path.join(csrc, "api.cu")]
+    todo = [os.path.join(csrc, "api.cu")]
+    for pat in OP_UNITS[op]:
+        todo += sorted(glob.glob(os.path.join(csrc, pat)))
     seen = set()
     while todo:
         f = todo.pop()
@@ -118,28 +126,35 @@ def decode_sources() -> list:
     return sorted(seen)
 
 
-def sources_digest() -> str:
-    """Digest of the decode kernels' sources: a recorded DRAM traffic figure
-    stands only for the exact sources it was taken on."""
+def decode_sources() -> list:
+    return op_sources("decode")
+
+
+def sources_digest(op: str = "decode") -> str:
+    """Digest of a row's kernel sources: a recorded DRAM traffic figure stands
+    only for the exact sources it was taken on."""
     h = hashlib.sha256()
-    for f in decode_sources():
+    for f in op_sources(op):
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())
     return h.hexdigest()
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel sources and this workload; else None."""
+def recorded_traffic(workload: str, op: str = "decode"):
+    """DRAM bytes (read + write) per launch of a row's dominant kernel from the
+    committed ncu record, if it was taken on the current sources of that row
+    and on this workload; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        j = json.load(f).get("decode", {})
-    if j.get("sources_sha256") != sources_digest() or j.get("workload") != workload:
-        return None
-    return j.get("dram_bytes_per_launch")
+        entries = json.load(f).get("entries", [])
+    for e in entries:
+        if e.get("op") == op and e.get("workload") == workload and \
+                e.get("sources_sha256") == sources_digest(op):
+            return e.get("dram_bytes_per_launch")
+    return None
 
 
 class ClockSampler:
@@ -466,7 +481,8 @@ def run_prefill(args):
             if tensor_bound else
             {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak_b, "unit": "GB/s",
              "frac": round(gbs / peak_b, 4), "peak_kind": f"{kind_b} HBM copy GB/s"})
-    roof.update({"traffic": None, "algorithmic_flops_per_launch": flops,
+    roof.update({"traffic": recorded_traffic(sp.name, "prefill"),
+                 "algorithmic_flops_per_launch": flops,
                  "algorithmic_bytes_per_launch": nbytes, "launch_ms": round(ms, 5)})
     line = {"metric": "multi-token paged attention TFLOP/s", "value": round(tflops, 3),
             "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -508,7 +524,8 @@ def run_copy(args):
         gbs = moved / (ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(gbs, 2), "peak": peak, "unit": "GB/s",
                 "frac": round(gbs / peak, 4), "peak_kind": f"{kind} HBM copy GB/s",
-                "traffic": None, "algorithmic_bytes_per_launch": moved, "launch_ms": round(ms, 5)}
+                "traffic": recorded_traffic("copy_blocks", "copy_blocks"),
+                "algorithmic_bytes_per_launch": moved, "launch_ms": round(ms, 5)}
         metric, workload = "block copy GB/s (read + write)", \
             f"copy-on-write: {n} block pairs of a 4352-block fp16 cache (16 x 32 x 128), K and V"
     else:
@@ -602,7 +619,7 @@ def decode_line(args, sp: wl.Spec, st: wl.Structure, world: int, step_ms: float,
                      "achieved": round(achieved, 2), "peak": peak,
                      "peak_kind": f"{peak_kind} HBM copy GB/s", "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": recorded_traffic(sp.name),
+                     "traffic": recorded_traffic(sp.name, "decode"),
                      "algorithmic_bytes_per_launch": dbytes,
                      "launch_ms": round(dec_ms, 5)},
         "gpu_launches": launches_per_step * args.steps,
@@ -614,8 +631,9 @@ def decode_line(args, sp: wl.Spec, st: wl.Structure, world: int, step_ms: float,
                        "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": round(e2e["ms_per_step"], 5),
                        "copies": "one packed host-to-device copy of the step's inputs and one "
-                                 "device-to-host copy of its output per step, on a copy stream, "
-                                 "double-buffered so they overlap the neighbouring steps"}
+                                 "device-to-host copy of its output per step, on an upload and a "
+                                 "read-back stream, double-buffered so they overlap the "
+                                 "neighbouring steps"}
     return line
 
 
@@ -623,9 +641,9 @@ class E2EStep:
     """One decode step through the public API from pinned host memory: the
     step's inputs (query, new K/V, block table, context lengths, slots) are
     packed in one pinned buffer and uploaded by one copy, and the output is
-    read back by one copy, both on a copy stream. Two device buffers of each
-    alternate, so the upload of step k+1 and the read-back of step k run under
-    the decode of the neighbouring step."""
+    read back by one copy, on an upload stream and a read-back stream. Two
+    device buffers of each alternate, so the upload of step k+1 and the
+    read-back of step k-1 run under the decode of step k."""
 
     NAMES = ("query", "new_key", "new_value", "bt", "cl", "sl")
 
@@ -653,35 +671,41 @@ class E2EStep:
         self.pin_out = [torch.empty(out_like.shape, dtype=out_like.dtype).pin_memory()
                         for _ in range(2)]
         self.d2h = out_like.numel() * out_like.element_size()
-        self.copy = torch.cuda.Stream(device=device)
+        # uploads and read-backs on streams of their own: a read-back waits for
+        # its step's decode, and the next upload must not queue behind it
+        self.up = torch.cuda.Stream(device=device)
+        self.down = torch.cuda.Stream(device=device)
         self.compute = torch.cuda.current_stream(device)
         ev = lambda: torch.cuda.Event()  # noqa: E731
         self.uploaded, self.consumed, self.produced, self.read = (
             [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()])
         self.run_step = run_step
+        # the same per-step event pair around the decode as in the device-timed
+        # loop, so that both loops carry the same instrumentation
+        self.ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
         self.k = 0
         for b in range(2):  # every buffer starts free
             self.consumed[b].record(self.compute)
-            self.read[b].record(self.copy)
+            self.read[b].record(self.down)
 
     def __call__(self):
         import torch
         b = self.k & 1
-        with torch.cuda.stream(self.copy):
-            self.copy.wait_event(self.consumed[b])        # the decode of step k-2 read it
+        with torch.cuda.stream(self.up):
+            self.up.wait_event(self.consumed[b])          # the decode of step k-2 read it
             self.dev_in[b].copy_(self.pin_in, non_blocking=True)
-            self.uploaded[b].record(self.copy)
+            self.uploaded[b].record(self.up)
         self.compute.wait_event(self.uploaded[b])
         self.compute.wait_event(self.read[b])             # step k-2's output was read back
         v = self.views[b]
         self.run_step(v["query"], v["new_key"], v["new_value"], v["bt"], v["cl"], v["sl"],
-                      self.out[b])
+                      self.out[b], self.ev)
         self.consumed[b].record(self.compute)
         self.produced[b].record(self.compute)
-        with torch.cuda.stream(self.copy):
-            self.copy.wait_event(self.produced[b])
+        with torch.cuda.stream(self.down):
+            self.down.wait_event(self.produced[b])
             self.pin_out[b].copy_(self.out[b], non_blocking=True)
-            self.read[b].record(self.copy)
+            self.read[b].record(self.down)
         self.k += 1
 
     def finish(self):

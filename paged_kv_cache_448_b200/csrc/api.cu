@@ -494,45 +494,15 @@ namespace {
 // multiple of 4) handled by separate CTAs and merged by a combine kernel.
 struct PrefillPlan {
   bool tc;                  // tcgen05 kernel (rows on M), else mma.sync
-  bool tm;                  // tcgen05 kernel with the key tokens on M (short chunks)
   int32_t q_tiles, partition_tiles, max_parts;
 };
-
-// The keys-on-M kernel for short chunks (prefill_tm.cu) is not routed yet:
-// measured on B200 it took 1.085 ms for 8-token verification of 64 sequences,
-// against 0.276 ms on the row-major tcgen05 kernel (one CTA per SM with 255
-// registers per softmax thread, and one thread issuing 32 loads per tile).
-constexpr bool kKeysOnM = false;
 
 PrefillPlan make_prefill_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t group,
                               int32_t head_dim, int32_t max_query_len, int32_t max_context_len,
                               bool fp8) {
   PrefillPlan p{};
   const int64_t rows = static_cast<int64_t>(max_query_len) * group;
-  if (kKeysOnM && !fp8 && head_dim == 128 && rows <= 64) {
-    // Short chunks with a 16-bit cache: the query rows (at most 64) are the N
-    // of tcgen05 tiles of 128 key tokens. One CTA per SM and (sequence,
-    // kv-head): below about six waves the key range is cut into parts of
-    // whole 128-token tiles, at least two per part.
-    p.tm = true;
-    p.q_tiles = 1;
-    const int32_t tiles16 = std::max<int32_t>(1, (max_context_len + 15) / 16);
-    const int32_t tiles128 = (tiles16 + 7) / 8;
-    p.partition_tiles = tiles128 * 8;
-    p.max_parts = 1;
-    const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
-    const int64_t want = 6LL * sm_count();
-    if (units < want && tiles128 >= 4) {
-      const int32_t parts = static_cast<int32_t>(
-          std::min<int64_t>((want + units - 1) / units, tiles128 / 2));
-      if (parts > 1) {
-        const int32_t per = (tiles128 + parts - 1) / parts;
-        p.partition_tiles = per * 8;
-        p.max_parts = (tiles16 + p.partition_tiles - 1) / p.partition_tiles;
-      }
-    }
-    return p;
-  }
+
   // query tokens per CTA: tcgen05 128 rows per group, two groups once the
   // chunks fill 256 rows; mma.sync 64 rows
   const int32_t qt_tc = (rows >= 256 ? 256 : 128) / group;
@@ -641,7 +611,7 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
   const PrefillPlan plan =
       make_prefill_plan(num_seqs, num_kv_heads, group, head_dim, max_query_len,
                         max_context_len, fp8);
-  const bool tc = plan.tc || plan.tm;   // both tcgen05 kernels take one-segment boxes
+  const bool tc = plan.tc;   // the tcgen05 kernel takes one-segment boxes
   const size_t need = prefill_workspace_bytes(plan, num_tokens, num_heads, head_dim);
   if (workspace_bytes < need)
     return fail(PA_ERR_INVALID_ARG, "chunked_prefill: workspace %zu bytes < %zu needed",
@@ -686,9 +656,8 @@ PA_API pa_status pa_chunked_prefill(void* out, const void* query, const int32_t*
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int cd = fp8 ? kE4M3 : qd;
   const cudaError_t e =
-      plan.tm ? launch_prefill_tm(a, kmap, vmap, qd, head_dim, group, max_query_len, cs)
-      : tc    ? launch_prefill_tc(a, kmap, vmap, qd, cd, head_dim, group, max_query_len, cs)
-              : launch_prefill(a, kmap, vmap, qd, cd, head_dim, group, max_query_len, cs);
+      tc ? launch_prefill_tc(a, kmap, vmap, qd, cd, head_dim, group, max_query_len, cs)
+         : launch_prefill(a, kmap, vmap, qd, cd, head_dim, group, max_query_len, cs);
   return cuda_status(e, "chunked_prefill");
 }
 

@@ -23,32 +23,35 @@
 // the two O^T products (hi with E4M3, residual with E5M2) add into the same
 // accumulator. V's scale multiplies the output.
 //
-// A CTA is one work unit (kv-head, sequence, context partition). The time
-// of a tile is the latency of its softmax chain (S load, the CTA-wide tile
-// maximum, P store, then O += P V), so a CTA keeps two tiles in that chain at
-// once: two softmax groups take the tiles in turn, each with its own S
-// buffers, P buffer, running maxima, sums and O accumulator, merged at the
-// end like two parts of the context. Twelve warps:
-//  * two groups of four softmax warps: thread i of a group owns tensor-memory
-//    lane i, i.e. token i of its tiles in S^T and dimension i of its O^T. Per
-//    tile it loads its S^T row, forms the G logits (masking tokens past the
-//    context), and the group takes each head's tile maximum (an ordered-
-//    integer warp reduction, then its four warps through shared memory
-//    behind an mbarrier). The running maximum moves only when a tile's
-//    maximum passes it by more than 8 (base 2), so probabilities stay below
-//    2^8 and O is rarely rescaled (in tensor memory, after the group's
-//    previous O += P V completed). Each thread keeps its own partial sums;
-//  * the MMA warp (one thread) owns the tensor memory: per group two
-//    16-column S^T buffers and 16 columns of O^T. It issues S^T two tiles
-//    ahead (the next tile of the same group), then O^T += V^T P'^T of tile k;
-//  * three TMA warps (one thread each, every third tile) load K and V tiles
-//    into 3-stage rings (one 16-row box per 16 tokens through the block
-//    table) and refill a stage when the MMAs that read it completed.
-// Every wait is bounded by wall time, and no barrier between softmax warps
-// is an unbounded one: their exchanges go through mbarriers. A wait that
-// gives up records the failure, sets a shared abort flag that ends the other
-// waits, and the roles drain their loads and MMAs before the tensor memory is
-// freed; the unit then leaves zeros (or an empty partial).
+// A CTA is one work unit (kv-head, sequence, context partition) with nine
+// warps:
+//  * four softmax warps: thread i owns tensor-memory lane i, i.e. token i of
+//    the tile in S^T and dimension i of O^T. Per tile it loads its S^T row,
+//    forms the G logits (masking tokens past the context), and the CTA takes
+//    each head's tile maximum (an ordered-integer warp reduction, then the
+//    four warps through shared memory behind an mbarrier). The running
+//    maximum moves only when a tile's maximum passes it by more than 8
+//    (base 2), so probabilities stay below 2^8 and O is rarely rescaled (in
+//    tensor memory, after the previous O += P V completed). Each thread keeps
+//    its own partial sums, added over the CTA at the end;
+//  * the MMA warp (one thread) owns the tensor memory: two 16-column S^T
+//    buffers and 16 columns of O^T. It polls and issues whichever is ready:
+//    S^T of the next tile, or O^T += V^T P'^T of the oldest tile whose P' is
+//    posted;
+//  * four TMA warps, two per ring: K tiles and V tiles are loaded each on its
+//    own (a V stage is held until O += P V, and that must not hold back a K
+//    load), and box j of a tile is issued by lane j / 2 of the ring's warp
+//    j % 2, the lanes of a warp at once, so a tile's 8 boxes are all in
+//    flight soon after its stage is free.
+// A tile's time is the latency of that chain (loads, S, the softmax with its
+// exchange, O += P V), so throughput comes from units in flight: two K and
+// two V stages keep a CTA near 70 KB of shared memory, and three CTAs share
+// an SM (query groups up to 4).
+// Every wait is bounded by wall time, and no barrier between the softmax
+// warps is an unbounded one: their exchanges go through mbarriers. A wait
+// that gives up records the failure, sets a shared abort flag that ends the
+// other waits, and the roles drain their loads and MMAs before the tensor
+// memory is freed; the unit then leaves zeros (or an empty partial).
 #include <math_constants.h>
 
 #include <type_traits>
@@ -63,22 +66,21 @@ namespace {
 
 constexpr int kTok = 128;                // tokens per tile (M of S^T)
 constexpr int kN = 16;                   // N of both products: hi and lo query rows, padded
-constexpr int kStages = 3;               // K and V ring depth
+constexpr int kStagesK = 2, kStagesV = 2;
 constexpr int kTileBytes = kTok * 128;   // one K (or V) tile: 128 rows of 128 B
-constexpr int kGroups = 2, kGroupWarps = 4;
-constexpr int kMmaWarp = kGroups * kGroupWarps;   // 8
-constexpr int kTmaWarp = kMmaWarp + 1;            // TMA warps 9 .. 9 + kProducers - 1
-constexpr int kProducers = 3;                     // tile k is loaded by TMA warp k % kProducers
-constexpr int kThreads = (kTmaWarp + kProducers) * 32;
-constexpr uint32_t kTmemCols = 128;      // per group 64: S^T x 2 (columns 0, 16), O^T (32)
-constexpr uint32_t kGroupCols = 64;
+constexpr int kSoftmaxWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kTmaWarp = 5;              // TMA warps 5, 6 load K tiles, 7, 8 V tiles
+constexpr int kRingWarps = 2;            // TMA warps per ring
+constexpr int kThreads = (kTmaWarp + 2 * kRingWarps) * 32;
+constexpr uint32_t kTmemCols = 64;       // S^T x 2 (columns 0, 16), O^T (32)
 constexpr uint32_t kColO = 32;
 // shared memory from the 1024-aligned base
-constexpr int kOffV = kStages * kTileBytes;
-constexpr int kOffQ = 2 * kStages * kTileBytes;
-constexpr int kOffP = kOffQ + kN * 128;            // [group][hi, lo][128 tokens][16 B]
+constexpr int kOffV = kStagesK * kTileBytes;
+constexpr int kOffQ = (kStagesK + kStagesV) * kTileBytes;
+constexpr int kOffP = kOffQ + kN * 128;  // P': [hi, lo][128 tokens][16 B]
 constexpr int kPBuf = 2 * kTok * 16;
-constexpr int kOffIds = kOffP + kGroups * kPBuf;
+constexpr int kOffIds = kOffP + kPBuf;
 constexpr float kLazy = 8.f;             // base-2 margin of the lazy maximum
 
 // Byte offset of 16-byte chunk c of row r of a 128-byte-swizzled K-major
@@ -105,7 +107,7 @@ __device__ __forceinline__ float2 q_pair(uint32_t w) {
 }
 
 template <class QF, int G>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, G <= 4 ? 3 : 2)
     paged_decode_fp8_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
                                const __grid_constant__ CUtensorMap vmap) {
   static_assert(G >= 1 && 2 * G <= kN, "query group");
@@ -117,52 +119,47 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sq = smem + kOffQ;
+  uint8_t* sp = smem + kOffP;
   int32_t* ids = reinterpret_cast<int32_t*>(smem + kOffIds);
-  auto sk = [&](int k) { return smem + (k % kStages) * kTileBytes; };
-  auto sv = [&](int k) { return smem + kOffV + (k % kStages) * kTileBytes; };
-  auto sp = [&](int g) { return smem + kOffP + g * kPBuf; };
-  // kfull/vfull: a tile's boxes landed; kempty/vempty: the MMAs reading the
-  // stage completed. Per group g: s_full[g][b] S^T buffer b computed;
-  // s_free[g][b] the group read it; p_full[g] the group wrote P' (and
-  // rescaled O); p_free[g] O += P V that read it completed; red_bar[g][b] the
-  // group's tile maxima posted; sum_bar[g] its partial sums posted;
-  // merge_bar the second group's result posted for the first.
-  __shared__ uint64_t kfull[kStages], kempty[kStages], vfull[kStages], vempty[kStages],
-      s_full[kGroups][2], s_free[kGroups][2], p_full[kGroups], p_free[kGroups],
-      red_bar[kGroups][2], sum_bar[kGroups], merge_bar, drain_bar;
+  auto sk = [&](int k) { return smem + (k % kStagesK) * kTileBytes; };
+  auto sv = [&](int k) { return smem + kOffV + (k % kStagesV) * kTileBytes; };
+  // kfull/vfull: a tile's boxes landed (one arrival per TMA warp of the
+  // ring); kempty/vempty: the MMAs reading the stage completed; s_full[b]:
+  // S^T buffer b computed; s_free[b]: the softmax warps read it; p_full: P'
+  // written (and O rescaled); p_free: O += P V that read it completed;
+  // red_bar[b]: the four warps' tile maxima posted; sum_bar: their partial
+  // sums posted.
+  __shared__ uint64_t kfull[kStagesK], kempty[kStagesK], vfull[kStagesV], vempty[kStagesV],
+      s_full[2], s_free[2], p_full, p_free, red_bar[2], sum_bar, drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int aborted;
-  __shared__ int last_k[kStages], last_v[kStages];  // last tile loaded into each stage
   __shared__ float qscale_s[G];
-  __shared__ float red[kGroups][2][kGroupWarps][G];
-  __shared__ float lsum[kGroups][kGroupWarps][G];
-  __shared__ float merge_ml[2][G];                   // second group: (max, sum) per head
+  __shared__ float red[2][kSoftmaxWarps][G];
+  __shared__ float lsum[kSoftmaxWarps][G];
 
   const int kvh = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint64_t lim = a.wait_limit_ns;
   if (tid == 0) {
-    for (int r = 0; r < kStages; ++r) {
-      mbar_init(&kfull[r], 1);
+    for (int r = 0; r < kStagesK; ++r) {
+      mbar_init(&kfull[r], kRingWarps);
       mbar_init(&kempty[r], 1);
-      mbar_init(&vfull[r], 1);
+    }
+    for (int r = 0; r < kStagesV; ++r) {
+      mbar_init(&vfull[r], kRingWarps);
       mbar_init(&vempty[r], 1);
     }
-    for (int g = 0; g < kGroups; ++g) {
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&s_full[g][b], 1);
-        mbar_init(&s_free[g][b], kGroupWarps);
-        mbar_init(&red_bar[g][b], kGroupWarps);
-      }
-      mbar_init(&p_full[g], kGroupWarps);
-      mbar_init(&p_free[g], 1);
-      mbar_init(&sum_bar[g], kGroupWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], kSoftmaxWarps);
+      mbar_init(&red_bar[b], kSoftmaxWarps);
     }
-    mbar_init(&merge_bar, kGroupWarps);
+    mbar_init(&p_full, kSoftmaxWarps);
+    mbar_init(&p_free, 1);
+    mbar_init(&sum_bar, kSoftmaxWarps);
     mbar_init(&drain_bar, 1);
     fence_mbar_init();
     aborted = 0;
-    for (int r = 0; r < kStages; ++r) last_k[r] = last_v[r] = -1;
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
   }
@@ -195,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     ids[i] = id;
   }
   // Q' -> shared memory: one warp per query head; lane l holds dims 4l..4l+3
-  if (warp < kGroups * kGroupWarps) {
-    for (int g = warp; g < G; g += kGroups * kGroupWarps) {
+  if (warp < kSoftmaxWarps) {
+    for (int g = warp; g < G; g += kSoftmaxWarps) {
       const uint2 raw = *reinterpret_cast<const uint2*>(
           static_cast<const uint8_t*>(a.query) +
           ((static_cast<int64_t>(s) * a.num_heads + kvh * G + g) * 128 + 4 * lane) * 2);
@@ -218,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       *reinterpret_cast<uint32_t*>(sq + sw128_off(G + g, c) + b) = lo;
       if (lane == 0) qscale_s[g] = a.scale_log2 * a.k_scale[kvh] * ldexpf(1.f, -e);
     }
-    for (int i = tid; i < (kN - 2 * G) * 8; i += kGroups * kGroupWarps * 32)
+    for (int i = tid; i < (kN - 2 * G) * 8; i += kSoftmaxWarps * 32)
       *reinterpret_cast<uint4*>(sq + sw128_off(2 * G + i / 8, i % 8)) = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
@@ -230,63 +227,53 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem = tmem_slot;
 
   if (warp >= kTmaWarp) {
-    // ================= TMA loads (one thread per TMA warp) =================
-    // Issuing a tensor load costs its thread hundreds of cycles, and a tile is
-    // 16 boxes of 2 KB: the tiles are dealt to kProducers warps so that
-    // enough loads are issued per SM.
+    // ================= TMA loads: two warps per ring =================
+    // Box j of a tile is issued by lane j / kRingWarps of the ring's warp
+    // j % kRingWarps; each warp's lane 0 posts the bytes of its boxes.
     const int producer = warp - kTmaWarp;
-    if (lane == 0) {
-      const uint64_t policy = l2_policy_evict_first();
-      auto issue = [&](int k, bool is_v) {
-        uint8_t* dst = is_v ? sv(k) : sk(k);
-        uint64_t* bar = is_v ? &vfull[k % kStages] : &kfull[k % kStages];
-        const CUtensorMap* map = is_v ? &vmap : &kmap;
-        const int u0 = k * kTok;
-        const int nsub = (min(kTok, ntok - u0) + TR - 1) / TR;  // boxes holding context tokens
-        if (!is_v && a.skip_tile >= u0 / TR && a.skip_tile < u0 / TR + nsub &&
-            skip_for_test(a.skip_tile, a.skip_tile))
-          return;
-        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nsub * TR * 128));
-        for (int j = 0; j < nsub; ++j) {
-          const int u = u0 + j * TR;
-          const int32_t bid = ids[u / a.block_size];
-          const int32_t row0 = bid >= 0 ? bid * a.block_size + u % a.block_size : -TR;
-          tma_load_4d(dst + j * TR * 128, map, bar, 0, row0, kvh, 0, policy);
-        }
-      };
-      bool ok = true;
-      int k = producer;
-      for (; ok && k < ntiles; k += kProducers) {
-        if (k >= kStages)
-          ok = mbar_wait(&kempty[k % kStages], ((k - kStages) / kStages) & 1, lim, &aborted);
-        if (!ok) break;
-        issue(k, false);
-        atomicMax(&last_k[k % kStages], k);
-        if (k >= kStages)
-          ok = mbar_wait(&vempty[k % kStages], ((k - kStages) / kStages) & 1, lim, &aborted);
-        if (!ok) break;
-        issue(k, true);
-        atomicMax(&last_v[k % kStages], k);
+    const bool is_v = producer >= kRingWarps;
+    const int pr = producer % kRingWarps;
+    const int NS_ = is_v ? kStagesV : kStagesK;
+    uint64_t* full = is_v ? vfull : kfull;
+    uint64_t* empty = is_v ? vempty : kempty;
+    const CUtensorMap* map = is_v ? &vmap : &kmap;
+    const uint64_t policy = l2_policy_evict_first();
+    bool ok = true;
+    int k = 0, issued = 0;
+    for (; k < ntiles; ++k) {
+      if (k >= NS_)
+        ok = __all_sync(FULL, mbar_wait(&empty[k % NS_], ((k - NS_) / NS_) & 1, lim, &aborted));
+      if (!ok) break;
+      uint8_t* dst = is_v ? sv(k) : sk(k);
+      uint64_t* bar = &full[k % NS_];
+      const int u0 = k * kTok;
+      const int nsub = (min(kTok, ntok - u0) + TR - 1) / TR;  // boxes holding context tokens
+      issued = k + 1;
+      if (!is_v && a.skip_tile >= u0 / TR && a.skip_tile < u0 / TR + nsub &&
+          skip_for_test(a.skip_tile, a.skip_tile))
+        continue;  // (both K warps leave it out: the tile never completes)
+      const int mine = nsub > pr ? (nsub - pr + kRingWarps - 1) / kRingWarps : 0;
+      if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(mine * TR * 128));
+      __syncwarp();
+      if (lane < mine) {
+        const int j = pr + kRingWarps * lane;
+        const int u = u0 + j * TR;
+        const int32_t bid = ids[u / a.block_size];
+        const int32_t row0 = bid >= 0 ? bid * a.block_size + u % a.block_size : -TR;
+        tma_load_4d(dst + j * TR * 128, map, bar, 0, row0, kvh, 0, policy);
       }
-      if (!ok) {
-        record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 0, k, ntiles, 0);
-        aborted = 1;
-        report(a.err, kErrWaitTimeout);
-      }
+      __syncwarp();
     }
-    // Every issued load lands before the CTA's shared memory goes away: once
-    // all TMA warps stopped (their loops end in bounded time), the last load
-    // of each stage is waited for (earlier ones were consumed before the stage
-    // was reused). The warp reconverges first: the named barrier is executed
-    // by whole warps.
-    __syncwarp();
-    asm volatile("bar.sync 1, %0;" ::"n"(kProducers * 32) : "memory");
-    if (producer == 0 && lane == 0) {
-      for (int r = 0; r < kStages; ++r) {
-        if (last_k[r] >= 0) mbar_wait(&kfull[r], (last_k[r] / kStages) & 1, lim);
-        if (last_v[r] >= 0) mbar_wait(&vfull[r], (last_v[r] / kStages) & 1, lim);
-      }
+    if (!ok && lane == 0) {
+      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 0, k, ntiles, producer);
+      aborted = 1;
+      report(a.err, kErrWaitTimeout);
     }
+    // every load this warp issued lands before the CTA's shared memory goes
+    // away (the last use of each stage; earlier ones were consumed)
+    if (lane == 0)
+      for (int t = max(0, issued - NS_); t < issued; ++t)
+        mbar_wait(&full[t % NS_], (t / NS_) & 1, lim);
     __syncwarp();  // whole warps reach the CTA barrier below
   } else if (warp == kMmaWarp) {
     // ================= MMA issue (one thread) =================
@@ -299,53 +286,56 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t qd = tc::sw128_desc(sq, 16, 1024);
       const uint64_t kd0 = tc::sw128_desc(smem, 16, 1024);
       const uint64_t vd0 = tc::sw128_desc(smem + kOffV, kTileBytes, 1024);
-      const uint64_t pd0 = tc::plain_desc(smem + kOffP, 128, 128);
-      int k = 0;
-      // tile t belongs to group t & 1 as its (t >> 1)-th tile
-      auto issue_s = [&](int t) {
-        const int g = t & 1, j = t >> 1;
-        if (j >= 2 && !mbar_wait(&s_free[g][j & 1], ((j - 2) >> 1) & 1, lim, &aborted))
-          return false;
-        if (!mbar_wait(&kfull[t % kStages], (t / kStages) & 1, lim, &aborted)) return false;
-        tc::fence_after_sync();
-        const uint64_t kd = kd0 + static_cast<uint64_t>(((t % kStages) * kTileBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // 32 dims (bytes) per K step
-          tc::mma_f8(tmem + g * kGroupCols + (j & 1) * kN, kd + 2 * kk, qd + 2 * kk, IDESC_S,
-                     kk > 0);
-        tc::commit(&s_full[g][j & 1]);
-        tc::commit(&kempty[t % kStages]);
-        return true;
-      };
+      const uint64_t ph = tc::plain_desc(sp, 128, 128);
+      const uint64_t pl = ph + static_cast<uint64_t>((kTok * 16) >> 4);
+      // Issue whichever is ready: S of the next tile (its S buffer read by the
+      // softmax warps, its K landed) or O += P V of the oldest tile whose P
+      // is posted (and V landed), so neither waits behind the other. Gives
+      // up after the wait limit without progress.
       bool ok = true;
-      for (int t = 0; ok && t < min(2, ntiles); ++t) ok = issue_s(t);
-      for (; ok && k < ntiles; ++k) {
-        // S of the group's next tile first, then O += P V of tile k
-        if (k + 2 < ntiles) ok = issue_s(k + 2);
-        if (!ok) break;
-        const int g = k & 1, j = k >> 1;
-        ok = mbar_wait(&vfull[k % kStages], (k / kStages) & 1, lim, &aborted) &&
-             mbar_wait(&p_full[g], j & 1, lim, &aborted);
-        if (!ok) break;
-        tc::fence_after_sync();
-        const uint64_t vd = vd0 + static_cast<uint64_t>(((k % kStages) * kTileBytes) >> 4);
-        const uint64_t ph = pd0 + static_cast<uint64_t>((g * kPBuf) >> 4);
-        const uint64_t pl = ph + static_cast<uint64_t>((kTok * 16) >> 4);
-        const uint32_t to = tmem + g * kGroupCols + kColO;
+      int ns = 0, k = 0;  // next tile for S, for P V
+      uint64_t t_last = global_timer_ns();
+      while (k < ntiles) {
+        bool progress = false;
+        if (ns < ntiles && (ns < 2 || mbar_test_wait(&s_free[ns & 1], ((ns - 2) >> 1) & 1)) &&
+            mbar_test_wait(&kfull[ns % kStagesK], (ns / kStagesK) & 1)) {
+          tc::fence_after_sync();
+          const uint64_t kd = kd0 + static_cast<uint64_t>(((ns % kStagesK) * kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kTok / 32; ++kk) {  // 32 tokens per K step
-          const uint64_t av = vd + static_cast<uint64_t>((kk * 32 * 128) >> 4);
-          const uint64_t off = static_cast<uint64_t>((kk * 32 * 16) >> 4);
-          tc::mma_f8(to, av, ph + off, IDESC_O_HI, j > 0 || kk > 0);
-          tc::mma_f8(to, av, pl + off, IDESC_O_LO, true);
+          for (int kk = 0; kk < 4; ++kk)  // 32 dims (bytes) per K step
+            tc::mma_f8(tmem + (ns & 1) * kN, kd + 2 * kk, qd + 2 * kk, IDESC_S, kk > 0);
+          tc::commit(&s_full[ns & 1]);
+          tc::commit(&kempty[ns % kStagesK]);
+          ++ns;
+          progress = true;
         }
-        tc::commit(&p_free[g]);
-        tc::commit(&vempty[k % kStages]);
+        if (k < ns && mbar_test_wait(&vfull[k % kStagesV], (k / kStagesV) & 1) &&
+            mbar_test_wait(&p_full, k & 1)) {
+          tc::fence_after_sync();
+          const uint64_t vd = vd0 + static_cast<uint64_t>(((k % kStagesV) * kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kTok / 32; ++kk) {  // 32 tokens per K step
+            const uint64_t av = vd + static_cast<uint64_t>((kk * 32 * 128) >> 4);
+            const uint64_t off = static_cast<uint64_t>((kk * 32 * 16) >> 4);
+            tc::mma_f8(tmem + kColO, av, ph + off, IDESC_O_HI, k > 0 || kk > 0);
+            tc::mma_f8(tmem + kColO, av, pl + off, IDESC_O_LO, true);
+          }
+          tc::commit(&p_free);
+          tc::commit(&vempty[k % kStagesV]);
+          ++k;
+          progress = true;
+        }
+        if (progress) {
+          t_last = global_timer_ns();
+        } else if (aborted || global_timer_ns() - t_last > lim) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) {
         // A wait gave up (never expected): let this CTA's MMAs finish (bounded)
         // before its tensor and shared memory go away.
-        record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 1, k, ntiles, 0);
+        record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 1, k, ntiles, ns);
         aborted = 1;
         report(a.err, kErrWaitTimeout);
         tc::commit(&drain_bar);
@@ -354,13 +344,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncwarp();  // whole warps reach the CTA barrier below
   } else {
-    // ================= softmax warps (two groups) =================
-    const int grp = warp / kGroupWarps, gw = warp % kGroupWarps;
-    const int gtid = tid - grp * kGroupWarps * 32;      // token / dimension of this thread
-    const uint32_t lane_base = static_cast<uint32_t>(gw * 32) << 16;
-    const uint32_t tbase = tmem + grp * kGroupCols;
-    const int ntg = ntiles > grp ? (ntiles - grp + 1) / 2 : 0;  // tiles of this group
-    uint8_t* pbuf = sp(grp);
+    // ================= softmax warps =================
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     float m[G], l[G], qs[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -369,43 +354,42 @@ __global__ void __launch_bounds__(kThreads, 2)
       qs[g] = qscale_s[g];
     }
     bool ok = true;
-    int j = 0;
-    for (; ok && j < ntg; ++j) {
-      const int k = 2 * j + grp;  // the tile
-      ok = __all_sync(FULL, mbar_wait(&s_full[grp][j & 1], (j >> 1) & 1, lim, &aborted));
+    int k = 0;
+    for (; ok && k < ntiles; ++k) {
+      ok = __all_sync(FULL, mbar_wait(&s_full[k & 1], (k >> 1) & 1, lim, &aborted));
       if (!ok) break;
       tc::fence_after_sync();
       uint32_t r[NL];
-      if constexpr (NL == 8) tc::ld8_nowait(tbase + (j & 1) * kN + lane_base, r);
-      else tc::ld16_nowait(tbase + (j & 1) * kN + lane_base, r);
+      if constexpr (NL == 8) tc::ld8_nowait(tmem + (k & 1) * kN + lane_base, r);
+      else tc::ld16_nowait(tmem + (k & 1) * kN + lane_base, r);
       tc::wait_ld();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[grp][j & 1]);
+      if (lane == 0) mbar_arrive(&s_free[k & 1]);
       const int vk = min(kTok, ntok - k * kTok);  // context tokens in this tile
-      const bool live = gtid < vk;
+      const bool live = tid < vk;
       float x[G];
 #pragma unroll
       for (int g = 0; g < G; ++g)
         x[g] = live ? (__uint_as_float(r[g]) + __uint_as_float(r[G + g])) * qs[g]
                     : -CUDART_INF_F;
-      // the tile's maximum per head over the group
+      // the tile's maximum per head over the CTA
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const int mx = __reduce_max_sync(FULL, ord_of(x[g]));
-        if (lane == 0) red[grp][j & 1][gw][g] = float_of(mx);
+        if (lane == 0) red[k & 1][warp][g] = float_of(mx);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&red_bar[grp][j & 1]);
-      ok = __all_sync(FULL, mbar_wait(&red_bar[grp][j & 1], (j >> 1) & 1, lim, &aborted));
+      if (lane == 0) mbar_arrive(&red_bar[k & 1]);
+      ok = __all_sync(FULL, mbar_wait(&red_bar[k & 1], (k >> 1) & 1, lim, &aborted));
       if (!ok) break;
       float alpha[G];
       bool rescale = false;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float tmax = red[grp][j & 1][0][g];
+        float tmax = red[k & 1][0][g];
 #pragma unroll
-        for (int w = 1; w < kGroupWarps; ++w) tmax = fmaxf(tmax, red[grp][j & 1][w][g]);
+        for (int w = 1; w < kSoftmaxWarps; ++w) tmax = fmaxf(tmax, red[k & 1][w][g]);
         alpha[g] = 1.f;
         if (tmax > m[g] + kLazy) {  // false while the head has seen nothing
           alpha[g] = tc::ex2(m[g] - tmax);
@@ -422,22 +406,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         p[g] = tc::ex2(x[g] - mu);
         l[g] = fmaf(l[g], alpha[g], p[g]);
       }
-      // The group's P' buffer is free, and its O^T may be rescaled, once
-      // O += P V of its previous tile completed
-      if (j >= 1) {
-        ok = __all_sync(FULL, mbar_wait(&p_free[grp], (j - 1) & 1, lim, &aborted));
+      // P' has one buffer, rewritten (and O^T rescaled) once O += P V of the
+      // previous tile completed
+      if (k >= 1) {
+        ok = __all_sync(FULL, mbar_wait(&p_free, (k - 1) & 1, lim, &aborted));
         if (!ok) break;
       }
-      if (rescale && j >= 1) {  // rare: the maximum moves lazily; uniform over the group
+      if (rescale && k >= 1) {  // rare: the maximum moves lazily; the same in every thread
         tc::fence_after_sync();
         uint32_t o[NL];
-        if constexpr (NL == 8) tc::ld8_nowait(tbase + kColO + lane_base, o);
-        else tc::ld16_nowait(tbase + kColO + lane_base, o);
+        if constexpr (NL == 8) tc::ld8_nowait(tmem + kColO + lane_base, o);
+        else tc::ld16_nowait(tmem + kColO + lane_base, o);
         tc::wait_ld();
 #pragma unroll
         for (int g = 0; g < G; ++g) o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
-        if constexpr (NL == 8) tc::st8u(tbase + kColO + lane_base, o);
-        else tc::st16u(tbase + kColO + lane_base, o);
+        if constexpr (NL == 8) tc::st8u(tmem + kColO + lane_base, o);
+        else tc::st16u(tmem + kColO + lane_base, o);
         tc::wait_st();
       }
       uint32_t hw[4], lw[4];
@@ -448,17 +432,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         hw[1] = lw[1] = 0u;
       }
       hw[2] = hw[3] = lw[2] = lw[3] = 0u;
-      *reinterpret_cast<uint4*>(pbuf + gtid * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(pbuf + kTok * 16 + gtid * 16) =
-          make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      *reinterpret_cast<uint4*>(sp + tid * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(sp + kTok * 16 + tid * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       // V rows without context tokens (end of the unit) may hold anything,
       // even NaN codes, and 0 * NaN is NaN inside the MMA: clear them once
       // the tile's loads landed
       if (vk < kTok) {
-        ok = __all_sync(FULL, mbar_wait(&vfull[k % kStages], (k / kStages) & 1, lim, &aborted));
+        ok = __all_sync(FULL, mbar_wait(&vfull[k % kStagesV], (k / kStagesV) & 1, lim, &aborted));
         if (!ok) break;
         if (!live) {
-          uint4* row = reinterpret_cast<uint4*>(sv(k) + gtid * 128);
+          uint4* row = reinterpret_cast<uint4*>(sv(k) + tid * 128);
 #pragma unroll
           for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -466,106 +449,63 @@ __global__ void __launch_bounds__(kThreads, 2)
       fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[grp]);
+      if (lane == 0) mbar_arrive(&p_full);
     }
-    if (ok && ntg > 0)
-      ok = __all_sync(FULL, mbar_wait(&p_free[grp], (ntg - 1) & 1, lim, &aborted));
+    if (ok && ntiles > 0)
+      ok = __all_sync(FULL, mbar_wait(&p_free, (ntiles - 1) & 1, lim, &aborted));
     // A warp that gave up says so before it posts its sums, so that the
     // others, which wait for those, see the flag.
     if (!ok && lane == 0) {
-      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 2 + grp, 2 * j + grp, ntiles, 0);
+      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 2, k, ntiles, 0);
       aborted = 1;
       report(a.err, kErrWaitTimeout);
     }
-    // the group's partial sums (every warp of the group posts its own)
+    // the partial sums over the CTA (every softmax warp posts its own)
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float v = l[g];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-      if (lane == 0) lsum[grp][gw][g] = v;
+      if (lane == 0) lsum[warp][g] = v;
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sum_bar[grp]);
-    const bool sums = __all_sync(FULL, mbar_wait(&sum_bar[grp], 0, lim, &aborted));
+    if (lane == 0) mbar_arrive(&sum_bar);
+    const bool sums = __all_sync(FULL, mbar_wait(&sum_bar, 0, lim, &aborted));
     if (!sums && lane == 0) {
-      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 4 + grp, 2 * j + grp, ntiles, 0);
+      record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 3, k, ntiles, 0);
       aborted = 1;
       report(a.err, kErrWaitTimeout);
     }
-    // thread i holds dimension i of the group's O for every head: normalised
-    // by the group's sum (0 where the group saw no token)
-    float L[G], on[G];
+    __syncwarp();
+    // A unit whose result is lost leaves zeros (single pass) or an empty
+    // partial that the combine kernel gives no weight, never stale data.
+    const bool good = __all_sync(FULL, ok && sums && *static_cast<volatile int*>(&aborted) == 0);
+    // ---- epilogue: thread i holds dimension i of every head's O
+    uint32_t o[NL];
+#pragma unroll
+    for (int i = 0; i < NL; ++i) o[i] = 0u;
+    if (good && ntiles > 0) {
+      tc::fence_after_sync();
+      if constexpr (NL == 8) tc::ld8_nowait(tmem + kColO + lane_base, o);
+      else tc::ld16_nowait(tmem + kColO + lane_base, o);
+      tc::wait_ld();
+    }
+    const bool single = parts == 1;
+    const int64_t row0 = static_cast<int64_t>(s) * a.num_heads + kvh * G;
+    const float vs = a.v_scale[kvh];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      L[g] = 0.f;
+      float L = 0.f;
 #pragma unroll
-      for (int w = 0; w < kGroupWarps; ++w) L[g] += lsum[grp][w][g];
-      on[g] = 0.f;
-    }
-    if (ok && sums && ntg > 0) {
-      tc::fence_after_sync();
-      uint32_t o[NL];
-      if constexpr (NL == 8) tc::ld8_nowait(tbase + kColO + lane_base, o);
-      else tc::ld16_nowait(tbase + kColO + lane_base, o);
-      tc::wait_ld();
-#pragma unroll
-      for (int g = 0; g < G; ++g) on[g] = L[g] > 0.f ? __uint_as_float(o[g]) / L[g] : 0.f;
-    }
-    // the second group hands (max, sum, O / sum) to the first through shared
-    // memory: the first K stage, which is idle once the group's last
-    // O += P V completed (every S, issued before it, is done then, and no K
-    // load follows); a group without a tile, or that gave up, posts sum 0 and
-    // leaves that memory alone
-    float* mo = reinterpret_cast<float*>(smem);   // [128 dims][G]
-    if (grp == 1) {
-      const bool has = ok && sums && ntg > 0;
-      if (has) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) mo[gtid * G + g] = on[g];
-      }
-      if (gtid == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          merge_ml[0][g] = m[g];
-          merge_ml[1][g] = has ? L[g] : 0.f;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&merge_bar);
-    } else {
-      const bool merged = __all_sync(FULL, mbar_wait(&merge_bar, 0, lim, &aborted));
-      if (!merged && lane == 0) {
-        record_failure(a.diag, kSiteFp8Tile, kvh, s, part, 6, ntiles, ntiles, 0);
-        aborted = 1;
-        report(a.err, kErrWaitTimeout);
-      }
-      __syncwarp();
-      const bool good =
-          __all_sync(FULL, ok && sums && merged && *static_cast<volatile int*>(&aborted) == 0);
-      const bool single = parts == 1;
-      const int64_t row0 = static_cast<int64_t>(s) * a.num_heads + kvh * G;
-      const float vs = a.v_scale[kvh];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        // the two groups as two parts of the context: weights L 2^(m - M)
-        const float m1 = merge_ml[0][g], L1 = merge_ml[1][g];
-        const float M = fmaxf(m[g], m1);
-        const float w0 = L[g] > 0.f ? L[g] * tc::ex2(m[g] - M) : 0.f;
-        const float w1 = L1 > 0.f ? L1 * tc::ex2(m1 - M) : 0.f;
-        const float W = w0 + w1;
-        float val = w0 * on[g];
-        if (w1 > 0.f) val += w1 * mo[gtid * G + g];
-        val = W > 0.f ? val / W * vs : 0.f;
-        if (!good) val = 0.f;
-        if (single) {
-          store_out(QF{}, a.out, (row0 + g) * 128 + gtid, val);
-        } else {
-          const int64_t pi = (row0 + g) * a.max_parts + part;
-          a.ws_o[pi * 128 + gtid] = val;
-          if (gtid == 0)
-            a.ws_ml[pi] = good && W > 0.f ? make_float2(M, W) : make_float2(-CUDART_INF_F, 0.f);
-        }
+      for (int w = 0; w < kSoftmaxWarps; ++w) L += lsum[w][g];
+      const bool has = good && L > 0.f;
+      const float val = has ? __uint_as_float(o[g]) / L * vs : 0.f;
+      if (single) {
+        store_out(QF{}, a.out, (row0 + g) * 128 + tid, val);
+      } else {
+        const int64_t pi = (row0 + g) * a.max_parts + part;
+        a.ws_o[pi * 128 + tid] = val;
+        if (tid == 0) a.ws_ml[pi] = has ? make_float2(m[g], L) : make_float2(-CUDART_INF_F, 0.f);
       }
     }
   }

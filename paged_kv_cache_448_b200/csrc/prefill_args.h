@@ -62,13 +62,4 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& kmap,
                               int head_dim, int group, int32_t max_query_len,
                               cudaStream_t stream);
 
-// Short chunks (max_query_len * group <= 64 rows, head_dim 128, 16-bit
-// cache) on tcgen05 with the key tokens on M: one CTA per (sequence, kv-head,
-// part of the key range), a.partition_tiles a multiple of 8 (128-token
-// tiles), the combine kernel after a split. The tensor maps are the
-// one-segment boxes. cudaErrorNotSupported for other shapes.
-cudaError_t launch_prefill_tm(const PrefillArgs& a, const CUtensorMap& kmap,
-                              const CUtensorMap& vmap, int q_dtype, int head_dim, int group,
-                              int32_t max_query_len, cudaStream_t stream);
-
 }  // namespace paged

@@ -164,21 +164,30 @@ def test_cpu_baseline_runs_on_one_core_and_on_all_cores():
         assert allc["cores"] >= 1 and allc["value"] > 0
 
 
-def test_recorded_traffic_is_tied_to_the_decode_sources():
-    """roofline.traffic comes from profiles/traffic.json only for the workload
-    it was captured on and while the decode kernels' sources (decode_*.cu,
-    their headers, api.cu) still hash to the recorded digest."""
+def test_recorded_traffic_is_tied_to_the_sources():
+    """roofline.traffic comes from profiles/traffic.json only for the bench row
+    (decode, multi-token query, block copy) and workload it was captured on,
+    and while that row's kernel sources (its units, their headers, api.cu)
+    still hash to the recorded digest."""
     import json
 
     import bench
-    names = {os.path.basename(f) for f in bench.decode_sources()}
-    assert {"decode_kernel.cuh", "api.cu", "decode_f16_f16.cu", "decode_reduce.cu"} <= names
+    names = {os.path.basename(f) for f in bench.op_sources("decode")}
+    assert {"decode_kernel.cuh", "api.cu", "decode_f16_f16.cu", "decode_reduce.cu",
+            "decode_fp8_tc.cu"} <= names
     assert "prefill_tc.cu" not in names and "copy_blocks.cu" not in names
-    assert bench.recorded_traffic("gqa70b_long") is None
+    names = {os.path.basename(f) for f in bench.op_sources("prefill")}
+    assert {"prefill_tc.cu", "prefill_kernel.cu", "api.cu", "tc_common.cuh"} <= names
+    assert "decode_f16_f16.cu" not in names
+    assert {"copy_blocks.cu", "api.cu"} <= {os.path.basename(f)
+                                            for f in bench.op_sources("copy_blocks")}
+    assert bench.recorded_traffic("no such workload") is None
     with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
-        rec = json.load(f)["decode"]
-    got = bench.recorded_traffic(rec["workload"])
-    if rec["sources_sha256"] == bench.sources_digest():
-        assert got == rec["dram_read_bytes"] + rec["dram_write_bytes"]
-    else:
-        assert got is None
+        entries = json.load(f)["entries"]
+    for e in entries:
+        assert e["dram_bytes_per_launch"] == e["dram_read_bytes"] + e["dram_write_bytes"]
+        got = bench.recorded_traffic(e["workload"], e["op"])
+        if e["sources_sha256"] == bench.sources_digest(e["op"]):
+            assert got == e["dram_bytes_per_launch"]
+        else:
+            assert got is None
