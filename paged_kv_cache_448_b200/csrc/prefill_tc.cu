@@ -20,10 +20,10 @@
 //    buffer that step k-1 released, so S is computed under the softmax of
 //    step k, and O += P V of step k (A = P from tensor memory, V read
 //    MN-major) once the group posted P;
-//  * the TMA warp (one thread) loads K and V of 64 tokens per step into
+//  * two TMA warps, one per ring, load K and V of 64 tokens per step into
 //    2-stage rings (16-row boxes of one 128-byte segment each, so a stage is
-//    [segment][64 rows][128 B]), K of step k ahead of V of step k-1, and
-//    refills a stage when the MMAs that read it completed.
+//    [segment][64 rows][128 B]), the boxes of a step from all lanes of the
+//    warp at once, and refill a stage when the MMAs that read it completed.
 // The epilogue divides each row of O by its sum and stores it. When the key
 // range is split (few CTAs), a CTA takes one part of its 16-token tiles and
 // writes (max, sum) and its normalised O per row for the combine kernel, as
@@ -55,7 +55,6 @@ namespace {
 
 constexpr int kTcRows = 128;       // M: rows of one row group (one MMA)
 constexpr int kTcNT = 64;          // tokens per step
-constexpr int kTcStages = 2;
 constexpr uint32_t kTmemGroup = 256;  // tensor-memory columns per row group: S x 2, then O
 constexpr uint32_t kTmemO = 128;      // column of O within the group (S buffers at 0 and 64)
 
@@ -74,8 +73,9 @@ struct TcCfg {
   static constexpr int QG_BYTES = (FP8 ? 2 : NSEG) * QPART;
   static constexpr int KV_SEG = kTcNT * 128;        // one segment of K or V in a stage
   static constexpr int KV_BYTES = NSEG * KV_SEG;    // one stage of K (or V)
-  // ring depths (K, needed first by S, and V)
-  static constexpr int KR = kTcStages, VR = kTcStages;
+  // ring depths (K, needed first by S, and V); deeper rings (4 for 16-bit
+  // caches, 6 for E4M3, with two row groups) measured no faster
+  static constexpr int KR = 2, VR = 2;
   static constexpr int OFF_K = NG * QG_BYTES;                   // K ring
   static constexpr int OFF_V = OFF_K + KR * KV_BYTES;           // V ring
   static constexpr int BYTES = OFF_V + VR * KV_BYTES;
@@ -108,14 +108,14 @@ __device__ __forceinline__ float2 unpack_q(uint32_t w) {
 }
 
 template <class QF, class CF, int D, int G, int NG>
-__global__ void __launch_bounds__(NG * kTcRows + 64, 1)
+__global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
     paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap kmap,
                             const __grid_constant__ CUtensorMap vmap) {
   using C = TcCfg<QF, CF, D, G, NG>;
   constexpr bool BF = C::BF, FP8 = C::FP8;
   constexpr int NSEG = C::NSEG, QT = C::QT, KR = C::KR, VR = C::VR, NT = kTcNT, TR = kTileRows;
   constexpr int kMma = NG * kTcRows / 32;   // warp issuing the MMAs (owns the tensor memory)
-  constexpr int kLoader = kMma + 1;         // warp issuing the TMA loads
+  constexpr int kLoader = kMma + 1;         // warps issuing the TMA loads: K, then V
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -259,78 +259,67 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
   tc::fence_after_sync();
   const uint32_t tmem = tmem_slot;
 
-  if (warp == kLoader) {
-    // ================= TMA loads (one thread) =================
-    // K of step k is issued before V of step k-1: K (needed first, by S) never
-    // waits behind the release of a V stage.
-    if (lane == 0) {
-      const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
-      const uint64_t policy = l2_policy_evict_last();  // other query tiles read them too
-      auto issue = [&](int k, const int32_t (&bid)[NT / TR], bool is_v) {
-        uint8_t* dst = is_v ? sv(k) : sk(k);
-        uint64_t* bar = is_v ? &vfull[k % VR] : &kfull[k % KR];
-        const CUtensorMap* map = is_v ? &vmap : &kmap;
-        const int t_begin = (kbase + k) * (NT / TR), t_end = min(tend, t_begin + NT / TR);
-        if (!is_v && a.skip_tile >= t_begin - tbase && a.skip_tile < t_end - tbase &&
-            skip_for_test(a.skip_tile, a.skip_tile))
-          return;
+  if (warp >= kLoader) {
+    // ================= TMA loads: a K warp and a V warp =================
+    // Each ring has a warp of its own, so a V stage (held until O += P V)
+    // never holds back a K load. The boxes of a step (16 rows of one 128-byte
+    // segment each) leave from all lanes of the warp at once, lane b issuing
+    // box b; each lane reads its block id one step ahead.
+    constexpr int BOXES = (NT / TR) * NSEG;
+    static_assert(BOXES <= 32, "one box per lane");
+    const bool is_v = warp == kLoader + 1;
+    const int R = is_v ? VR : KR;
+    uint64_t* full = is_v ? vfull : kfull;
+    uint64_t* empty = is_v ? vempty : kempty;
+    const CUtensorMap* map = is_v ? &vmap : &kmap;
+    const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq;
+    const uint64_t policy = l2_policy_evict_last();  // other query tiles read them too
+    const int bj = lane / NSEG, bsg = lane % NSEG;   // this lane's 16-row tile and segment
+    auto load_id = [&](int k) {
+      const int t = (kbase + k) * (NT / TR) + bj;
+      return lane < BOXES && k < nsteps && t < tend ? table[(t * TR) / a.block_size] : 0;
+    };
+    bool ok = true;
+    int issued = 0;
+    int32_t bid = load_id(0);
+    for (int k = 0; k < nsteps; ++k) {
+      const int32_t nbid = load_id(k + 1);  // in flight during the wait below
+      if (k >= R)
+        ok = __all_sync(0xffffffffu, mbar_wait(&empty[k % R], ((k - R) / R) & 1, lim, &aborted));
+      if (!ok) break;
+      issued = k + 1;
+      const int t_begin = (kbase + k) * (NT / TR), t_end = min(tend, t_begin + NT / TR);
+      if (!is_v && a.skip_tile >= t_begin - tbase && a.skip_tile < t_end - tbase &&
+          skip_for_test(a.skip_tile, a.skip_tile)) {
+        bid = nbid;
+        continue;  // (the K warp leaves it out: the step never completes)
+      }
+      uint64_t* bar = &full[k % R];
+      if (lane == 0)
         mbar_arrive_expect_tx(bar, static_cast<uint32_t>(NSEG * (t_end - t_begin) * TR * 128));
-#pragma unroll
-        for (int j = 0; j < NT / TR; ++j) {
-          const int t = t_begin + j;
-          if (t >= t_end) break;
-          int32_t b = bid[j];
-          if (b < 0 || b >= a.num_blocks) {
-            if (!is_v) report(a.err, kErrBadBlockId);
-            b = -1;  // read as a box outside the pool: zero-filled
-          }
-          const int32_t row0 = b >= 0 ? b * a.block_size + (t * TR) % a.block_size : -TR;
-#pragma unroll
-          for (int sg = 0; sg < NSEG; ++sg)
-            tma_load_4d(dst + sg * C::KV_SEG + j * TR * 128, map, bar, 0, row0, kvh, sg, policy);
+      __syncwarp();
+      const int t = t_begin + bj;
+      if (lane < BOXES && t < t_end) {
+        int32_t b = bid;
+        if (b < 0 || b >= a.num_blocks) {
+          if (!is_v) report(a.err, kErrBadBlockId);
+          b = -1;  // read as a box outside the pool: zero-filled
         }
-      };
-      // block ids: of step k (for K) and of step k-1 (kept for V)
-      int32_t bid[NT / TR], pbid[NT / TR];
-      auto load_ids = [&](int k, int32_t (&dst)[NT / TR]) {
-#pragma unroll
-        for (int j = 0; j < NT / TR; ++j) {
-          const int t = (kbase + k) * (NT / TR) + j;
-          dst[j] = t < tend ? table[(t * TR) / a.block_size] : 0;
-        }
-      };
-      bool ok = true;
-      int kk_issued = 0, vv_issued = 0;
-      for (int k = 0; ok && k <= nsteps; ++k) {
-        if (k < nsteps) {
-          load_ids(k, bid);
-          if (k >= KR) ok = mbar_wait(&kempty[k % KR], ((k - KR) / KR) & 1, lim, &aborted);
-          if (ok) {
-            issue(k, bid, false);
-            kk_issued = k + 1;
-          }
-        }
-        if (ok && k >= 1) {
-          if (k - 1 >= VR) ok = mbar_wait(&vempty[(k - 1) % VR], ((k - 1 - VR) / VR) & 1, lim, &aborted);
-          if (ok) {
-            issue(k - 1, pbid, true);
-            vv_issued = k;
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < NT / TR; ++j) pbid[j] = bid[j];
+        const int32_t row0 = b >= 0 ? b * a.block_size + (t * TR) % a.block_size : -TR;
+        uint8_t* dst = (is_v ? sv(k) : sk(k)) + bsg * C::KV_SEG + bj * TR * 128;
+        tma_load_4d(dst, map, bar, 0, row0, kvh, bsg, policy);
       }
-      if (!ok) {
-        aborted = 1;
-        report(a.err, kErrWaitTimeout);
-      }
-      // before the CTA's shared memory goes away every issued load must have
-      // landed (the last use of each stage; earlier ones completed already)
-      for (int j = max(0, kk_issued - KR); j < kk_issued; ++j)
-        mbar_wait(&kfull[j % KR], (j / KR) & 1, lim);
-      for (int j = max(0, vv_issued - VR); j < vv_issued; ++j)
-        mbar_wait(&vfull[j % VR], (j / VR) & 1, lim);
+      __syncwarp();
+      bid = nbid;
     }
+    if (!ok && lane == 0) {
+      aborted = 1;
+      report(a.err, kErrWaitTimeout);
+    }
+    // before the CTA's shared memory goes away every issued load must have
+    // landed (the last use of each stage; earlier ones completed already)
+    if (lane == 0)
+      for (int j = max(0, issued - R); j < issued; ++j) mbar_wait(&full[j % R], (j / R) & 1, lim);
     __syncwarp();  // whole warps reach the CTA barrier below
   } else if (warp == kMma) {
     // ================= MMA issue (one thread) =================
@@ -497,18 +486,23 @@ __global__ void __launch_bounds__(NG * kTcRows + 64, 1)
         tc::st16u(t_p + 16, wl);
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       } else {
-        uint32_t w[NT / 2], wl[NT / 2];
-#pragma unroll
-        for (int i = 0; i < NT / 2; ++i) {
-          const float p0 = x[2 * i], p1 = x[2 * i + 1];
-          w[i] = pack_pair(BF, p0, p1);
-          if constexpr (BF)
-            wl[i] = pack2<true>(p0 - __uint_as_float(w[i] << 16),
-                                p1 - __uint_as_float(w[i] & 0xffff0000u));
-        }
+        // in two halves of 32 probabilities (16 columns each), so that fewer
+        // registers are live at once
         const uint32_t t_p = t_grp + (k & 1) * NT + lane_base;
-        tc::st32u(t_p, w);
-        if constexpr (BF) tc::st32u(t_p + 32, wl);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w[NT / 4], wl[NT / 4];
+#pragma unroll
+          for (int i = 0; i < NT / 4; ++i) {
+            const float p0 = x[h * NT / 2 + 2 * i], p1 = x[h * NT / 2 + 2 * i + 1];
+            w[i] = pack_pair(BF, p0, p1);
+            if constexpr (BF)
+              wl[i] = pack2<true>(p0 - __uint_as_float(w[i] << 16),
+                                  p1 - __uint_as_float(w[i] & 0xffff0000u));
+          }
+          tc::st16u(t_p + h * NT / 4, w);
+          if constexpr (BF) tc::st16u(t_p + NT / 2 + h * NT / 4, wl);
+        }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
       // V rows without real data in this step (past the context, or tiles not
@@ -604,7 +598,7 @@ cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUten
   if (a.q_tiles != (max_query_len + C::QT - 1) / C::QT) return cudaErrorInvalidValue;
   e = launch_pdl(kern, dim3(static_cast<unsigned>(a.q_tiles * a.max_parts), a.num_kv_heads,
                             a.num_seqs),
-                 NG * kTcRows + 64, smem, stream, a, kmap, vmap);
+                 NG * kTcRows + 96, smem, stream, a, kmap, vmap);
   if (e != cudaSuccess || a.max_parts <= 1) return e;
   return launch_prefill_combine(a, std::is_same<QF, BF16>::value ? kBF16 : kF16, D, C::QT,
                                 max_query_len, stream);
