@@ -490,8 +490,8 @@ namespace {
 // with fewer CTAs or rows they run on the 64-row mma.sync kernel. When the
 // CTAs (query tiles x kv-heads x sequences) cannot fill a wave of the
 // tcgen05 kernel, or about four waves of three mma.sync CTAs per SM, the
-// tiles of each CTA are cut into parts of at least 256 tokens (16 tiles, a
-// multiple of 4) handled by separate CTAs and merged by a combine kernel.
+// tiles of each CTA are cut into parts of at least 256 tokens (16 tiles, whole
+// steps of the kernel) handled by separate CTAs and merged by a combine kernel.
 struct PrefillPlan {
   bool tc;                  // tcgen05 kernel (rows on M), else mma.sync
   int32_t q_tiles, partition_tiles, max_parts;
@@ -526,8 +526,11 @@ PrefillPlan make_prefill_plan(int32_t num_seqs, int32_t num_kv_heads, int32_t gr
   const int64_t by_work = (want + ctas - 1) / ctas;
   const int32_t parts = static_cast<int32_t>(std::min<int64_t>(by_work, max_tiles / 16));
   if (parts <= 1) return p;
+  // whole steps of the kernel: 4 tiles (64 tokens), 8 for the tcgen05 kernel
+  // with two row groups (128 tokens)
+  const int32_t step_tiles = p.tc && rows >= 256 ? 8 : 4;
   int32_t pt = (max_tiles + parts - 1) / parts;
-  pt = (pt + 3) / 4 * 4;
+  pt = (pt + step_tiles - 1) / step_tiles * step_tiles;
   p.partition_tiles = pt;
   p.max_parts = (max_tiles + pt - 1) / pt;
   return p;

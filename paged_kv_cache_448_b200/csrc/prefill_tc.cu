@@ -54,14 +54,21 @@ namespace paged {
 namespace {
 
 constexpr int kTcRows = 128;       // M: rows of one row group (one MMA)
-constexpr int kTcNT = 64;          // tokens per step
-constexpr uint32_t kTmemGroup = 256;  // tensor-memory columns per row group: S x 2, then O
-constexpr uint32_t kTmemO = 128;      // column of O within the group (S buffers at 0 and 64)
+constexpr uint32_t kTmemGroup = 256;  // tensor-memory columns per row group: S, then O
+constexpr uint32_t kTmemO = 128;      // column of O within the group
 
 // NG row groups of 128 rows share each K/V step (NG = 2: 256 rows, eight
-// softmax warps, and two independent MMA streams per step).
+// softmax warps, and two independent MMA streams per step). With one group a
+// step is 64 tokens and S has two buffers (S of step k+1 is computed under
+// the softmax of step k); with two groups a step is 128 tokens (S = Q K^T
+// with N = 128, which keeps the tensor core ahead of its shared-memory
+// operand reads) and each group has one S buffer: the other group's work
+// fills the tensor core while a group's softmax runs.
 template <class QF, class CF, int D, int G, int NG>
 struct TcCfg {
+  static constexpr int NT = NG == 2 ? 128 : 64;      // tokens per step
+  static constexpr int SB = NG == 2 ? 1 : 2;         // S buffers per group
+  static constexpr int H = NT / 64;                  // 64-token halves of a step
   static constexpr bool FP8 = CF::kBytes == 1;
   static constexpr bool BF = std::is_same<QF, BF16>::value;
   static constexpr int NSEG = D * CF::kBytes / 128;  // 128-byte segments of a cache row
@@ -71,7 +78,7 @@ struct TcCfg {
   // Q of one group: NSEG segments (16-bit), or the E4M3 hi and lo parts
   static constexpr int QPART = kTcRows * 128;
   static constexpr int QG_BYTES = (FP8 ? 2 : NSEG) * QPART;
-  static constexpr int KV_SEG = kTcNT * 128;        // one segment of K or V in a stage
+  static constexpr int KV_SEG = NT * 128;           // one segment of K or V in a stage
   static constexpr int KV_BYTES = NSEG * KV_SEG;    // one stage of K (or V)
   // ring depths (K, needed first by S, and V); deeper rings (4 for 16-bit
   // caches, 6 for E4M3, with two row groups) measured no faster
@@ -80,12 +87,12 @@ struct TcCfg {
   static constexpr int OFF_V = OFF_K + KR * KV_BYTES;           // V ring
   static constexpr int BYTES = OFF_V + VR * KV_BYTES;
   static constexpr uint32_t TMEM_COLS = NG * kTmemGroup;
-  static constexpr uint32_t IDESC_S = FP8 ? tc::idesc_f8<0, 0, kTcRows, kTcNT, false>()
-                                           : tc::idesc_f16<BF, kTcRows, kTcNT, false>();
+  static constexpr uint32_t IDESC_S = FP8 ? tc::idesc_f8<0, 0, kTcRows, NT, false>()
+                                           : tc::idesc_f16<BF, kTcRows, NT, false>();
   static constexpr uint32_t IDESC_PV = FP8 ? tc::idesc_f8<0, 0, kTcRows, D, true>()
                                             : tc::idesc_f16<BF, kTcRows, D, true>();
   static constexpr uint32_t IDESC_PV_LO = tc::idesc_f8<1, 0, kTcRows, D, true>();  // E5M2 P
-  static_assert(kTcNT == 64, "P (64 16-bit values) fills half of its S buffer's columns");
+  static_assert(SB * NT <= static_cast<int>(kTmemO), "S buffers below O");
   static_assert(BYTES + 1024 <= 227 * 1024, "shared memory of one CTA");
 };
 
@@ -113,7 +120,8 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
                             const __grid_constant__ CUtensorMap vmap) {
   using C = TcCfg<QF, CF, D, G, NG>;
   constexpr bool BF = C::BF, FP8 = C::FP8;
-  constexpr int NSEG = C::NSEG, QT = C::QT, KR = C::KR, VR = C::VR, NT = kTcNT, TR = kTileRows;
+  constexpr int NSEG = C::NSEG, QT = C::QT, KR = C::KR, VR = C::VR, NT = C::NT, TR = kTileRows;
+  constexpr int SB = C::SB, H = C::H;
   constexpr int kMma = NG * kTcRows / 32;   // warp issuing the MMAs (owns the tensor memory)
   constexpr int kLoader = kMma + 1;         // warps issuing the TMA loads: K, then V
 
@@ -186,7 +194,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
   const int pos0 = ctx - qlen + tok0;
   const int p_max = pos0 + ntok - 1;
   // 16-token tiles holding tokens 0..p_max, cut into parts of partition_tiles
-  // (a multiple of the 4 tiles of a step); this CTA takes part `part`: tiles
+  // (a multiple of the NT / 16 tiles of a step); this CTA takes part `part`: tiles
   // tbase .. tend-1, steps kbase .. kbase+nsteps-1
   const int ntiles_all = p_max / TR + 1;
   const int parts = (ntiles_all + a.partition_tiles - 1) / a.partition_tiles;
@@ -324,90 +332,114 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
   } else if (warp == kMma) {
     // ================= MMA issue (one thread) =================
     if (lane == 0) {
-      int k_waited = 0, v_waited = 0;
       // descriptors computed once; a k-step or stage offset is added to the
       // start-address field (bits 0-13, in 16-byte units)
       uint64_t qd[NG];
       for (int g = 0; g < NG; ++g) qd[g] = tc::sw128_desc(sq(g), 16, 1024);
       const uint64_t kd0 = tc::sw128_desc(sk(0), 16, 1024);
       const uint64_t vd0 = tc::sw128_desc(sv(0), NT * 128, 1024);
-      auto issue_s = [&](int k) {  // S of step k for every group
-        if (!mbar_wait(&kfull[k % KR], (k / KR) & 1, lim, &aborted)) return false;
-        k_waited = k + 1;
-        tc::fence_after_sync();
-        const uint64_t kd = kd0 + static_cast<uint64_t>(((k % KR) * C::KV_BYTES) >> 4);
+      // Per group: ns[g] = next step whose S is issued, np[g] = next step
+      // whose O += P V is issued. The thread polls and issues whatever is
+      // ready, so neither group waits behind the other:
+      //  * S(g, k): K of step k landed and the group's S buffer is free, i.e.
+      //    O += P V of step k - SB (which read the P written over that S)
+      //    completed;
+      //  * O += P V (g, k): S(g, k) issued, the group posted P of step k and
+      //    V of step k landed.
+      // A K stage is released once every group's S of its step was issued, a
+      // V stage once every group's O += P V (a commit completes when all of
+      // the thread's earlier MMAs have). Gives up after the wait limit
+      // without progress.
+      int ns[NG], np[NG];
+#pragma unroll
+      for (int g = 0; g < NG; ++g) ns[g] = np[g] = 0;
+      int k_rel = 0, v_rel = 0;  // K / V stages released so far (steps)
+      bool ok = true;
+      uint64_t t_last = global_timer_ns();
+      auto all_issued = [&](const int (&c)[NG]) {
+        int m = c[0];
+#pragma unroll
+        for (int g = 1; g < NG; ++g) m = min(m, c[g]);
+        return m;
+      };
+      while (all_issued(np) < nsteps) {
+        bool progress = false;
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-          if constexpr (!FP8) {
+          const uint32_t t_grp = tmem + g * kTmemGroup;
+          const int j = np[g];
+          if (j < ns[g] && mbar_test_wait(&p_bar[g][j & 1], (j >> 1) & 1) &&
+              mbar_test_wait(&vfull[j % VR], (j / VR) & 1)) {
+            tc::fence_after_sync();
+            // P of step j over its S: per 32 tokens (quarter qq) the 16-bit
+            // pairs (or E4M3 codes) from column 32 qq, the bf16 (or E5M2)
+            // residual 16 (8) columns further; 8 columns per k-step
+            const uint32_t t_p = t_grp + (SB == 2 ? (j & 1) * NT : 0);
+            const uint32_t t_o = t_grp + kTmemO;
+            const uint64_t vd = vd0 + static_cast<uint64_t>(((j % VR) * C::KV_BYTES) >> 4);
+            if constexpr (!FP8) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const int sg = kk / 4, off = (kk % 4) * 32;
-              tc::mma_f16(tmem + g * kTmemGroup + (k & 1) * NT,
-                          qd[g] + static_cast<uint64_t>((sg * C::QPART + off) >> 4),
-                          kd + static_cast<uint64_t>((sg * C::KV_SEG + off) >> 4), C::IDESC_S,
-                          kk > 0);
-            }
-          } else {
-            // Q hi, then Q lo, each 4 K steps of 32 dims (32 bytes) along the row
+              for (int kk = 0; kk < NT / 16; ++kk) {
+                const uint32_t col = (kk / 2) * 32 + (kk % 2) * 8;
+                const uint64_t bv = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
+                tc::mma_f16_ts(t_o, t_p + col, bv, C::IDESC_PV, j > 0 || kk > 0);
+                if constexpr (BF) tc::mma_f16_ts(t_o, t_p + col + 16, bv, C::IDESC_PV, true);
+              }
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const int part = kk / 4, off = (kk % 4) * 32;
-              tc::mma_f8(tmem + g * kTmemGroup + (k & 1) * NT,
-                         qd[g] + static_cast<uint64_t>((part * C::QPART + off) >> 4),
-                         kd + static_cast<uint64_t>(off >> 4), C::IDESC_S, kk > 0);
+              for (int kk = 0; kk < NT / 32; ++kk) {  // 32 tokens per k-step
+                const uint32_t col = kk * 32;
+                const uint64_t bv = vd + static_cast<uint64_t>((kk * 32 * 128) >> 4);
+                tc::mma_f8_ts(t_o, t_p + col, bv, C::IDESC_PV, j > 0 || kk > 0);
+                tc::mma_f8_ts(t_o, t_p + col + 8, bv, C::IDESC_PV_LO, true);
+              }
             }
+            tc::commit(&pv_bar[g][j & 1]);
+            np[g] = j + 1;
+            for (const int m = all_issued(np); v_rel < m; ++v_rel) tc::commit(&vempty[v_rel % VR]);
+            progress = true;
           }
-          tc::commit(&s_bar[g][k & 1]);
-        }
-        tc::commit(&kempty[k % KR]);
-        return true;
-      };
-      bool ok = issue_s(0);
-      for (int k = 0; ok && k < nsteps; ++k) {
-        // S of the next step, into the S buffers of step k-1: their softmax read
-        // S and wrote P there, and O += P V of step k-1 read P
-        if (k + 1 < nsteps) {
-          for (int g = 0; ok && g < NG && k >= 1; ++g)
-            ok = mbar_wait(&p_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted) &&
-                 mbar_wait(&pv_bar[g][(k + 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted);
-          ok = ok && issue_s(k + 1);
-        }
-        if (ok) ok = mbar_wait(&vfull[k % VR], (k / VR) & 1, lim, &aborted);
-        if (ok) v_waited = k + 1;
-        // O += P V of each group once its softmax warps wrote P of step k
-        const uint64_t vd = vd0 + static_cast<uint64_t>(((k % VR) * C::KV_BYTES) >> 4);
-        for (int g = 0; ok && g < NG; ++g) {
-          ok = mbar_wait(&p_bar[g][k & 1], (k >> 1) & 1, lim, &aborted);
-          if (!ok) break;
-          tc::fence_after_sync();
-          // P of step k in tensor memory: the S buffer's columns 0-31 (and the
-          // bf16 residual in columns 32-63), 8 columns per 16-token k-step
-          const uint32_t t_p = tmem + g * kTmemGroup + (k & 1) * NT;
-          const uint32_t t_o = tmem + g * kTmemGroup + kTmemO;
-          if constexpr (!FP8) {
+          const int k = ns[g];
+          if (k < nsteps &&
+              (k < SB || mbar_test_wait(&pv_bar[g][(k - SB) & 1], ((k - SB) >> 1) & 1)) &&
+              mbar_test_wait(&kfull[k % KR], (k / KR) & 1)) {
+            tc::fence_after_sync();
+            const uint32_t t_s = t_grp + (SB == 2 ? (k & 1) * NT : 0);
+            const uint64_t kd = kd0 + static_cast<uint64_t>(((k % KR) * C::KV_BYTES) >> 4);
+            if constexpr (!FP8) {
 #pragma unroll
-            for (int kk = 0; kk < NT / 16; ++kk) {
-              const uint64_t bv = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
-              tc::mma_f16_ts(t_o, t_p + kk * 8, bv, C::IDESC_PV, k > 0 || kk > 0);
-              if constexpr (BF) tc::mma_f16_ts(t_o, t_p + 32 + kk * 8, bv, C::IDESC_PV, true);
-            }
-          } else {
-            // E4M3 P in columns 0-15, its E5M2 residual in 16-31; 32 tokens per K step
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const int sg = kk / 4, off = (kk % 4) * 32;
+                tc::mma_f16(t_s, qd[g] + static_cast<uint64_t>((sg * C::QPART + off) >> 4),
+                            kd + static_cast<uint64_t>((sg * C::KV_SEG + off) >> 4), C::IDESC_S,
+                            kk > 0);
+              }
+            } else {
+              // Q hi, then Q lo, each 4 K steps of 32 dims (32 bytes) along the row
 #pragma unroll
-            for (int kk = 0; kk < NT / 32; ++kk) {
-              const uint64_t bv = vd + static_cast<uint64_t>((kk * 32 * 128) >> 4);
-              tc::mma_f8_ts(t_o, t_p + kk * 8, bv, C::IDESC_PV, k > 0 || kk > 0);
-              tc::mma_f8_ts(t_o, t_p + 16 + kk * 8, bv, C::IDESC_PV_LO, true);
+              for (int kk = 0; kk < 8; ++kk) {
+                const int part = kk / 4, off = (kk % 4) * 32;
+                tc::mma_f8(t_s, qd[g] + static_cast<uint64_t>((part * C::QPART + off) >> 4),
+                           kd + static_cast<uint64_t>(off >> 4), C::IDESC_S, kk > 0);
+              }
             }
+            tc::commit(&s_bar[g][k & 1]);
+            ns[g] = k + 1;
+            for (const int m = all_issued(ns); k_rel < m; ++k_rel) tc::commit(&kempty[k_rel % KR]);
+            progress = true;
           }
-          tc::commit(&pv_bar[g][k & 1]);
         }
-        if (ok) tc::commit(&vempty[k % VR]);
+        if (progress) {
+          t_last = global_timer_ns();
+        } else if (aborted || global_timer_ns() - t_last > lim) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) {
         // A wait gave up (never expected): let this CTA's MMAs finish (bounded)
         // before its tensor and shared memory go away.
-        record_failure(a.diag, kSiteTcStep, blockIdx.x, blockIdx.y, blockIdx.z, k_waited, v_waited,
+        record_failure(a.diag, kSiteTcStep, blockIdx.x, blockIdx.y, blockIdx.z, k_rel, v_rel,
                        nsteps, NG);
         aborted = 1;
         report(a.err, kErrWaitTimeout);
@@ -431,40 +463,106 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
       ok = mbar_wait(&s_bar[g][k & 1], (k >> 1) & 1, lim, &aborted);
       if (!ok) break;
       tc::fence_after_sync();
-      float x[NT];
-      tc::ld64(t_grp + (k & 1) * NT + lane_base, x);
+      const uint32_t t_s = t_grp + (SB == 2 ? (k & 1) * NT : 0) + lane_base;
       const int tk0 = (kbase + k) * NT;
-      // causal mask only where the step reaches past this row's position
-      if (tk0 + NT - 1 > p_row) {
+      // this row's logits of 64-token half h, masked after the row's position
+      // (the causal rule) only where the half reaches past it
+      float x[64];
+      auto load_half = [&](int h) {
+        tc::ld64(t_s + h * 64, x);
+        const int t0 = tk0 + h * 64;
+        if (t0 + 63 > p_row) {
 #pragma unroll
-        for (int i = 0; i < NT; ++i) x[i] = tk0 + i <= p_row ? x[i] : -CUDART_INF_F;
+          for (int i = 0; i < 64; ++i) x[i] = t0 + i <= p_row ? x[i] : -CUDART_INF_F;
+        }
+      };
+      // maximum of 64 raw logits (the scale is positive): 8 partial chains
+      auto half_max = [&]() {
+        float m8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m8[j] = x[j];
+#pragma unroll
+        for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+        return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      };
+      // the row maximum of the step: with two halves the upper one is read
+      // first for its maximum alone and read again after the lower one
+      float mraw = -CUDART_INF_F;
+      if constexpr (H == 2) {
+        load_half(1);
+        mraw = half_max();
       }
-      // row maximum of the raw logits (the scale is positive): 8 partial chains
-      float m8[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) m8[j] = x[j];
-#pragma unroll
-      for (int i = 8; i < NT; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * qscale;
+      load_half(0);
+      mraw = fmaxf(mraw, half_max());
+      const float mx = mraw * qscale;
       const bool rescale = mx > m_used + 8.f;   // false while the row sees nothing
       const float alpha = rescale ? tc::ex2(m_used - mx) : 1.f;
       if (rescale) m_used = mx;
       const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
-      // p = 2^(s * scale - m), summed in 8 partial chains
-      float s8[8] = {};
+      // P -> tensor memory over the S it came from, 32 probabilities at a time:
+      // quarter qq of the step (tokens 32 qq ..) goes to its own 32 S columns,
+      // from column 32 qq: 16-bit pairs (16 columns; for bf16 the residual
+      // P - bf16(P) in the next 16), or E4M3 codes (8 columns, the E5M2
+      // residual in the next 8). A quarter's writes touch no S column still
+      // to be read, so the upper half is read again a quarter at a time and
+      // fewer registers are live.
+      float lsum = 0.f;
+      auto emit32 = [&](float* v, int h, int q) {
+        float s8[8] = {};  // p = 2^(s * scale - m), summed in 8 partial chains
 #pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        x[i] = tc::ex2(fmaf(x[i], qscale, -mu));
-        s8[i & 7] += x[i];
+        for (int i = 0; i < 32; ++i) {
+          v[i] = tc::ex2(fmaf(v[i], qscale, -mu));
+          s8[i & 7] += v[i];
+        }
+        lsum += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+        const uint32_t t_p = t_s + 32 * (2 * h + q);
+        if constexpr (FP8) {
+          uint32_t w[8], wl[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            tc::split_fp8x4<true>(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3], w[i], wl[i]);
+          tc::st8u(t_p, w);
+          tc::st8u(t_p + 8, wl);
+        } else {
+          uint32_t w[16], wl[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            w[i] = pack_pair(BF, v[2 * i], v[2 * i + 1]);
+            if constexpr (BF)
+              wl[i] = pack2<true>(v[2 * i] - __uint_as_float(w[i] << 16),
+                                  v[2 * i + 1] - __uint_as_float(w[i] & 0xffff0000u));
+          }
+          tc::st16u(t_p, w);
+          if constexpr (BF) tc::st16u(t_p + 16, wl);
+        }
+      };
+      emit32(x, 0, 0);
+      emit32(x + 32, 0, 1);
+      if constexpr (H == 2) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          float y[32];
+          tc::ld32(t_s + 64 + 32 * q, y);
+          const int t0 = tk0 + 64 + 32 * q;
+          if (t0 + 31 > p_row) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) y[i] = t0 + i <= p_row ? y[i] : -CUDART_INF_F;
+          }
+          emit32(y, 1, q);
+        }
       }
-      l = l * alpha + (((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7])));
-      // O may be rescaled only once O += P V of step k-1 completed (rare: the
-      // maximum moves lazily), otherwise that MMA keeps running under this softmax
+      l = l * alpha + lsum;
+      // O is rescaled (rare: the maximum moves lazily) after P is written, when
+      // fewer registers are live, and before P is posted; only once O += P V
+      // of step k-1 completed. With one S buffer it has: S of this step was
+      // issued after it.
       if (k >= 1 && rescale) {
-        ok = mbar_wait(&pv_bar[g][(k - 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted);
-        if (!ok) break;
-        tc::fence_after_sync();
+        if constexpr (SB == 2) {
+          ok = mbar_wait(&pv_bar[g][(k - 1) & 1], ((k - 1) >> 1) & 1, lim, &aborted);
+          if (!ok) break;
+          tc::fence_after_sync();
+        }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
@@ -474,37 +572,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
           tc::st32(t_o + c * 32, o);
         }
       }
-      // P row (and for bf16 the residual P - bf16(P)) -> tensor memory, over the
-      // S it came from: columns 0-31 (pairs of 16-bit values), residual 32-63
-      if constexpr (FP8) {
-        uint32_t w[NT / 4], wl[NT / 4];
-#pragma unroll
-        for (int i = 0; i < NT / 4; ++i)
-          tc::split_fp8x4<true>(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3], w[i], wl[i]);
-        const uint32_t t_p = t_grp + (k & 1) * NT + lane_base;
-        tc::st16u(t_p, w);
-        tc::st16u(t_p + 16, wl);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      } else {
-        // in two halves of 32 probabilities (16 columns each), so that fewer
-        // registers are live at once
-        const uint32_t t_p = t_grp + (k & 1) * NT + lane_base;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t w[NT / 4], wl[NT / 4];
-#pragma unroll
-          for (int i = 0; i < NT / 4; ++i) {
-            const float p0 = x[h * NT / 2 + 2 * i], p1 = x[h * NT / 2 + 2 * i + 1];
-            w[i] = pack_pair(BF, p0, p1);
-            if constexpr (BF)
-              wl[i] = pack2<true>(p0 - __uint_as_float(w[i] << 16),
-                                  p1 - __uint_as_float(w[i] & 0xffff0000u));
-          }
-          tc::st16u(t_p + h * NT / 4, w);
-          if constexpr (BF) tc::st16u(t_p + NT / 2 + h * NT / 4, wl);
-        }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       // V rows without real data in this step (past the context, or tiles not
       // loaded) may hold anything, even NaN, and 0 * NaN is NaN inside the MMA;
       // every group's warps clear them (the same zeros) before their P is posted
@@ -596,6 +664,7 @@ cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUten
   cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   if (a.q_tiles != (max_query_len + C::QT - 1) / C::QT) return cudaErrorInvalidValue;
+  if (a.max_parts > 1 && a.partition_tiles % (C::NT / kTileRows) != 0) return cudaErrorInvalidValue;
   e = launch_pdl(kern, dim3(static_cast<unsigned>(a.q_tiles * a.max_parts), a.num_kv_heads,
                             a.num_seqs),
                  NG * kTcRows + 96, smem, stream, a, kmap, vmap);
