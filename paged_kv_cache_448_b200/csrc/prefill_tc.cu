@@ -100,6 +100,32 @@ struct TcCfg {
   static_assert(BYTES + 1024 <= 227 * 1024, "shared memory of one CTA");
 };
 
+// 32 consecutive fp32 columns of this thread's lane into v[0..31], without
+// waiting (tcgen05.wait::ld follows, then tie16 on the registers).
+__device__ __forceinline__ void ld32f_nowait(uint32_t taddr, float* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31}, [%32];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+        "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]),
+        "=f"(v[14]), "=f"(v[15]), "=f"(v[16]), "=f"(v[17]), "=f"(v[18]), "=f"(v[19]),
+        "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]), "=f"(v[24]), "=f"(v[25]),
+        "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// An empty statement that takes and gives back 16 registers: placed after a
+// wait for tensor-memory loads, it keeps every use of the loaded values after
+// the wait.
+__device__ __forceinline__ void tie16(float* v) {
+  asm volatile(""
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                 "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]),
+                 "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]));
+}
+
 // 16-byte chunk `c` of row `r` of a 128-byte-swizzled [rows][128 B] tile.
 __device__ __forceinline__ uint32_t sw128(int r, int c) {
   return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
@@ -469,11 +495,18 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
       tc::fence_after_sync();
       const uint32_t t_s = t_grp + (SB == 2 ? (k & 1) * NT : 0) + lane_base;
       const int tk0 = (kbase + k) * NT;
+      // With an f16 cache and two groups the row's 128 logits are held at once
+      // (read in one go: the loads issued together, one wait); otherwise 64
+      // at a time (measured on B200, chunked prefill: 685-703 against 653 TFLOP/s
+      // for f16, but 550 against 573 for bf16 and 665 against 702 for E4M3,
+      // whose softmax needs more registers)
+      constexpr bool kHoldAll = NG == 2 && !BF && !FP8;
+      float x[kHoldAll ? 128 : 64];
+      float mraw = -CUDART_INF_F;
       // this row's logits of 64-token half h, masked after the row's position
       // (the causal rule) only where the half reaches past it
-      float x[64];
       auto load_half = [&](int h) {
-        tc::ld64(t_s + h * 64, x);
+        tc::ld64(t_s + h * 64, *reinterpret_cast<float(*)[64]>(x));
         const int t0 = tk0 + h * 64;
         if (t0 + 63 > p_row) {
 #pragma unroll
@@ -490,15 +523,41 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
         return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                      fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       };
-      // the row maximum of the step: with two halves the upper one is read
-      // first for its maximum alone and read again after the lower one
-      float mraw = -CUDART_INF_F;
-      if constexpr (H == 2) {
-        load_half(1);
-        mraw = half_max();
+      if constexpr (kHoldAll) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ld32f_nowait(t_s + 32 * q, x + 32 * q);
+        tc::wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tie16(x + 32 * q), tie16(x + 32 * q + 16);
+        // masked after the row's position (the causal rule) only where a
+        // 32-token quarter reaches past it
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t0 = tk0 + 32 * q;
+          if (t0 + 31 > p_row) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              x[32 * q + i] = t0 + i <= p_row ? x[32 * q + i] : -CUDART_INF_F;
+          }
+        }
+        // row maximum of the raw logits (the scale is positive): 8 partial chains
+        float m8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m8[j] = x[j];
+#pragma unroll
+        for (int i = 8; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+        mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      } else {
+        // the row maximum of the step: with two halves the upper one is read
+        // first for its maximum alone and read again after the lower one
+        if constexpr (H == 2) {
+          load_half(1);
+          mraw = half_max();
+        }
+        load_half(0);
+        mraw = fmaxf(mraw, half_max());
       }
-      load_half(0);
-      mraw = fmaxf(mraw, half_max());
       const float mx = mraw * qscale;
       const bool rescale = mx > m_used + 8.f;   // false while the row sees nothing
       const float alpha = rescale ? tc::ex2(m_used - mx) : 1.f;
@@ -540,9 +599,14 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
           if constexpr (BF) tc::st16u(t_p + 16, wl);
         }
       };
-      emit32(x, 0, 0);
-      emit32(x + 32, 0, 1);
-      if constexpr (H == 2) {
+      if constexpr (kHoldAll) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) emit32(x + 32 * q, q / 2, q % 2);
+      } else {
+        emit32(x, 0, 0);
+        emit32(x + 32, 0, 1);
+      }
+      if constexpr (H == 2 && !kHoldAll) {
         // the upper half again: in one read for a bf16 cache, a quarter at a
         // time otherwise (measured on B200: 583 against 540 TFLOP/s for bf16,
         // 636 against 652 for f16 and 670 against 701 for E4M3 chunks)
