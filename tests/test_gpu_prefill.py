@@ -139,6 +139,8 @@ def test_short_chunks_of_many_sequences_on_tcgen05(cache, G, q):
 
 @pytest.mark.parametrize("qdt,cache,G,D,bs,qlens", [
     ("bf16", "bf16", 8, 128, 16, [150, 129, 140]),   # two row groups (>= 256 rows)
+    ("f16", "f16", 2, 128, 16, [200, 150, 131]),     # two groups, f16: rows held whole
+    ("bf16", "e4m3", 8, 128, 32, [100, 70, 65]),     # two groups over an E4M3 cache
     ("f16", "f16", 1, 128, 32, [200, 129, 160]),     # one row group
     ("bf16", "e4m3", 4, 128, 16, [64, 40, 33]),
     ("f16", "f16", 2, 64, 32, [100, 70, 65]),
