@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 3 : 2)
       uint32_t r[NL];
       if constexpr (NL == 8) tc::ld8_nowait(tmem + (k & 1) * kN + lane_base, r);
       else tc::ld16_nowait(tmem + (k & 1) * kN + lane_base, r);
-      tc::wait_ld();
+      tc::wait_ld(r);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[k & 1]);
@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 3 : 2)
         uint32_t o[NL];
         if constexpr (NL == 8) tc::ld8_nowait(tmem + kColO + lane_base, o);
         else tc::ld16_nowait(tmem + kColO + lane_base, o);
-        tc::wait_ld();
+        tc::wait_ld(o);
 #pragma unroll
         for (int g = 0; g < G; ++g) o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
         if constexpr (NL == 8) tc::st8u(tmem + kColO + lane_base, o);
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 3 : 2)
       tc::fence_after_sync();
       if constexpr (NL == 8) tc::ld8_nowait(tmem + kColO + lane_base, o);
       else tc::ld16_nowait(tmem + kColO + lane_base, o);
-      tc::wait_ld();
+      tc::wait_ld(o);
     }
     const bool single = parts == 1;
     const int64_t row0 = static_cast<int64_t>(s) * a.num_heads + kvh * G;
