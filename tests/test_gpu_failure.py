@@ -46,7 +46,7 @@ def _decode_step(G, cache, seed):
 
 
 @pytest.mark.parametrize("cache", ["bf16", "e4m3"])
-@pytest.mark.parametrize("G,part", [(1, 0), (2, 128), (4, 256), (8, 0)])
+@pytest.mark.parametrize("G,part", [(1, 0), (2, 128), (4, 256), (8, 0), (2, 64)])
 def test_decode_wait_that_runs_out(G, part, cache):
     g = _decode_step(G, cache, seed=50 + G)
     g.reshape()
