@@ -368,102 +368,138 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
       for (int g = 0; g < NG; ++g) qd[g] = tc::sw128_desc(sq(g), 16, 1024);
       const uint64_t kd0 = tc::sw128_desc(sk(0), 16, 1024);
       const uint64_t vd0 = tc::sw128_desc(sv(0), NT * 128, 1024);
-      // Per group: ns[g] = next step whose S is issued, np[g] = next step
-      // whose O += P V is issued. The thread polls and issues whatever is
-      // ready, so neither group waits behind the other:
-      //  * S(g, k): K of step k landed and the group's S buffer is free, i.e.
-      //    O += P V of step k - SB (which read the P written over that S)
-      //    completed;
-      //  * O += P V (g, k): S(g, k) issued, the group posted P of step k and
-      //    V of step k landed.
-      // A K stage is released once every group's S of its step was issued, a
-      // V stage once every group's O += P V (a commit completes when all of
-      // the thread's earlier MMAs have). Gives up after the wait limit
-      // without progress.
-      int ns[NG], np[NG];
+      // S = Q K^T of step k for group g (K landed, the S buffer free)
+      auto issue_s = [&](int g, int k) {
+        const uint32_t t_s = tmem + g * kTmemGroup + (SB == 2 ? (k & 1) * NT : 0);
+        const uint64_t kd = kd0 + static_cast<uint64_t>(((k % KR) * C::KV_BYTES) >> 4);
+        if constexpr (!FP8) {
 #pragma unroll
-      for (int g = 0; g < NG; ++g) ns[g] = np[g] = 0;
-      int k_rel = 0, v_rel = 0;  // K / V stages released so far (steps)
-      bool ok = true;
-      uint64_t t_last = global_timer_ns();
-      auto all_issued = [&](const int (&c)[NG]) {
-        int m = c[0];
-#pragma unroll
-        for (int g = 1; g < NG; ++g) m = min(m, c[g]);
-        return m;
-      };
-      while (all_issued(np) < nsteps) {
-        bool progress = false;
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-          const uint32_t t_grp = tmem + g * kTmemGroup;
-          const int j = np[g];
-          if (j < ns[g] && mbar_test_wait(&p_bar[g][j & 1], (j >> 1) & 1) &&
-              mbar_test_wait(&vfull[j % VR], (j / VR) & 1)) {
-            tc::fence_after_sync();
-            // P of step j over its S: per 32 tokens (quarter qq) the 16-bit
-            // pairs (or E4M3 codes) from column 32 qq, the bf16 (or E5M2)
-            // residual 16 (8) columns further; 8 columns per k-step
-            const uint32_t t_p = t_grp + (SB == 2 ? (j & 1) * NT : 0);
-            const uint32_t t_o = t_grp + kTmemO;
-            const uint64_t vd = vd0 + static_cast<uint64_t>(((j % VR) * C::KV_BYTES) >> 4);
-            if constexpr (!FP8) {
-#pragma unroll
-              for (int kk = 0; kk < NT / 16; ++kk) {
-                const uint32_t col = (kk / 2) * 32 + (kk % 2) * 8;
-                const uint64_t bv = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
-                tc::mma_f16_ts(t_o, t_p + col, bv, C::IDESC_PV, j > 0 || kk > 0);
-                if constexpr (BF) tc::mma_f16_ts(t_o, t_p + col + 16, bv, C::IDESC_PV, true);
-              }
-            } else {
-#pragma unroll
-              for (int kk = 0; kk < NT / 32; ++kk) {  // 32 tokens per k-step
-                const uint32_t col = kk * 32;
-                const uint64_t bv = vd + static_cast<uint64_t>((kk * 32 * 128) >> 4);
-                tc::mma_f8_ts(t_o, t_p + col, bv, C::IDESC_PV, j > 0 || kk > 0);
-                tc::mma_f8_ts(t_o, t_p + col + 8, bv, C::IDESC_PV_LO, true);
-              }
-            }
-            tc::commit(&pv_bar[g][j & 1]);
-            np[g] = j + 1;
-            for (const int m = all_issued(np); v_rel < m; ++v_rel) tc::commit(&vempty[v_rel % VR]);
-            progress = true;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int sg = kk / 4, off = (kk % 4) * 32;
+            tc::mma_f16(t_s, qd[g] + static_cast<uint64_t>((sg * C::QPART + off) >> 4),
+                        kd + static_cast<uint64_t>((sg * C::KV_SEG + off) >> 4), C::IDESC_S,
+                        kk > 0);
           }
-          const int k = ns[g];
-          if (k < nsteps &&
-              (k < SB || mbar_test_wait(&pv_bar[g][(k - SB) & 1], ((k - SB) >> 1) & 1)) &&
-              mbar_test_wait(&kfull[k % KR], (k / KR) & 1)) {
-            tc::fence_after_sync();
-            const uint32_t t_s = t_grp + (SB == 2 ? (k & 1) * NT : 0);
-            const uint64_t kd = kd0 + static_cast<uint64_t>(((k % KR) * C::KV_BYTES) >> 4);
-            if constexpr (!FP8) {
+        } else {
+          // Q hi, then Q lo, each 4 K steps of 32 dims (32 bytes) along the row
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const int sg = kk / 4, off = (kk % 4) * 32;
-                tc::mma_f16(t_s, qd[g] + static_cast<uint64_t>((sg * C::QPART + off) >> 4),
-                            kd + static_cast<uint64_t>((sg * C::KV_SEG + off) >> 4), C::IDESC_S,
-                            kk > 0);
-              }
-            } else {
-              // Q hi, then Q lo, each 4 K steps of 32 dims (32 bytes) along the row
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const int part = kk / 4, off = (kk % 4) * 32;
-                tc::mma_f8(t_s, qd[g] + static_cast<uint64_t>((part * C::QPART + off) >> 4),
-                           kd + static_cast<uint64_t>(off >> 4), C::IDESC_S, kk > 0);
-              }
-            }
-            tc::commit(&s_bar[g][k & 1]);
-            ns[g] = k + 1;
-            for (const int m = all_issued(ns); k_rel < m; ++k_rel) tc::commit(&kempty[k_rel % KR]);
-            progress = true;
+          for (int kk = 0; kk < 8; ++kk) {
+            const int part = kk / 4, off = (kk % 4) * 32;
+            tc::mma_f8(t_s, qd[g] + static_cast<uint64_t>((part * C::QPART + off) >> 4),
+                       kd + static_cast<uint64_t>(off >> 4), C::IDESC_S, kk > 0);
           }
         }
-        if (progress) {
-          t_last = global_timer_ns();
-        } else if (aborted || global_timer_ns() - t_last > lim) {
-          ok = false;
-          break;
+        tc::commit(&s_bar[g][k & 1]);
+      };
+      // O += P V of step j for group g (P posted, V landed). P of step j lies
+      // over its S: per 32 tokens (quarter qq) the 16-bit pairs (or E4M3
+      // codes) from column 32 qq, the bf16 (or E5M2) residual 16 (8) columns
+      // further; 8 columns per k-step
+      auto issue_pv = [&](int g, int j) {
+        const uint32_t t_grp = tmem + g * kTmemGroup;
+        const uint32_t t_p = t_grp + (SB == 2 ? (j & 1) * NT : 0);
+        const uint32_t t_o = t_grp + kTmemO;
+        const uint64_t vd = vd0 + static_cast<uint64_t>(((j % VR) * C::KV_BYTES) >> 4);
+        if constexpr (!FP8) {
+#pragma unroll
+          for (int kk = 0; kk < NT / 16; ++kk) {
+            const uint32_t col = (kk / 2) * 32 + (kk % 2) * 8;
+            const uint64_t bv = vd + static_cast<uint64_t>((kk * 16 * 128) >> 4);
+            tc::mma_f16_ts(t_o, t_p + col, bv, C::IDESC_PV, j > 0 || kk > 0);
+            if constexpr (BF) tc::mma_f16_ts(t_o, t_p + col + 16, bv, C::IDESC_PV, true);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < NT / 32; ++kk) {  // 32 tokens per k-step
+            const uint32_t col = kk * 32;
+            const uint64_t bv = vd + static_cast<uint64_t>((kk * 32 * 128) >> 4);
+            tc::mma_f8_ts(t_o, t_p + col, bv, C::IDESC_PV, j > 0 || kk > 0);
+            tc::mma_f8_ts(t_o, t_p + col + 8, bv, C::IDESC_PV_LO, true);
+          }
+        }
+        tc::commit(&pv_bar[g][j & 1]);
+      };
+      // A K stage is released once every group's S of its step was issued, a
+      // V stage once every group's O += P V (a commit completes when all of
+      // the thread's earlier MMAs have).
+      int k_rel = 0, v_rel = 0;  // K / V stages released so far (steps)
+      bool ok = true;
+      if constexpr (NG == 2) {
+        // Two groups, one S buffer each: a group's chain is softmax, O += P V,
+        // its next S (once O += P V, which read P over S, completed). The
+        // MMAs go in a fixed order per step: O += P V of group 0, its next S,
+        // then the same for group 1, so that the groups' tensor work
+        // alternates and a group's next S follows its O += P V at once. (Issued
+        // greedily, whatever was ready first, the groups drifted into each
+        // other: a group's O += P V queued behind the other's work.)
+        ok = mbar_wait(&kfull[0], 0, lim, &aborted);
+        if (ok) {
+          tc::fence_after_sync();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          tc::commit(&kempty[0]);
+          k_rel = 1;
+        }
+        for (int k = 0; ok && k < nsteps; ++k) {
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+            ok = (g > 0 || mbar_wait(&vfull[k % VR], (k / VR) & 1, lim, &aborted)) &&
+                 mbar_wait(&p_bar[g][k & 1], (k >> 1) & 1, lim, &aborted);
+            if (!ok) break;
+            tc::fence_after_sync();
+            issue_pv(g, k);
+            if (g == NG - 1) {
+              tc::commit(&vempty[k % VR]);
+              v_rel = k + 1;
+            }
+            if (k + 1 < nsteps) {
+              ok = mbar_wait(&pv_bar[g][k & 1], (k >> 1) & 1, lim, &aborted) &&
+                   mbar_wait(&kfull[(k + 1) % KR], ((k + 1) / KR) & 1, lim, &aborted);
+              if (!ok) break;
+              tc::fence_after_sync();
+              issue_s(g, k + 1);
+              if (g == NG - 1) {
+                tc::commit(&kempty[(k + 1) % KR]);
+                k_rel = k + 2;
+              }
+            }
+          }
+        }
+      } else {
+        // One group, two S buffers: the thread polls and issues whatever is
+        // ready. ns = next step whose S is issued, np = next step whose
+        // O += P V is issued:
+        //  * S(k): K of step k landed and the S buffer is free, i.e. O += P V
+        //    of step k - 2 (which read the P written over that S) completed;
+        //  * O += P V (k): S(k) issued, P of step k posted, V landed.
+        // Gives up after the wait limit without progress.
+        int ns = 0, np = 0;
+        uint64_t t_last = global_timer_ns();
+        while (np < nsteps) {
+          bool progress = false;
+          if (np < ns && mbar_test_wait(&p_bar[0][np & 1], (np >> 1) & 1) &&
+              mbar_test_wait(&vfull[np % VR], (np / VR) & 1)) {
+            tc::fence_after_sync();
+            issue_pv(0, np);
+            tc::commit(&vempty[np % VR]);
+            v_rel = ++np;
+            progress = true;
+          }
+          if (ns < nsteps &&
+              (ns < SB || mbar_test_wait(&pv_bar[0][(ns - SB) & 1], ((ns - SB) >> 1) & 1)) &&
+              mbar_test_wait(&kfull[ns % KR], (ns / KR) & 1)) {
+            tc::fence_after_sync();
+            issue_s(0, ns);
+            tc::commit(&kempty[ns % KR]);
+            k_rel = ++ns;
+            progress = true;
+          }
+          if (progress) {
+            t_last = global_timer_ns();
+          } else if (aborted || global_timer_ns() - t_last > lim) {
+            ok = false;
+            break;
+          }
         }
       }
       if (!ok) {
