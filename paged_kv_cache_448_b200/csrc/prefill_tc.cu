@@ -531,12 +531,12 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
       tc::fence_after_sync();
       const uint32_t t_s = t_grp + (SB == 2 ? (k & 1) * NT : 0) + lane_base;
       const int tk0 = (kbase + k) * NT;
-      // With an f16 cache and two groups the row's 128 logits are held at once
-      // (read in one go: the loads issued together, one wait); otherwise 64
-      // at a time (measured on B200, chunked prefill: 685-703 against 653 TFLOP/s
-      // for f16, but 550 against 573 for bf16 and 665 against 702 for E4M3,
-      // whose softmax needs more registers)
-      constexpr bool kHoldAll = NG == 2 && !BF && !FP8;
+      // With a 16-bit cache and two groups the row's 128 logits are held at
+      // once (read in one go: the loads issued together, one wait); with one
+      // group, or an E4M3 cache, 64 at a time (measured on B200 with the
+      // fixed MMA order, chunked prefill: bf16 687 against 657 TFLOP/s held
+      // and not; E4M3 733 against 781, its softmax needing more registers)
+      constexpr bool kHoldAll = NG == 2 && !FP8;
       float x[kHoldAll ? 128 : 64];
       float mraw = -CUDART_INF_F;
       // this row's logits of 64-token half h, masked after the row's position
@@ -643,25 +643,18 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
         emit32(x + 32, 0, 1);
       }
       if constexpr (H == 2 && !kHoldAll) {
-        // the upper half again: in one read for a bf16 cache, a quarter at a
-        // time otherwise (measured on B200: 583 against 540 TFLOP/s for bf16,
-        // 636 against 652 for f16 and 670 against 701 for E4M3 chunks)
-        if constexpr (BF && !FP8) {
-          load_half(1);
-          emit32(x, 1, 0);
-          emit32(x + 32, 1, 1);
-        } else {
+        // the upper half again (E4M3 cache), a quarter at a time (measured on
+        // B200: 701 against 670 TFLOP/s for the whole half in one read)
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            float y[32];
-            tc::ld32(t_s + 64 + 32 * q, y);
-            const int t0 = tk0 + 64 + 32 * q;
-            if (t0 + 31 > p_row) {
+        for (int q = 0; q < 2; ++q) {
+          float y[32];
+          tc::ld32(t_s + 64 + 32 * q, y);
+          const int t0 = tk0 + 64 + 32 * q;
+          if (t0 + 31 > p_row) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) y[i] = t0 + i <= p_row ? y[i] : -CUDART_INF_F;
-            }
-            emit32(y, 1, q);
+            for (int i = 0; i < 32; ++i) y[i] = t0 + i <= p_row ? y[i] : -CUDART_INF_F;
           }
+          emit32(y, 1, q);
         }
       }
       l = l * alpha + lsum;
