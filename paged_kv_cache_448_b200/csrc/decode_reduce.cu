@@ -36,15 +36,29 @@ __global__ void __launch_bounds__(128) paged_decode_reduce(const DecodeArgs a) {
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
   float L = 0.f;
   const float* o = a.ws_o + row * a.max_parts * D;
-  for (int p = 0; p < parts; ++p) {
-    const float2 v = ml[p];
-    // a partition that saw no token (or gave up) has no weight, and its o
-    // was never written: it is not read
-    if (v.x == -CUDART_INF_F || !(v.y > 0.f)) continue;
-    const float w = v.y * exp2f(v.x - M);
-    L += w;
+  // kBatch partitions at a time, all their loads issued before any is used
+  // (one L2 round trip per batch, not per partition). A partition that saw
+  // no token (or gave up) has no weight, and its o was never written: its
+  // values, whatever they are, are selected away, never multiplied.
+  constexpr int kBatch = 8;
+  for (int p0 = 0; p0 < parts; p0 += kBatch) {
+    float2 v[kBatch];
+    float ov[kBatch][PER];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, o[p * D + lane + 32 * i], acc[i]);
+    for (int u = 0; u < kBatch; ++u) {
+      const int p = min(p0 + u, parts - 1);
+      v[u] = ml[p];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) ov[u][i] = o[p * D + lane + 32 * i];
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const bool use = p0 + u < parts && v[u].x != -CUDART_INF_F && v[u].y > 0.f;
+      const float w = use ? v[u].y * exp2f(v[u].x - M) : 0.f;
+      L += w;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] = use ? fmaf(w, ov[u][i], acc[i]) : acc[i];
+    }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
