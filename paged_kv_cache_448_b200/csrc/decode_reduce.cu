@@ -26,21 +26,18 @@ __global__ void __launch_bounds__(128) paged_decode_reduce(const DecodeArgs a) {
   if (parts <= 1) return;  // written directly by the decode kernel
   const int64_t row = static_cast<int64_t>(s) * a.num_heads + h;
   const float2* ml = a.ws_ml + row * a.max_parts;
-  float M = -CUDART_INF_F;
-  for (int p = lane; p < parts; p += 32) M = fmaxf(M, ml[p].x);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   constexpr int PER = D / 32;
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  float L = 0.f;
+  float M = -CUDART_INF_F, L = 0.f;
   const float* o = a.ws_o + row * a.max_parts * D;
   // kBatch partitions at a time, all their loads issued before any is used
-  // (one L2 round trip per batch, not per partition). A partition that saw
+  // (one L2 round trip per batch, not per partition), with a running maximum
+  // (the sums so far rescaled when a batch raises it). A partition that saw
   // no token (or gave up) has no weight, and its o was never written: its
   // values, whatever they are, are selected away, never multiplied.
-  constexpr int kBatch = 8;
+  constexpr int kBatch = 16;
   for (int p0 = 0; p0 < parts; p0 += kBatch) {
     float2 v[kBatch];
     float ov[kBatch][PER];
@@ -51,13 +48,26 @@ __global__ void __launch_bounds__(128) paged_decode_reduce(const DecodeArgs a) {
 #pragma unroll
       for (int i = 0; i < PER; ++i) ov[u][i] = o[p * D + lane + 32 * i];
     }
+    bool use[kBatch];
+    float bm = M;
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const bool use = p0 + u < parts && v[u].x != -CUDART_INF_F && v[u].y > 0.f;
-      const float w = use ? v[u].y * exp2f(v[u].x - M) : 0.f;
+      use[u] = p0 + u < parts && v[u].x != -CUDART_INF_F && v[u].y > 0.f;
+      if (use[u]) bm = fmaxf(bm, v[u].x);
+    }
+    if (bm > M) {  // the same in every lane (the loads are broadcasts)
+      const float f = M == -CUDART_INF_F ? 0.f : exp2f(M - bm);
+      L *= f;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] *= f;
+      M = bm;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const float w = use[u] ? v[u].y * exp2f(v[u].x - M) : 0.f;
       L += w;
 #pragma unroll
-      for (int i = 0; i < PER; ++i) acc[i] = use ? fmaf(w, ov[u][i], acc[i]) : acc[i];
+      for (int i = 0; i < PER; ++i) acc[i] = use[u] ? fmaf(w, ov[u][i], acc[i]) : acc[i];
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
