@@ -612,7 +612,9 @@ def decode_line(args, sp: wl.Spec, st: wl.Structure, world: int, step_ms: float,
                    "l2": f"inputs larger than L2: {wl.kv_bytes(sp) / 1e9:.2f} GB of K/V "
                          "per step vs 126 MB L2; no flush"},
         "pct_of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2),
-        "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+        # against the copy bandwidth measured on this machine, or the fallback
+        # figure when no measurement is present (peak_kind says which)
+        "pct_of_copy_peak": round(100 * value / world / peak, 2),
         "tokens_per_s_per_layer": round(world * sp.num_seqs / (step_ms * 1e-3), 1),
         "roofline": {"bound": "hbm", "kernel": "pa_decode (decode" +
                      (" + partition combine)" if split else ")"),

@@ -43,10 +43,15 @@ __global__ void __launch_bounds__(128) paged_decode_reduce(const DecodeArgs a) {
     float ov[kBatch][PER];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const int p = min(p0 + u, parts - 1);
-      v[u] = ml[p];
+      const int p = p0 + u;
+      v[u] = make_float2(-CUDART_INF_F, 0.f);
 #pragma unroll
-      for (int i = 0; i < PER; ++i) ov[u][i] = o[p * D + lane + 32 * i];
+      for (int i = 0; i < PER; ++i) ov[u][i] = 0.f;
+      if (p < parts) {  // the same in every lane
+        v[u] = ml[p];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) ov[u][i] = o[p * D + lane + 32 * i];
+      }
     }
     bool use[kBatch];
     float bm = M;
