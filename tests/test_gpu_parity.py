@@ -322,3 +322,36 @@ def test_full_size_workload_sampled(cfg):
     ref = oracle.decode(q_h, kc_h, vc_h, ctable, lens[seqs], scale=np.float32(sp.scale),
                         q_dtype=sp.q_dtype, cache_dtype=sp.cache_dtype, k_scale=ks, v_scale=vs)
     assert_close(gpu, ref, sp.cache_dtype, f"full cfg{cfg} seqs {seqs}")
+
+
+def _as_f32(codes: np.ndarray, dt: str) -> np.ndarray:
+    if dt == "f16":
+        return codes.view(np.float16).astype(np.float32)
+    return (codes.astype(np.uint32) << 16).view(np.float32)
+
+
+@pytest.mark.parametrize("qdt,G", [("f16", 1), ("bf16", 8)])
+def test_combine_running_maximum_across_batches(qdt, G):
+    """Many partitions per sequence (47 of 32 tokens), combined 16 at a time
+    with a running maximum: one sequence's largest logit sits in its last
+    batch of partitions (the sums so far are rescaled when it arrives), the
+    other's in its first."""
+    Hkv, D, bs = 2, 128, 16
+    sp, st, hd = custom([1500, 1500, 700], Hkv * G, Hkv, D, bs, qdt, qdt, seed=4242 + G)
+    q = _as_f32(hd.query, qdt)
+    kc = hd.key_cache
+    for s, t in ((0, 1490), (1, 5)):
+        blk = st.block_tables[s][t // bs]
+        for kvh in range(Hkv):
+            # the key of token t is the group's first query head: that head's
+            # logit there (about |q|^2 / sqrt(D) ~ 11) outweighs the rest by
+            # ~2^16, so partitions combined before it must be rescaled
+            row = q[s, kvh * G]
+            kc[blk, t % bs, kvh] = wl._f32_to_codes(row.astype(np.float32), qdt)
+    _, _, ref = oracle_step(sp, st, hd)
+    g = GpuStep(sp, st, hd)
+    g.reshape()
+    g.out.fill_(float("nan"))
+    g.decode(partition_tokens=2 * bs)
+    torch.cuda.synchronize()
+    assert_close(g.out_f64(), ref, qdt, f"{qdt} G{G} 47 partitions")
