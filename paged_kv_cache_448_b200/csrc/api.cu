@@ -308,7 +308,6 @@ PA_API pa_status pa_decode_check(void* workspace, pa_stream_t stream) {
                        : r[0] == kSitePrefill  ? "multi-token (mma.sync) tile"
                        : r[0] == kSiteTcStep   ? "multi-token (tcgen05) step"
                        : r[0] == kSiteFp8Tile  ? "decode (tcgen05 FP8) tile"
-                       : r[0] == kSiteTmTile   ? "multi-token (tcgen05, keys on M) tile"
                                                : "unknown site";
     return fail(PA_ERR_CUDA,
                 "decode: a pipeline wait timed out; first failure: site %d (%s), CTA (%d, %d, "

@@ -25,11 +25,10 @@ enum : int32_t {
   kSitePrefill = 5,     // multi-token query on mma.sync: a tile or a stage release
                         //   (values: CTA x, y, z, warp or step, tile, tiles, 0 / 1 = producer)
   kSiteTcStep = 6,      // multi-token query on tcgen05: an MMA-warp wait
-                        //   (values: CTA x, y, z, K steps received, V steps received, steps, groups)
+                        //   (values: the CTA's unit - query tile + q_tiles * part, kv-head,
+                        //   sequence - then K steps received, V steps received, steps, groups)
   kSiteFp8Tile = 7,     // decode on tcgen05 (E4M3 cache): a role's wait
                         //   (values: kv-head, sequence, partition, role, tile, tiles)
-  kSiteTmTile = 8,      // multi-token query with the key tokens on M: a role's wait
-                        //   (values: CTA x, y, z, role, tile, tiles)
 };
 
 // Words of the workspace header (int32): the error word and, from kWordDiag,

@@ -112,6 +112,13 @@ __device__ __forceinline__ bool skip_for_test(int32_t skip_tile, int tile) {
          blockIdx.z == 0;
 }
 
+// The same for a kernel whose CTAs take their work units in another order
+// than their index: `first_unit` says whether this CTA runs the unit whose
+// coordinates are all 0.
+__device__ __forceinline__ bool skip_unit_for_test(int32_t skip_tile, int tile, bool first_unit) {
+  return skip_tile >= 0 && tile == skip_tile && first_unit;
+}
+
 // First failure of a launch: where it happened and the state there, written
 // once (words: site, then up to 7 values) to the diagnostic words.
 __device__ __forceinline__ void record_failure(int32_t* diag, int32_t site, int32_t v0,

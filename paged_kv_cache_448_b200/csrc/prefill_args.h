@@ -33,8 +33,9 @@ struct PrefillArgs {
   int32_t max_parts;
   float* ws_o;                   // [T * H][max_parts][D] partial outputs (normalised)
   float2* ws_ml;                 // [T * H][max_parts] (max, sum) in base-2 units
-  int32_t skip_tile;             // failure-detection test: 16-token tile of CTA (0,0,0)
-                                 // whose loads are left out; -1 none
+  int32_t skip_tile;             // failure-detection test: 16-token tile of the unit
+                                 // (query tile 0, kv-head 0, sequence 0) whose loads are
+                                 // left out; -1 none
   uint64_t wait_limit_ns;        // bound of every pipeline wait
 };
 

@@ -144,6 +144,32 @@ __device__ __forceinline__ float2 unpack_q(uint32_t w) {
   return __half22float2(h);
 }
 
+constexpr int kOrderSeqs = 256;  // launches of up to this many sequences are reordered
+
+// The sequence of rank `rank` when the sequences are ordered by context length,
+// longest first (ties by index): sequence i has rank #{j : len_j > len_i} +
+// #{j < i : len_j == len_i}, a permutation for any lengths. Launches of more
+// than kOrderSeqs sequences keep their order (rank = sequence). Every thread of
+// the CTA calls it (two barriers).
+__device__ __forceinline__ int sequence_of_rank(const int32_t* context_lens, int n, int rank,
+                                                int32_t* lens, int* pick) {
+  if (n > kOrderSeqs) return rank;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) lens[i] = context_lens[i];
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int32_t li = lens[i];
+    int r = 0;
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) {
+      const int32_t lj = lens[j];
+      r += (lj > li) | ((lj == li) & (j < i));
+    }
+    if (r == rank) *pick = i;
+  }
+  __syncthreads();
+  return *pick;
+}
+
 template <class QF, class CF, int D, int G, int NG>
 __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
     paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap kmap,
@@ -169,9 +195,9 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
       pv_bar[NG][2], drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int aborted;
+  __shared__ int32_t order_lens[kOrderSeqs];
+  __shared__ int order_pick;
 
-  const int z = blockIdx.x % a.q_tiles, part = blockIdx.x / a.q_tiles;
-  const int kvh = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint64_t lim = a.wait_limit_ns;
   if (tid == 0) {
@@ -196,6 +222,20 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
     prefetch_tensormap(&vmap);
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // This CTA's unit. CTAs are dispatched in the order of their linear index,
+  // and the units' work differs with the context length, so the launch takes
+  // the sequences longest context first and, within one, its last query tile
+  // (the most keys) first: list scheduling with the longest jobs first keeps
+  // the last wave short.
+  const int per_seq = static_cast<int>(gridDim.x * gridDim.y);
+  const int64_t lin = blockIdx.x + static_cast<int64_t>(gridDim.x) *
+                                       (blockIdx.y + static_cast<int64_t>(gridDim.y) * blockIdx.z);
+  const int rank = static_cast<int>(lin / per_seq), in_seq = static_cast<int>(lin % per_seq);
+  const int kvh = in_seq / static_cast<int>(gridDim.x), xi = in_seq % static_cast<int>(gridDim.x);
+  const int z = a.q_tiles - 1 - xi % a.q_tiles, part = xi / a.q_tiles;
+  const int s = sequence_of_rank(a.context_lens, a.num_seqs, rank, order_lens, &order_pick);
+  const bool first_unit = z == 0 && part == 0 && kvh == 0 && s == 0;
 
   const int q0 = a.cu_query_lens[s];
   const int qlen = a.cu_query_lens[s + 1] - q0;
@@ -328,7 +368,7 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
       issued = k + 1;
       const int t_begin = (kbase + k) * (NT / TR), t_end = min(tend, t_begin + NT / TR);
       if (!is_v && a.skip_tile >= t_begin - tbase && a.skip_tile < t_end - tbase &&
-          skip_for_test(a.skip_tile, a.skip_tile)) {
+          skip_unit_for_test(a.skip_tile, a.skip_tile, first_unit)) {
         bid = nbid;
         continue;  // (the K warp leaves it out: the step never completes)
       }
@@ -505,8 +545,8 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
       if (!ok) {
         // A wait gave up (never expected): let this CTA's MMAs finish (bounded)
         // before its tensor and shared memory go away.
-        record_failure(a.diag, kSiteTcStep, blockIdx.x, blockIdx.y, blockIdx.z, k_rel, v_rel,
-                       nsteps, NG);
+        record_failure(a.diag, kSiteTcStep, z + a.q_tiles * part, kvh, s, k_rel, v_rel, nsteps,
+                       NG);
         aborted = 1;
         report(a.err, kErrWaitTimeout);
         tc::commit(&drain_bar);
