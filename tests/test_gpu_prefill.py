@@ -137,6 +137,33 @@ def test_short_chunks_of_many_sequences_on_tcgen05(cache, G, q):
                  f"short chunks {cache} G{G} q{q}")
 
 
+@pytest.mark.parametrize("n,equal", [(256, False), (257, False), (300, True), (40, True)])
+def test_units_in_launch_order_cover_every_row(n, equal):
+    """The tcgen05 CTAs take their units longest context first (each CTA ranks
+    the sequences by context length) up to 256 sequences, in index order above.
+    Both sides of that bound, and contexts that all tie (ranks broken by
+    index), must still give every row exactly once: the output starts as NaN
+    and is compared whole. The 40-sequence case has 300-token chunks over two
+    row groups (three query tiles per sequence, the last one first)."""
+    rng = np.random.default_rng(90 + n)
+    if n == 40:
+        G, D = 2, 128
+        ctxs = np.full(n, 400)
+        qlens = rng.integers(1, 301, size=n)
+        qlens[0] = 300
+    else:
+        G, D = 8, 64
+        ctxs = np.full(n, 180) if equal else rng.integers(1, 300, size=n)
+        qlens = np.minimum(rng.integers(1, 9, size=n), ctxs)
+        qlens[0] = 8
+    sp, st, hd, qv, qlens = custom(list(ctxs), list(qlens), 2 * G, 2, D, 16, "f16",
+                                   seed=80 + n)
+    out, ws, cu = run_gpu(sp, st, hd, qv, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, qv, cu), "f16",
+                 f"launch order n{n} equal={equal}")
+
+
 @pytest.mark.parametrize("qdt,cache,G,D,bs,qlens", [
     ("bf16", "bf16", 8, 128, 16, [150, 129, 140]),   # two row groups (>= 256 rows)
     ("f16", "f16", 2, 128, 16, [200, 150, 131]),     # two groups, f16: rows held whole
