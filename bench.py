@@ -679,33 +679,34 @@ class E2EStep:
         self.down = torch.cuda.Stream(device=device)
         self.compute = torch.cuda.current_stream(device)
         ev = lambda: torch.cuda.Event()  # noqa: E731
-        self.uploaded, self.consumed, self.produced, self.read = (
-            [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()])
+        self.uploaded, self.done, self.read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
         self.run_step = run_step
         # the same per-step event pair around the decode as in the device-timed
         # loop, so that both loops carry the same instrumentation
         self.ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
         self.k = 0
         for b in range(2):  # every buffer starts free
-            self.consumed[b].record(self.compute)
+            self.done[b].record(self.compute)
             self.read[b].record(self.down)
 
     def __call__(self):
         import torch
         b = self.k & 1
         with torch.cuda.stream(self.up):
-            self.up.wait_event(self.consumed[b])          # the decode of step k-2 read it
+            # buffer pair b is free once the decode of step k-2 read its inputs
+            # and that step's output was read back; the upload stream takes
+            # both waits, so the decode waits for the upload alone
+            self.up.wait_event(self.done[b])
+            self.up.wait_event(self.read[b])
             self.dev_in[b].copy_(self.pin_in, non_blocking=True)
             self.uploaded[b].record(self.up)
         self.compute.wait_event(self.uploaded[b])
-        self.compute.wait_event(self.read[b])             # step k-2's output was read back
         v = self.views[b]
         self.run_step(v["query"], v["new_key"], v["new_value"], v["bt"], v["cl"], v["sl"],
                       self.out[b], self.ev)
-        self.consumed[b].record(self.compute)
-        self.produced[b].record(self.compute)
+        self.done[b].record(self.compute)
         with torch.cuda.stream(self.down):
-            self.down.wait_event(self.produced[b])
+            self.down.wait_event(self.done[b])
             self.pin_out[b].copy_(self.out[b], non_blocking=True)
             self.read[b].record(self.down)
         self.k += 1
