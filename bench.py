@@ -635,7 +635,9 @@ def decode_line(args, sp: wl.Spec, st: wl.Structure, world: int, step_ms: float,
                        "copies": "one packed host-to-device copy of the step's inputs and one "
                                  "device-to-host copy of its output per step, on an upload and a "
                                  "read-back stream, double-buffered so they overlap the "
-                                 "neighbouring steps"}
+                                 "neighbouring steps",
+                       "checked": "both read-back buffers equal the device-timed loop's "
+                                  "output bit for bit"}
     return line
 
 
@@ -824,6 +826,12 @@ def main():
         e2e = {"ms_per_step": a.elapsed_time(b) / e2e_steps, "h2d": e2e_step.h2d,
                "d2h": e2e_step.d2h}
         pk.decode_check(ws)
+        # both read-back buffers hold a step's output: the same inputs through
+        # the same kernels give the device-timed loop's output, bit for bit
+        ref = out.cpu().view(torch.int16)
+        for hb in e2e_step.pin_out:
+            if not torch.equal(hb.view(torch.int16), ref):
+                raise SystemExit("bench.py: an e2e read-back differs from the device-timed output")
 
     # max over ranks
     step_ms, dec_ms, e2e_ms = max_over_ranks(
