@@ -36,6 +36,9 @@ struct PrefillArgs {
   int32_t skip_tile;             // failure-detection test: 16-token tile of the unit
                                  // (query tile 0, kv-head 0, sequence 0) whose loads are
                                  // left out; -1 none
+  int32_t dup_rows;              // tcgen05 kernel, one row group, units of <= 64 rows:
+                                 // each row repeated 64 lanes further on (set by
+                                 // launch_prefill_tc)
   uint64_t wait_limit_ns;        // bound of every pipeline wait
 };
 

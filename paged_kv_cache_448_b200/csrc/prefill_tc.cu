@@ -247,15 +247,25 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
   const int tok0 = z * QT;
   if (tok0 >= qlen) return;  // ragged chunk lengths: nothing for this CTA
   const int ntok = min(QT, qlen - tok0);
-  // softmax threads: row tid of the CTA = token tid / G, head tid % G
-  const int tok = tid / G;
+  // One row group whose units hold at most 64 rows (short chunks, a few draft
+  // tokens): lanes 64..127 repeat rows 0..63, and the two copies of a row take
+  // the lower and the upper 32 tokens of every step, each with its own
+  // maximum, sum and O (rows of one MMA), merged at the end like two parts of
+  // a split key range. The tensor work is the same (the MMA has 128 rows
+  // either way); each softmax thread handles half as many tokens.
+  const bool dup = NG == 1 && a.dup_rows != 0;
+  const int half = dup ? tid / 64 : 0;  // softmax threads: which copy
+  // softmax threads: row srow of the unit = token srow / G, head srow % G
+  const int srow = dup ? (tid & 63) : tid;
+  const int tok = srow / G;
   const bool valid = warp < kMma && tok < ntok;
+  const bool out_row = valid && half == 0;  // the copy that writes the row's result
   const int64_t row_off =
-      (static_cast<int64_t>(q0 + tok0 + tok) * a.num_heads + kvh * G + tid % G) * D;
+      (static_cast<int64_t>(q0 + tok0 + tok) * a.num_heads + kvh * G + srow % G) * D;
   if (qlen > ctx) {  // a query longer than its context: rows become zeros
     if (part > 0) return;
     if (tid == 0 && z == 0 && kvh == 0) report(a.err, kErrQueryLonger);
-    if (valid) {
+    if (out_row) {
       uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
       for (int c = 0; c < D / 8; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
     }
@@ -624,6 +634,21 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
         for (int i = 8; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
         mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                      fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      } else if (dup) {
+        // this copy's 32 tokens of the step, masked after the row's position
+        tc::ld32(t_s + 32 * half, *reinterpret_cast<float(*)[32]>(x));
+        const int t0 = tk0 + 32 * half;
+        if (t0 + 31 > p_row) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = t0 + i <= p_row ? x[i] : -CUDART_INF_F;
+        }
+        float m8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m8[j] = x[j];
+#pragma unroll
+        for (int i = 8; i < 32; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+        mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       } else {
         // the row maximum of the step: with two halves the upper one is read
         // first for its maximum alone and read again after the lower one
@@ -678,6 +703,22 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
       if constexpr (kHoldAll) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) emit32(x + 32 * q, q / 2, q % 2);
+      } else if (dup) {
+        // this copy's quarter of P, and zeros where the other copy's tokens
+        // go (those are the other lane's, P of this lane has no weight there)
+        emit32(x, 0, half);
+        const uint32_t t_z = t_s + 32 * (1 - half);
+        if constexpr (FP8) {
+          const uint32_t zw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          tc::st8u(t_z, zw);
+          tc::st8u(t_z + 8, zw);
+        } else {
+          uint32_t zw[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) zw[i] = 0u;
+          tc::st16u(t_z, zw);
+          if constexpr (BF) tc::st16u(t_z + 16, zw);
+        }
       } else {
         emit32(x, 0, 0);
         emit32(x + 32, 0, 1);
@@ -739,11 +780,52 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
     }
     if (ok)
       ok = mbar_wait(&pv_bar[g][(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, lim, &aborted);
+    // two copies of a row: the upper copy hands (maximum, sum, O) to the lower
+    // through shared memory (Q's space, whose last reader, the last S, has
+    // completed), column-major so that a warp's accesses are conflict-free;
+    // every softmax thread reaches the barrier, also after a wait gave up
+    float fa = 1.f, fb = 0.f;  // weights of this lane's O and of the other copy's
+    const float* so = reinterpret_cast<const float*>(sq(0));
+    if constexpr (NG == 1) {
+      __shared__ float2 dup_ml[64];
+      static_assert(64 * D * 4 <= C::QG_BYTES, "O of 64 rows fits in Q's space");
+      float* sow = reinterpret_cast<float*>(sq(0));
+      if (dup) {
+        ok = __all_sync(0xffffffffu, ok);
+        if (half == 1) {
+          if (ok) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              float o[32];
+              tc::ld32(t_o + c * 32, o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) sow[(c * 32 + i) * 64 + srow] = o[i];
+            }
+          }
+          dup_ml[srow] = ok ? make_float2(m_used, l) : make_float2(-CUDART_INF_F, -1.f);
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (half == 0) {
+          const float2 t = dup_ml[srow];
+          if (t.y < 0.f) {
+            ok = false;  // the other copy gave up: the row's result is lost
+          } else if (ok && t.y > 0.f) {
+            const float mm = fmaxf(m_used, t.x);
+            fa = m_used == -CUDART_INF_F ? 0.f : tc::ex2(m_used - mm);
+            fb = tc::ex2(t.x - mm);
+            l = l * fa + t.y * fb;
+            m_used = mm;
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
+      }
+    }
     if (!ok) {
       // The row's result is lost: leave zeros (whole key range) or an empty
       // part that the combine kernel gives no weight, never stale data.
       aborted = 1;
-      if (valid) {
+      if (out_row) {
         if (parts == 1) {
           uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + row_off * 2);
           for (int c = 0; c < D / 8; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
@@ -763,7 +845,11 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
           tc::ld32(t_o + c * 32, o);
-          if (valid) {
+          if (dup && fb != 0.f) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = o[i] * fa + so[(c * 32 + i) * 64 + srow] * fb;
+          }
+          if (out_row) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               o4[c * 4 + q] = make_uint4(pack_pair(BF, o[8 * q] * inv, o[8 * q + 1] * inv),
@@ -774,13 +860,17 @@ __global__ void __launch_bounds__(NG * kTcRows + 96, NG == 1 ? 2 : 1)
         }
       } else {
         const int64_t prow = (row_off / D) * a.max_parts + part;
-        if (valid) a.ws_ml[prow] = make_float2(m_used, l);
+        if (out_row) a.ws_ml[prow] = make_float2(m_used, l);
         float4* w4 = reinterpret_cast<float4*>(a.ws_o + prow * D);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
           tc::ld32(t_o + c * 32, o);
-          if (valid) {
+          if (dup && fb != 0.f) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = o[i] * fa + so[(c * 32 + i) * 64 + srow] * fb;
+          }
+          if (out_row) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               w4[c * 8 + q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv,
@@ -810,9 +900,11 @@ cudaError_t launch_tc(const PrefillArgs& a, const CUtensorMap& kmap, const CUten
   if (e != cudaSuccess) return e;
   if (a.q_tiles != (max_query_len + C::QT - 1) / C::QT) return cudaErrorInvalidValue;
   if (a.max_parts > 1 && a.partition_tiles % (C::NT / kTileRows) != 0) return cudaErrorInvalidValue;
+  PrefillArgs b = a;
+  b.dup_rows = NG == 1 && static_cast<int64_t>(max_query_len) * G <= kTcRows / 2 ? 1 : 0;
   e = launch_pdl(kern, dim3(static_cast<unsigned>(a.q_tiles * a.max_parts), a.num_kv_heads,
                             a.num_seqs),
-                 NG * kTcRows + 96, smem, stream, a, kmap, vmap);
+                 NG * kTcRows + 96, smem, stream, b, kmap, vmap);
   if (e != cudaSuccess || a.max_parts <= 1) return e;
   return launch_prefill_combine(a, std::is_same<QF, BF16>::value ? kBF16 : kF16, D, C::QT,
                                 max_query_len, stream);

@@ -141,6 +141,38 @@ def test_multi_token_wait_that_runs_out(kernel, cache, D, site):
     assert_close(out.double().cpu().numpy(), ref, cache, "clean call after the timeout")
 
 
+@pytest.mark.parametrize("cache", ["bf16", "e4m3"])
+def test_short_chunks_on_tcgen05_wait_that_runs_out(cache):
+    """Short chunks of many sequences run on tcgen05 with each of their at
+    most 64 rows per unit held in two lanes, which take the two halves of
+    every step and are merged at the end through shared memory behind a
+    barrier of the softmax warps. A wait that runs out in the first unit must
+    still let every softmax warp reach that barrier: the unit's rows are
+    zeros, every other row matches the oracle, and the next call is clean."""
+    G = 4
+    rng = np.random.default_rng(81)
+    n = 150  # x 2 kv-heads: 300 units, enough to fill the tcgen05 kernel's wave
+    ctxs = rng.integers(100, 700, size=n)
+    ctxs[0] = 600
+    qlens = np.minimum(rng.integers(1, 9, size=n), ctxs)
+    qlens[0] = 8
+    sp, out, ws, call, ref = _prefill(list(ctxs), list(qlens), G, 128, "bf16", seed=83,
+                                      cache=None if cache == "bf16" else "e4m3")
+    pk.inject_wait_timeout(5, LIMIT_NS)  # tile 5 of sequence 0, kv-head 0
+    call()
+    _expect_timeout(lambda: pk.decode_check(ws), 6)
+    o = out.double().cpu().numpy()
+    assert np.isfinite(o).all()
+    lost = np.zeros(o.shape[:2], bool)
+    lost[:qlens[0], :G] = True  # the query tokens of sequence 0, heads of kv-head 0
+    assert (o[lost] == 0).all()
+    assert_close(o[~lost], ref[~lost], cache, "rows of the other units")
+    out.fill_(float("nan"))
+    call()
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), ref, cache, "clean call after the timeout")
+
+
 def test_injection_is_used_up_and_can_be_cancelled():
     g = _decode_step(4, "bf16", seed=70)
     g.reshape()
