@@ -28,6 +28,11 @@
 //    (16-row boxes of one 128-byte segment each, so a stage is
 //    [segment][step rows][128 B]), the boxes of a step from all lanes of the
 //    warp at once, and refill a stage when the MMAs that read it completed.
+// Units of at most 64 rows (a few draft tokens x the query group) hold each
+// row twice, in lanes r and r + 64: the two copies take the lower and upper
+// 32 tokens of every step with their own maximum, sum and O, and are merged
+// before the epilogue (the MMAs cost 128 rows either way; the softmax work
+// per thread halves).
 // The epilogue divides each row of O by its sum and stores it. When the key
 // range is split (few CTAs), a CTA takes one part of its 16-token tiles and
 // writes (max, sum) and its normalised O per row for the combine kernel, as
