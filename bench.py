@@ -21,7 +21,10 @@ table entries + context lengths) per step over the device time of the step.
 `--impl reference` times the CPU oracle (plain fp64 C) on the host cores
 instead, on a sample of the same workload sized so the run ends in minutes.
 
-The other rows of the path, one JSON line each:
+The other rows of the path, one JSON line each (a default run at one GPU
+also measures each of them, with fewer steps, in a child process of its own
+after the headline, and adds a summary of each under the line's "rows" key;
+--no-rows leaves them out):
     --op prefill --workload chunk_llama7b|chunk_gqa70b|verify_gqa70b|chunk_gqa70b_fp8
         multi-token query (TFLOP/s; against the tensor or HBM roofline,
         whichever the work per byte makes binding)
@@ -79,6 +82,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="leave out the other rows of the path (measured by default with "
+                         "the headline at one GPU, under the line's \"rows\" key)")
     return ap.parse_args()
 
 
@@ -560,6 +566,73 @@ def run_copy(args):
                       "clocks": clocks}), flush=True)
 
 
+# The other rows of the hot path: (name, arguments of this script). A default
+# run at one GPU measures each in a child process of its own after the
+# headline, with fewer steps, and reports a summary under "rows".
+ROWS = [
+    ("llama13b_mix", ["--config", "3", "--no-e2e"]),
+    ("gqa70b_long", ["--config", "4", "--no-e2e"]),
+    ("prefix_fp8", ["--config", "5", "--no-e2e"]),
+    ("chunk_llama7b", ["--op", "prefill", "--workload", "chunk_llama7b"]),
+    ("chunk_gqa70b", ["--op", "prefill", "--workload", "chunk_gqa70b"]),
+    ("verify_gqa70b", ["--op", "prefill", "--workload", "verify_gqa70b"]),
+    ("chunk_gqa70b_fp8", ["--op", "prefill", "--workload", "chunk_gqa70b_fp8"]),
+    ("copy_blocks", ["--op", "copy_blocks"]),
+    ("swap", ["--op", "swap"]),
+]
+ROW_STEPS, ROW_WARMUP = 500, 5
+
+
+def row_summary(name: str, line: dict) -> dict:
+    """The figures of a row's JSON line that the headline line carries."""
+    out = {"row": name}
+    for k in ("metric", "value", "unit", "ms_per_step", "dtype"):
+        if k in line:
+            out[k] = line[k]
+    roof = line.get("roofline") or {}
+    out["roofline"] = {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                            "traffic", "peak_kind") if k in roof}
+    clocks = line.get("clocks") or {}
+    out["clocks"] = {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons") if k in clocks}
+    return out
+
+
+def run_rows(rows=None, budget_s: float = 300.0, child_timeout_s: float = 150.0,
+             command=None) -> list:
+    """Each row measured by this script in a child process, one after the
+    other, so that a row's failure, hang or memory cannot reach the headline's
+    measurement or line: a row that fails or runs out of time is reported as
+    such. `command(args)` builds a child's command line."""
+    rows = ROWS if rows is None else rows
+    if command is None:
+        def command(extra):
+            return ([sys.executable, os.path.abspath(__file__), "--steps", str(ROW_STEPS),
+                     "--warmup", str(ROW_WARMUP), "--no-cpu-baseline", "--no-rows"] + extra)
+    out = []
+    t_end = time.time() + budget_s
+    for name, extra in rows:
+        left = t_end - time.time()
+        if left < 10:
+            out.append({"row": name, "skipped": "the time budget of the rows was spent"})
+            continue
+        try:
+            r = subprocess.run(command(extra), capture_output=True, text=True, cwd=ROOT,
+                               timeout=min(child_timeout_s, left))
+        except subprocess.TimeoutExpired:
+            out.append({"row": name, "error": "timed out"})
+            continue
+        lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+        if r.returncode != 0 or not lines:
+            tail = (r.stderr.strip().splitlines() or ["no output"])[-1][:200]
+            out.append({"row": name, "error": f"exit {r.returncode}: {tail}"})
+            continue
+        try:
+            out.append(row_summary(name, json.loads(lines[-1])))
+        except ValueError as e:
+            out.append({"row": name, "error": f"unreadable line: {e}"})
+    return out
+
+
 def relaunch_command(gpus: int, port: int, argv: list) -> list:
     """One process per GPU through torch.distributed.run on this node (the
     form the multi-GPU contract uses), bounded by `timeout` as the last
@@ -844,6 +917,8 @@ def main():
                            clocks, e2e)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(sp, args.cpu_seconds)
+        if world == 1 and args.config == 2 and args.partition < 0 and not args.no_rows:
+            line["rows"] = run_rows()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -191,3 +191,42 @@ def test_recorded_traffic_is_tied_to_the_sources():
             assert got == e["dram_bytes_per_launch"]
         else:
             assert got is None
+
+
+def test_rows_run_in_children_and_their_failures_stay_there():
+    """bench.py's other rows: each is measured in a child process; its last
+    JSON line is summarised, and a child that fails, prints no line or runs
+    out of time is reported as such instead of raising, so that the headline
+    line is printed whatever a row does. A spent time budget skips the rest."""
+    import json
+    import sys
+
+    import bench
+    line = {"metric": "m", "value": 1.5, "unit": "GB/s", "ms_per_step": 0.1, "dtype": "bf16",
+            "roofline": {"bound": "hbm", "achieved": 2.0, "peak": 4.0, "unit": "GB/s",
+                         "frac": 0.5, "traffic": None, "peak_kind": "measured", "kernel": "k"},
+            "clocks": {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3},
+            "config": {"workload": "w"}}
+    scripts = {
+        "ok": "print('log line'); print(" + repr(json.dumps(line)) + ")",
+        "fail": "import sys; print('boom', file=sys.stderr); sys.exit(3)",
+        "silent": "pass",
+        "slow": "import time; time.sleep(30)",
+    }
+    rows = [(k, [k]) for k in scripts]
+
+    def command(extra):
+        return [sys.executable, "-c", scripts[extra[0]]]
+
+    out = bench.run_rows(rows, budget_s=60, child_timeout_s=3, command=command)
+    assert out[0] == {"row": "ok", "metric": "m", "value": 1.5, "unit": "GB/s",
+                      "ms_per_step": 0.1, "dtype": "bf16",
+                      "roofline": {"bound": "hbm", "achieved": 2.0, "peak": 4.0, "unit": "GB/s",
+                                   "frac": 0.5, "traffic": None, "peak_kind": "measured"},
+                      "clocks": {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": []}}
+    assert out[1]["row"] == "fail" and out[1]["error"] == "exit 3: boom"
+    assert out[2]["row"] == "silent" and out[2]["error"].startswith("exit 0")
+    assert out[3] == {"row": "slow", "error": "timed out"}
+    skipped = bench.run_rows(rows[:2], budget_s=5, child_timeout_s=3, command=command)
+    assert [r.get("skipped") for r in skipped] == ["the time budget of the rows was spent"] * 2
+    assert [r[0] for r in bench.ROWS][:3] == ["llama13b_mix", "gqa70b_long", "prefix_fp8"]
