@@ -137,6 +137,33 @@ def test_short_chunks_of_many_sequences_on_tcgen05(cache, G, q):
                  f"short chunks {cache} G{G} q{q}")
 
 
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [1, 2])
+@pytest.mark.parametrize("D", [64, 128])
+def test_short_units_with_rows_held_twice(dt, G, D):
+    """Units of at most 64 rows on tcgen05 hold each row in two lanes, which
+    take the lower and the upper 32 tokens of every 64-token step and are
+    merged at the end. 150 sequences x 2 kv-heads fill the kernel's wave; the
+    chunks reach 64 rows per unit (64 / G tokens), and the contexts sit on
+    both sides of the half-step and step boundaries (a copy that sees no
+    token at all, a last step that one copy only reaches)."""
+    rng = np.random.default_rng(300 + 10 * G + D)
+    n = 150
+    qmax = 64 // G
+    ctxs = rng.integers(1, 400, size=n)
+    ctxs[:10] = [1, 31, 32, 33, 63, 64, 65, 95, 96, 97]
+    qlens = np.minimum(rng.integers(1, qmax + 1, size=n), ctxs)
+    qlens[6] = qmax  # contexts of 65 and 97 tokens: full-length chunks
+    qlens[9] = qmax
+    sp, st, hd, qv, qlens = custom(list(ctxs), list(qlens), 2 * G, 2, D, 16, dt,
+                                   seed=310 + 10 * G + D)
+    assert int(qlens.max()) * G == 64
+    out, ws, cu = run_gpu(sp, st, hd, qv, qlens)
+    pk.decode_check(ws)
+    assert_close(out.double().cpu().numpy(), run_oracle(sp, st, hd, qv, cu), dt,
+                 f"rows held twice {dt} G{G} D{D}")
+
+
 @pytest.mark.parametrize("n,equal", [(256, False), (257, False), (300, True), (40, True)])
 def test_units_in_launch_order_cover_every_row(n, equal):
     """The tcgen05 CTAs take their units longest context first (each CTA ranks
